@@ -1,0 +1,191 @@
+"""Seeded synthetic inputs shared by the oracle tests, the GPU tests and the bench.
+
+This module draws random numbers and lays out camera rigs. It holds none of
+the view transform's arithmetic (no projection, no validity test, no
+sampling) and imports nothing else from this package, so that the oracle
+and the CUDA path can both consume identical bytes without sharing code.
+
+Workloads (shapes after the LSS tutorial's worked sizes, "Lift" section:
+128x352 images at stride 16 give an 8x22 feature map; "Splat" section: a
+-50..50 m BEV at 0.5 m per cell gives 200x200):
+
+  tiny        B1 N6 C16  8x22  (img 128x352)   50x50x4   over +-25 m  fp32
+  nuscenes    B1 N6 C64  16x44 (img 256x704)   200x200x8 over +-50 m  fp32
+  batched     B4 N6 C128 32x88 (img 512x1408)  200x200x16 over +-50 m bf16
+  large       B1 N6 C80  32x88 (img 512x1408)  400x400x16 over +-50 m fp32
+  backward    nuscenes shapes with B2, upstream gradient N(0,1)
+
+z always spans [-5, 3] m.  Rig: camera n has nominal yaw 60 deg * n, sits at
+(cos yaw, sin yaw, 1.5) m plus U(-0.05, 0.05) m jitter per axis, and looks
+horizontally along yaw + U(-2, 2) deg with no pitch or roll.  Ego frame:
+x forward, y left, z up.  Camera frame: x right, y down, z forward.  The
+extrinsic maps ego to camera (SparseDriveV2 notes, "Deformable Aggregation"
+pitfalls: the extrinsic takes ego coordinates into the camera frame).
+Pinhole intrinsics fx = fy = 0.7 * W_img, cx = W_img / 2, cy = H_img / 2.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    index: int            # seed family
+    B: int
+    N: int
+    C: int
+    Hf: int
+    Wf: int
+    img_h: int
+    img_w: int
+    X: int
+    Y: int
+    Z: int
+    xr: tuple
+    yr: tuple
+    zr: tuple
+    dtype: str            # "f32" or "bf16" feature storage
+    backward: bool = False
+
+    @property
+    def ranges(self):
+        return (self.xr[0], self.xr[1], self.yr[0], self.yr[1], self.zr[0], self.zr[1])
+
+    @property
+    def res(self):
+        """Cell sizes that reproduce the stated counts (extent / count)."""
+        return ((self.xr[1] - self.xr[0]) / self.X,
+                (self.yr[1] - self.yr[0]) / self.Y,
+                (self.zr[1] - self.zr[0]) / self.Z)
+
+    @property
+    def out_elems(self):
+        return self.B * self.C * self.X * self.Y
+
+    def scaled(self, **kw):
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 0, 1, 6, 16, 8, 22, 128, 352, 50, 50, 4,
+                     (-25.0, 25.0), (-25.0, 25.0), (-5.0, 3.0), "f32"),
+    "nuscenes": Workload("nuscenes", 1, 1, 6, 64, 16, 44, 256, 704, 200, 200, 8,
+                         (-50.0, 50.0), (-50.0, 50.0), (-5.0, 3.0), "f32"),
+    "batched_bf16": Workload("batched_bf16", 2, 4, 6, 128, 32, 88, 512, 1408, 200, 200, 16,
+                             (-50.0, 50.0), (-50.0, 50.0), (-5.0, 3.0), "bf16"),
+    "large": Workload("large", 3, 1, 6, 80, 32, 88, 512, 1408, 400, 400, 16,
+                      (-50.0, 50.0), (-50.0, 50.0), (-5.0, 3.0), "f32"),
+    "backward": Workload("backward", 4, 2, 6, 64, 16, 44, 256, 704, 200, 200, 8,
+                         (-50.0, 50.0), (-50.0, 50.0), (-5.0, 3.0), "f32", backward=True),
+}
+
+
+def pinhole_intrinsics(img_h: int, img_w: int) -> np.ndarray:
+    f = 0.7 * img_w
+    return np.array([[f, 0.0, img_w / 2.0], [0.0, f, img_h / 2.0], [0.0, 0.0, 1.0]])
+
+
+def camera_extrinsic(yaw: float, pos) -> np.ndarray:
+    """Ego-to-camera 4x4 for a level camera looking along ``yaw`` from ``pos``.
+
+    Rows of R are the camera axes written in ego coordinates:
+    x_c = (sin yaw, -cos yaw, 0), y_c = (0, 0, -1), z_c = (cos yaw, sin yaw, 0);
+    E = [R | -R pos; 0 0 0 1].  Built in float64.
+    """
+    R = np.array([[math.sin(yaw), -math.cos(yaw), 0.0],
+                  [0.0, 0.0, -1.0],
+                  [math.cos(yaw), math.sin(yaw), 0.0]])
+    E = np.eye(4)
+    E[:3, :3] = R
+    E[:3, 3] = -R @ np.asarray(pos, dtype=np.float64)
+    return E
+
+
+def make_rig(seed: int, N: int, img_h: int, img_w: int, jitter: bool = True):
+    """Return (K [N,3,3], E [N,4,4]) as float32 arrays for one batch item.
+
+    Per camera, in order, the generator draws the yaw jitter and then the
+    three position jitters.
+    """
+    rng = np.random.default_rng(seed)
+    K = np.empty((N, 3, 3))
+    E = np.empty((N, 4, 4))
+    for n in range(N):
+        yaw0 = math.radians(60.0 * n)
+        dyaw = rng.uniform(-2.0, 2.0) if jitter else 0.0
+        dpos = rng.uniform(-0.05, 0.05, size=3) if jitter else np.zeros(3)
+        pos = np.array([math.cos(yaw0), math.sin(yaw0), 1.5]) + dpos
+        K[n] = pinhole_intrinsics(img_h, img_w)
+        E[n] = camera_extrinsic(yaw0 + math.radians(dyaw), pos)
+    return K.astype(np.float32), E.astype(np.float32)
+
+
+def rig_seed(w: Workload, b: int, shard: int = 0) -> int:
+    return 2000 + 16 * w.index + b + 100003 * shard
+
+
+def make_rigs(w: Workload, shard: int = 0):
+    """Calibrations for every batch item: (K [B,N,3,3], E [B,N,4,4]) float32 torch (CPU)."""
+    Ks, Es = [], []
+    for b in range(w.B):
+        K, E = make_rig(rig_seed(w, b, shard), w.N, w.img_h, w.img_w)
+        Ks.append(K)
+        Es.append(E)
+    return torch.from_numpy(np.stack(Ks)), torch.from_numpy(np.stack(Es))
+
+
+def make_features(w: Workload, shard: int = 0, layout: str = "nchw") -> torch.Tensor:
+    """i.i.d. N(0,1) features [B,N,C,Hf,Wf] (or [B,N,Hf,Wf,C] for ``nhwc``) on CPU.
+
+    bf16 workloads round the float32 draw to nearest-even.
+    """
+    g = torch.Generator().manual_seed(1000 + w.index + 100003 * shard)
+    f = torch.randn((w.B, w.N, w.C, w.Hf, w.Wf), generator=g, dtype=torch.float32)
+    if w.dtype == "bf16":
+        f = f.to(torch.bfloat16)
+    if layout == "nhwc":
+        f = f.permute(0, 1, 3, 4, 2).contiguous()
+    return f
+
+
+def make_dout(w: Workload, shard: int = 0) -> torch.Tensor:
+    """Upstream gradient [B,C,X,Y] float32, i.i.d. N(0,1)."""
+    g = torch.Generator().manual_seed(3000 + w.index + 100003 * shard)
+    return torch.randn((w.B, w.C, w.X, w.Y), generator=g, dtype=torch.float32)
+
+
+def random_rig(seed: int, N: int, img_h: int, img_w: int, height=(0.5, 2.5), spread=1.0):
+    """A looser rig for property tests: random yaw, small pitch and roll, random mount.
+
+    Cameras get yaw U(0, 360) deg, pitch and roll U(-8, 8) deg, position within
+    ``spread`` m of the origin at a random height, and intrinsics with unequal
+    focal lengths, skew 0 and a principal point off centre.  Float32 output.
+    """
+    rng = np.random.default_rng(seed)
+    K = np.empty((N, 3, 3))
+    E = np.empty((N, 4, 4))
+    for n in range(N):
+        yaw = rng.uniform(0, 2 * math.pi)
+        pitch = math.radians(rng.uniform(-8, 8))
+        roll = math.radians(rng.uniform(-8, 8))
+        pos = np.array([rng.uniform(-spread, spread), rng.uniform(-spread, spread),
+                        rng.uniform(*height)])
+        base = camera_extrinsic(yaw, np.zeros(3))[:3, :3]
+        cp, sp, cr, sr = math.cos(pitch), math.sin(pitch), math.cos(roll), math.sin(roll)
+        Rx = np.array([[1, 0, 0], [0, cp, -sp], [0, sp, cp]])
+        Rz = np.array([[cr, -sr, 0], [sr, cr, 0], [0, 0, 1]])
+        R = Rz @ Rx @ base
+        E[n] = np.eye(4)
+        E[n, :3, :3] = R
+        E[n, :3, 3] = -R @ pos
+        fx = rng.uniform(0.5, 0.9) * img_w
+        fy = fx * rng.uniform(0.9, 1.1)
+        K[n] = np.array([[fx, 0.0, img_w * rng.uniform(0.4, 0.6)],
+                         [0.0, fy, img_h * rng.uniform(0.4, 0.6)],
+                         [0.0, 0.0, 1.0]])
+    return K.astype(np.float32), E.astype(np.float32)

@@ -1,0 +1,146 @@
+"""Python front of the CPU oracle (``bev_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the bench's
+CPU-baseline leg are the only callers.  The product path (the CUDA library and
+its binding) never imports this package.
+
+The oracle is the plain definition of the exact dense Sampling-VT written as a
+loop nest (FlashBEV reading notes, "Method" items 1 and 4): per height bin the
+mean over valid cameras of the bilinear samples, summed over height.  See the
+header comment of ``bev_oracle.c`` for every reading it takes.
+
+Pins (in ``tests/test_oracle.py``): a materialised tensorized evaluation with
+``torch.nn.functional.grid_sample`` on tiny grids, a hand-derived worked example
+(``tests/golden/``), affine and constant feature closed forms, camera
+permutation, duplicate-camera and per-bin decompositions, linearity, the
+adjoint identity and finite differences for the backward.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bev_oracle.c")
+_LIB = os.path.join(_HERE, "libbevoracle.so")
+_lib = None
+
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+          "-fno-fast-math", "-msse2", "-mfpmath=sse", "-Wall"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (fp contraction off, SSE float math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        F = ctypes.c_float
+        lib.oracle_grid_spec.argtypes = [P, P, P, P]
+        lib.oracle_grid_spec.restype = I
+        lib.oracle_project.argtypes = [P, P, F, F, F, I, I, I, I, P, P, P, P]
+        lib.oracle_project.restype = I
+        lib.oracle_forward.argtypes = [P, I, I, I, I, I, P, P, I, I, I, I, I, P, P, P, P, P, I]
+        lib.oracle_forward.restype = None
+        lib.oracle_backward.argtypes = [P, I, I, I, I, I, P, P, I, I, I, I, I, P, P, P, P, I]
+        lib.oracle_backward.restype = None
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _np(x, dtype):
+    """Contiguous numpy copy; torch tensors (any dtype, incl. bf16) widen exactly."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu()
+            if dtype == np.float64:
+                x = x.double()
+            elif dtype == np.float32:
+                x = x.float()
+            x = x.numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=dtype))
+
+
+class Grid:
+    """Counts and fp32 cell sizes from ranges and resolutions (oracle's own)."""
+
+    def __init__(self, ranges, res):
+        r = np.asarray(ranges, dtype=np.float32)
+        s = np.asarray(res, dtype=np.float32)
+        counts = np.zeros(3, dtype=np.int32)
+        cell = np.zeros(3, dtype=np.float32)
+        if _load().oracle_grid_spec(_ptr(r), _ptr(s), _ptr(counts), _ptr(cell)) != 0:
+            raise ValueError(f"grid ranges {ranges} / resolution {res} do not give integral counts")
+        self.X, self.Y, self.Z = (int(v) for v in counts)
+        self.lo = np.array([r[0], r[2], r[4]], dtype=np.float32)
+        self.cell = cell
+
+    def centres(self, axis: int) -> np.ndarray:
+        n = (self.X, self.Y, self.Z)[axis]
+        return (self.lo[axis] + ((np.arange(n, dtype=np.float32) + np.float32(0.5))
+                                 * self.cell[axis]).astype(np.float32)).astype(np.float32)
+
+
+def project(K, E, p, img_h, img_w, Hf, Wf):
+    """Single point through single camera: (valid, u, v, fx, fy)."""
+    K = _np(K, np.float32).reshape(9)
+    E = _np(E, np.float32).reshape(16)
+    u, v, fx, fy = (np.zeros(1, dtype=np.float32) for _ in range(4))
+    ok = _load().oracle_project(_ptr(K), _ptr(E), float(np.float32(p[0])), float(np.float32(p[1])),
+                                float(np.float32(p[2])), img_h, img_w, Hf, Wf,
+                                _ptr(u), _ptr(v), _ptr(fx), _ptr(fy))
+    out = [u[0], v[0], fx[0], fy[0]]
+    return bool(ok), float(out[0]), float(out[1]), float(out[2]), float(out[3])
+
+
+def forward(features, K, E, img_h, img_w, grid: Grid, threads: int = 0):
+    """Returns (out [B,C,X,Y] f64, bound [B,C,X,Y] f64, count [B,X,Y,Z] int32).
+
+    ``features`` is [B,N,C,Hf,Wf] (fp32 or bf16; widened exactly to fp64).
+    ``threads`` = OpenMP threads (0: the runtime default).
+    """
+    F = _np(features, np.float64)
+    B, N, C, Hf, Wf = F.shape
+    Kc = _np(K, np.float32).reshape(B, N, 3, 3)
+    Ec = _np(E, np.float32).reshape(B, N, 4, 4)
+    out = np.zeros((B, C, grid.X, grid.Y), dtype=np.float64)
+    bound = np.zeros_like(out)
+    count = np.zeros((B, grid.X, grid.Y, grid.Z), dtype=np.int32)
+    _load().oracle_forward(_ptr(F), B, N, C, Hf, Wf, _ptr(Kc), _ptr(Ec), img_h, img_w,
+                           grid.X, grid.Y, grid.Z, _ptr(grid.lo), _ptr(grid.cell),
+                           _ptr(out), _ptr(bound), _ptr(count), threads)
+    return out, bound, count
+
+
+def backward(dout, N, Hf, Wf, K, E, img_h, img_w, grid: Grid, threads: int = 0):
+    """Returns (dF [B,N,C,Hf,Wf] f64, bound [B,N,C,Hf,Wf] f64) for dout [B,C,X,Y]."""
+    G = _np(dout, np.float64)
+    B, C, X, Y = G.shape
+    assert (X, Y) == (grid.X, grid.Y)
+    Kc = _np(K, np.float32).reshape(B, N, 3, 3)
+    Ec = _np(E, np.float32).reshape(B, N, 4, 4)
+    dF = np.zeros((B, N, C, Hf, Wf), dtype=np.float64)
+    dB = np.zeros_like(dF)
+    _load().oracle_backward(_ptr(G), B, N, C, Hf, Wf, _ptr(Kc), _ptr(Ec), img_h, img_w,
+                            grid.X, grid.Y, grid.Z, _ptr(grid.lo), _ptr(grid.cell),
+                            _ptr(dF), _ptr(dB), threads)
+    return dF, dB

@@ -1,0 +1,258 @@
+/*
+ * bev_oracle.c -- CPU oracle for the exact dense Sampling-VT gather-reduction.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links or calls this
+ * file; only the tests, the smoke check and the bench's CPU-baseline leg do.
+ * It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (FlashBEV reading notes, "Core Idea" and "Method" item 1):
+ * for every BEV output element (b, c, i, j) and every height bin k, each camera
+ * n projects the voxel centre, the valid cameras' bilinear samples are averaged
+ * ("valid mean" per height bin), and the per-bin means are summed over height
+ * (the notes' "Key Insight": a height sum, not a learned height reduction).
+ *
+ *   voxel centre      x_i = xmin + (i + 0.5) dx  (same for y_j, z_k)
+ *   projection        [u v 1]^T ~ K (R p + t)    (SparseDriveV2 notes,
+ *                     "Deformable Aggregation", step 2; E = [R|t] maps ego to
+ *                     camera, per the same section's pitfalls)
+ *   validity          depth = camera z > 0.1 and (u, v) in [0, W_img] x [0, H_img]
+ *                     (same step: the projection must land inside the image)
+ *   sampling          bilinear, align_corners=False, zero padding:
+ *                     fx = u * Wf / W_img - 0.5, fy = v * Hf / H_img - 0.5
+ *                     (same section's pitfalls: bilinear, so gradients flow)
+ *   reduction         out = sum_k [cnt_k > 0] (1 / cnt_k) sum_{n valid} sample_n
+ *
+ * Precision.  Geometry follows one fixed fp32 expression order, every product
+ * and sum rounded on its own (this file must be compiled with
+ * -ffp-contract=off and SSE float arithmetic), so that the validity counts --
+ * integers decided by floating point -- come out identical on any IEEE
+ * machine that evaluates the same expression:
+ *   pc_r = ((E_r0 x + E_r1 y) + E_r2 z) + E_r3
+ *   uh   = (K_00 pc_x + K_01 pc_y) + K_02 pc_z,   u = uh / pc_z   (IEEE divide)
+ *   fx   = u * (Wf / W_img) - 0.5,  x0 = floor(fx), wx1 = fx - x0, wx0 = 1 - wx1
+ *   corner weight w = wy * wx
+ * Accumulation of features times weights is done in fp64.  Alongside each
+ * result the oracle returns a condition bound: the same sum taken over
+ * absolute values of the terms, which scales the parity tolerance.
+ *
+ * Where the notes are silent this oracle takes these readings: the image test
+ * is closed on both ends; a camera that passes the test counts towards the
+ * mean even if some bilinear corners fall outside the feature map (those
+ * corners contribute zero); an empty height bin contributes zero; K's last row
+ * is taken to be [0 0 1] and E's bottom row is ignored.
+ *
+ * Backward: the operator is linear in the features, so dL/dF is the adjoint:
+ *   dF[b,n,c,y,x] += w * dout[b,c,i,j] / cnt_k  over every valid sample and
+ *   in-range corner (y, x) it touches.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Grid from ranges and resolutions.  counts = round(extent / res) when that
+ * ratio is within 1e-4 of an integer, else failure; the cell size used for
+ * the centres is recomputed as extent / count in fp32.  Returns 0 on success. */
+int oracle_grid_spec(const float range[6], const float res[3], int counts[3], float cell[3])
+{
+    for (int a = 0; a < 3; ++a) {
+        float lo = range[2 * a], hi = range[2 * a + 1];
+        if (!(isfinite(lo) && isfinite(hi) && isfinite(res[a]))) return 1;
+        if (!(hi > lo) || !(res[a] > 0.0f)) return 1;
+        float extent = hi - lo;
+        double ratio = (double)extent / (double)res[a];
+        double nearest = floor(ratio + 0.5);
+        if (fabs(ratio - nearest) > 1e-4 || nearest < 1.0 || nearest > 1e6) return 1;
+        counts[a] = (int)nearest;
+        cell[a] = extent / (float)counts[a];
+    }
+    return 0;
+}
+
+/* Voxel centre along one axis, fp32: lo + ((float)i + 0.5f) * d. */
+static float centre(float lo, int i, float d)
+{
+    float t = (float)i + 0.5f;
+    t = t * d;
+    return lo + t;
+}
+
+/* Project one ego point through one camera.  Returns 1 when valid and writes
+ * the feature-map sampling position (fx, fy) and the image position (u, v). */
+int oracle_project(const float* K, const float* E, float px, float py, float pz,
+                   int img_h, int img_w, int Hf, int Wf,
+                   float* u_out, float* v_out, float* fx_out, float* fy_out)
+{
+    float pc[3];
+    for (int r = 0; r < 3; ++r) {
+        float t = E[4 * r + 0] * px;
+        float s = E[4 * r + 1] * py;
+        t = t + s;
+        s = E[4 * r + 2] * pz;
+        t = t + s;
+        t = t + E[4 * r + 3];
+        pc[r] = t;
+    }
+    float depth = pc[2];
+    if (!(depth > 0.1f)) return 0;
+    float uh = K[0] * pc[0];
+    float s = K[1] * pc[1];
+    uh = uh + s;
+    s = K[2] * pc[2];
+    uh = uh + s;
+    float vh = K[3] * pc[0];
+    s = K[4] * pc[1];
+    vh = vh + s;
+    s = K[5] * pc[2];
+    vh = vh + s;
+    float u = uh / depth;
+    float v = vh / depth;
+    *u_out = u;
+    *v_out = v;
+    if (!(u >= 0.0f && u <= (float)img_w && v >= 0.0f && v <= (float)img_h)) return 0;
+    float sW = (float)Wf / (float)img_w;
+    float sH = (float)Hf / (float)img_h;
+    float fx = u * sW;
+    fx = fx - 0.5f;
+    float fy = v * sH;
+    fy = fy - 0.5f;
+    *fx_out = fx;
+    *fy_out = fy;
+    return 1;
+}
+
+/* The four bilinear corners of (fx, fy): feature-map row/col and weight. */
+static void corners(float fx, float fy, int ys[4], int xs[4], float ws[4])
+{
+    float x0f = floorf(fx), y0f = floorf(fy);
+    float wx1 = fx - x0f, wy1 = fy - y0f;
+    float wx0 = 1.0f - wx1, wy0 = 1.0f - wy1;
+    int x0 = (int)x0f, y0 = (int)y0f;
+    ys[0] = y0;     xs[0] = x0;     ws[0] = wy0 * wx0;
+    ys[1] = y0;     xs[1] = x0 + 1; ws[1] = wy0 * wx1;
+    ys[2] = y0 + 1; xs[2] = x0;     ws[2] = wy1 * wx0;
+    ys[3] = y0 + 1; xs[3] = x0 + 1; ws[3] = wy1 * wx1;
+}
+
+/* Forward.  features [B,N,C,Hf,Wf] fp64 (exact copies of the fp32/bf16
+ * inputs); K [B,N,3,3], E [B,N,4,4] fp32; counts X,Y,Z; lo = (xmin,ymin,zmin);
+ * cell = (dx,dy,dz).  Writes out and bound [B,C,X,Y] fp64 and count
+ * [B,X,Y,Z] int32.  Rows (b, i) are independent and may run on `threads`
+ * OpenMP threads; each output element's arithmetic is unchanged by that. */
+void oracle_forward(const double* F, int B, int N, int C, int Hf, int Wf,
+                    const float* K, const float* E, int img_h, int img_w,
+                    int X, int Y, int Z, const float lo[3], const float cell[3],
+                    double* out, double* bound, int32_t* count, int threads)
+{
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic)
+#endif
+    for (long bi = 0; bi < (long)B * X; ++bi) {
+        int b = (int)(bi / X), i = (int)(bi % X);
+        double* acc = (double*)malloc(sizeof(double) * 4 * (size_t)C);
+        double* abs_acc = acc + C;
+        double* s = acc + 2 * C;
+        double* a = acc + 3 * C;
+        float x = centre(lo[0], i, cell[0]);
+        for (int j = 0; j < Y; ++j) {
+            float y = centre(lo[1], j, cell[1]);
+            for (int c = 0; c < C; ++c) { acc[c] = 0.0; abs_acc[c] = 0.0; }
+            for (int k = 0; k < Z; ++k) {
+                float z = centre(lo[2], k, cell[2]);
+                for (int c = 0; c < C; ++c) { s[c] = 0.0; a[c] = 0.0; }
+                int cnt = 0;
+                for (int n = 0; n < N; ++n) {
+                    const float* Kn = K + ((size_t)b * N + n) * 9;
+                    const float* En = E + ((size_t)b * N + n) * 16;
+                    float u, v, fx, fy;
+                    if (!oracle_project(Kn, En, x, y, z, img_h, img_w, Hf, Wf, &u, &v, &fx, &fy))
+                        continue;
+                    ++cnt;
+                    int ys[4], xs[4];
+                    float ws[4];
+                    corners(fx, fy, ys, xs, ws);
+                    for (int q = 0; q < 4; ++q) {
+                        if (ys[q] < 0 || ys[q] >= Hf || xs[q] < 0 || xs[q] >= Wf) continue;
+                        const double* Fp = F + (((size_t)b * N + n) * C * Hf + ys[q]) * Wf + xs[q];
+                        for (int c = 0; c < C; ++c) {
+                            double term = (double)ws[q] * Fp[(size_t)c * Hf * Wf];
+                            s[c] += term;
+                            a[c] += fabs(term);
+                        }
+                    }
+                }
+                count[(((size_t)b * X + i) * Y + j) * Z + k] = cnt;
+                if (cnt > 0) {
+                    for (int c = 0; c < C; ++c) {
+                        acc[c] += s[c] / cnt;
+                        abs_acc[c] += a[c] / cnt;
+                    }
+                }
+            }
+            for (int c = 0; c < C; ++c) {
+                size_t o = (((size_t)b * C + c) * X + i) * Y + j;
+                out[o] = acc[c];
+                bound[o] = abs_acc[c];
+            }
+        }
+        free(acc);
+    }
+}
+
+/* Backward (gradient with respect to the features only).  dout [B,C,X,Y]
+ * fp64.  Writes dF and dbound [B,N,C,Hf,Wf] fp64 (overwritten).  Work is split
+ * over (b, n) pairs so that each thread owns its slice of dF. */
+void oracle_backward(const double* dout, int B, int N, int C, int Hf, int Wf,
+                     const float* K, const float* E, int img_h, int img_w,
+                     int X, int Y, int Z, const float lo[3], const float cell[3],
+                     double* dF, double* dbound, int threads)
+{
+    memset(dF, 0, sizeof(double) * (size_t)B * N * C * Hf * Wf);
+    memset(dbound, 0, sizeof(double) * (size_t)B * N * C * Hf * Wf);
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic)
+#endif
+    for (long bn = 0; bn < (long)B * N; ++bn) {
+        int b = (int)(bn / N), n = (int)(bn % N);
+        const float* Kn = K + ((size_t)b * N + n) * 9;
+        const float* En = E + ((size_t)b * N + n) * 16;
+        double* dFn = dF + ((size_t)b * N + n) * C * Hf * Wf;
+        double* dBn = dbound + ((size_t)b * N + n) * C * Hf * Wf;
+        for (int i = 0; i < X; ++i) {
+            float x = centre(lo[0], i, cell[0]);
+            for (int j = 0; j < Y; ++j) {
+                float y = centre(lo[1], j, cell[1]);
+                for (int k = 0; k < Z; ++k) {
+                    float z = centre(lo[2], k, cell[2]);
+                    float u, v, fx, fy;
+                    int cnt = 0;
+                    for (int m = 0; m < N; ++m) {
+                        const float* Km = K + ((size_t)b * N + m) * 9;
+                        const float* Em = E + ((size_t)b * N + m) * 16;
+                        cnt += oracle_project(Km, Em, x, y, z, img_h, img_w, Hf, Wf, &u, &v, &fx, &fy);
+                    }
+                    if (!oracle_project(Kn, En, x, y, z, img_h, img_w, Hf, Wf, &u, &v, &fx, &fy))
+                        continue;
+                    int ys[4], xs[4];
+                    float ws[4];
+                    corners(fx, fy, ys, xs, ws);
+                    for (int q = 0; q < 4; ++q) {
+                        if (ys[q] < 0 || ys[q] >= Hf || xs[q] < 0 || xs[q] >= Wf) continue;
+                        for (int c = 0; c < C; ++c) {
+                            double g = dout[(((size_t)b * C + c) * X + i) * Y + j];
+                            double term = (double)ws[q] * g / cnt;
+                            size_t o = ((size_t)c * Hf + ys[q]) * Wf + xs[q];
+                            dFn[o] += term;
+                            dBn[o] += fabs(term);
+                        }
+                    }
+                }
+            }
+        }
+    }
+}
