@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark of the exact dense Sampling-VT on B200.
+
+One step = the whole hot path over one batch: channels-last copy of the
+features, fused forward gather-reduction, and the feature gradient (zero-init,
+scatter, layout back), on the nuScenes-like workload (B1, 6 cameras, C64,
+16x44 features from 256x704 images, BEV 200x200x8 over +-50 m, fp32).
+
+Timing: inputs resident in HBM; L2 flushed (256 MiB write) before every timed
+step; each stage captured once as a CUDA graph and replayed between CUDA
+events on the launching stream; W warm-up steps, then K timed steps between a
+barrier and a device synchronize; the max over ranks is reported.  SM clocks
+and throttle reasons are sampled through NVML during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank transforms its own batch (independent
+calibrations and features); there is no exchange step, so no collective is
+used on the data path ("scaling": "weak").
+
+--impl reference times the CPU oracle (oracle/, plain C loop nest in fp64) on
+the host cores, on a band of BEV rows per step, and prints the same JSON line
+with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BEV output elements/s (B·C·X·Y) and achieved HBM GB/s vs roofline, 1×B200"
+UNIT = "elements/s"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="nuscenes")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def workload_desc(w):
+    return (f"{w.name}: B{w.B} N{w.N} C{w.C} {w.Hf}x{w.Wf} features (img {w.img_h}x{w.img_w}) -> "
+            f"BEV {w.X}x{w.Y}x{w.Z} over x[{w.xr[0]},{w.xr[1]}] y[{w.yr[0]},{w.yr[1]}] "
+            f"z[{w.zr[0]},{w.zr[1]}] m, {w.dtype} features, forward + feature gradient")
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        v = float(json.load(open(p))["hbm_gbs"])
+        return v, "measured (STREAM-style copy on this pool's B200)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (earlier measurement on this pool)"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "camera_bev_view_b200", "csrc", "*"))):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(p))
+        ent = rec[kernel][workload]
+        if ent.get("source_digest") == source_digest():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """NVML sampling of the SM clock and clock-event reasons."""
+
+    BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.err = [], set(), None
+        self.stop_ev = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = f"nvml unavailable: {e}"
+            self.h = None
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = int(self.get_reasons(self.h))
+                for b, name in self.BITS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception as e:  # pragma: no cover
+                self.err = str(e)
+                return
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.h is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.h is not None:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if self.h is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err or "no samples"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step_sample(w, rows, threads):
+    """One oracle forward + backward over BEV rows [i0, i0 + rows) of the
+    workload (same calibrations and features); returns (seconds, elements)."""
+    import oracle
+    from camera_bev_view_b200 import inputs as I
+    F = I.make_features(w)
+    K, E = I.make_rigs(w)
+    dout = I.make_dout(w)
+    dx = (w.xr[1] - w.xr[0]) / w.X
+    i0 = max(0, w.X // 2 - rows // 2)
+    rng = (w.xr[0] + i0 * dx, w.xr[0] + (i0 + rows) * dx) + w.ranges[2:]
+    grid = oracle.Grid(rng, w.res)
+    d = dout[:, :, i0:i0 + rows].contiguous()
+    t0 = time.perf_counter()
+    oracle.forward(F, K, E, w.img_h, w.img_w, grid, threads=threads)
+    oracle.backward(d, w.N, w.Hf, w.Wf, K, E, w.img_h, w.img_w, grid, threads=threads)
+    return time.perf_counter() - t0, w.B * w.C * rows * w.Y
+
+
+def cpu_baseline(w, seconds):
+    """The oracle as it stands, on the host cores, whole workload steps until
+    `seconds` of CPU work (at least one step)."""
+    threads = cpu_cores()
+    spent, elems, steps = 0.0, 0, 0
+    while steps == 0 or spent < seconds:
+        t, e = oracle_step_sample(w, w.X, threads)
+        spent += t
+        elems += e
+        steps += 1
+    return {"value": elems / spent, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{steps} whole forward+backward step(s) of the {w.name} workload "
+                      f"({spent:.1f} s, OpenMP over BEV rows / (batch, camera))"}
+
+
+def run_reference(args):
+    from camera_bev_view_b200 import inputs as I
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = I.WORKLOADS[args.workload]
+    threads = cpu_cores()
+    rows = 8
+    for _ in range(args.warmup):
+        oracle_step_sample(w, rows, threads)
+    times, elems = [], 0
+    for _ in range(args.steps):
+        t, e = oracle_step_sample(w, rows, threads)
+        times.append(t)
+        elems += e
+    total = sum(times)
+    value = elems / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) features and 6-camera rigs; nuScenes-like shapes)",
+        "config": {"workload": workload_desc(w), "sample": f"{rows} BEV rows at the grid centre per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} of {w.X} BEV rows per step, forward + backward"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from camera_bev_view_b200 import inputs as I
+    from camera_bev_view_b200 import ops
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = I.WORKLOADS[args.workload]
+    B, N, C, Hf, Wf, X, Y = w.B, w.N, w.C, w.Hf, w.Wf, w.X, w.Y
+    F_h = I.make_features(w, shard=rank)
+    K_h, E_h = I.make_rigs(w, shard=rank)
+    dout_h = I.make_dout(w, shard=rank)
+    F, K, E, dout = (t.to(dev) for t in (F_h, K_h, E_h, dout_h))
+    esize = F.element_size()
+    grid = ops.bev_grid_spec(w.ranges, w.res)
+    Fcl = torch.empty((B, N, Hf, Wf, C), dtype=F.dtype, device=dev)
+    out = torch.empty((B, C, X, Y), dtype=torch.float32, device=dev)
+    dF = torch.empty((B, N, C, Hf, Wf), dtype=torch.float32, device=dev)
+    ws_b = torch.empty(ops.bev_workspace_size(ops.F32, ops.NCHW, B, N, C, Hf, Wf, 1), dtype=torch.uint8,
+                       device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    stages = {
+        "to_channels_last": lambda: ops.bev_features_to_channels_last(F, out=Fcl),
+        "forward": lambda: ops.bev_sample_forward(Fcl, K, E, w.img_h, w.img_w, grid, layout=ops.NHWC,
+                                                  out=out),
+        "backward": lambda: ops.bev_sample_backward(dout, K, E, w.img_h, w.img_w, grid, N, Hf, Wf, out=dF,
+                                                    workspace=ws_b),
+    }
+    launches_per_step = {"to_channels_last": 1, "forward": 1, "backward": 2}  # + one driver memset
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for f in stages.values():   # eager warm-up (also sets kernel attributes)
+            f()
+        stream.synchronize()
+        for name, f in stages.items():
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                f()
+            graphs[name] = g
+        for _ in range(args.warmup):
+            flush.zero_()
+            for g in graphs.values():
+                g.replay()
+        stream.synchronize()
+
+        names = list(stages)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local) as clocks:
+            for k in range(args.steps):
+                flush.zero_()
+                ev[k][0].record(stream)
+                for s, name in enumerate(names):
+                    graphs[name].replay()
+                    ev[k][s + 1].record(stream)
+            torch.cuda.synchronize(dev)
+            if world > 1:
+                dist.barrier()
+        per = {name: [ev[k][s].elapsed_time(ev[k][s + 1]) for k in range(args.steps)]
+               for s, name in enumerate(names)}
+    stage_ms = {name: sum(v) / len(v) for name, v in per.items()}
+    ms_local = sum(stage_ms.values())
+    ms = ms_local
+    if world > 1:
+        t = torch.tensor([ms_local], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    elems = B * C * X * Y
+    value = world * elems / (ms * 1e-3)
+
+    # roofline of the dominant kernel (by time)
+    peak, peak_src = hbm_peak()
+    fwd_bytes = B * N * Hf * Wf * C * esize + elems * 4
+    bwd_bytes = elems * 4 + B * N * C * Hf * Wf * 4
+    if stage_ms["forward"] >= stage_ms["backward"]:
+        dom, dom_ms, dom_bytes, kname = "forward", stage_ms["forward"], fwd_bytes, "sample_forward_kernel"
+        dom_note = "features read once + output written once; one launch"
+    else:
+        dom, dom_ms, dom_bytes, kname = "backward", stage_ms["backward"], bwd_bytes, "sample_backward_kernel"
+        dom_note = ("dout read once + dF written once; timed over the whole backward call "
+                    "(memset + scatter + layout kernel)")
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": recorded_traffic(kname, w.name), "kernel": kname, "stage": dom,
+                "algorithmic_bytes_per_launch": dom_bytes, "note": dom_note, "peak_source": peak_src}
+    fwd_gbs = fwd_bytes / (stage_ms["forward"] * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers
+    pin = lambda t: t.pin_memory()
+    F_p, K_p, E_p, dout_p = pin(F_h), pin(K_h), pin(E_h), pin(dout_h)
+    out_p = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dF_p = torch.empty(dF.shape, dtype=dF.dtype).pin_memory()
+    ws_f = torch.empty(max(256, ops.bev_workspace_size(ops.F32 if esize == 4 else ops.BF16, ops.NCHW, B, N, C,
+                                                       Hf, Wf, 0)), dtype=torch.uint8, device=dev)
+    e2e_times = []
+    with torch.cuda.stream(stream):
+        for k in range(args.e2e_steps + 5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            F.copy_(F_p, non_blocking=True)
+            K.copy_(K_p, non_blocking=True)
+            E.copy_(E_p, non_blocking=True)
+            dout.copy_(dout_p, non_blocking=True)
+            ops.bev_sample_forward(F, K, E, w.img_h, w.img_w, grid, out=out, workspace=ws_f)
+            ops.bev_sample_backward(dout, K, E, w.img_h, w.img_w, grid, N, Hf, Wf, out=dF, workspace=ws_b)
+            out_p.copy_(out, non_blocking=True)
+            dF_p.copy_(dF, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if k >= 5:
+                e2e_times.append(e0.elapsed_time(e1))
+    e2e_ms = statistics.median(e2e_times)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (F_h, K_h, E_h, dout_h))
+    d2h = out.numel() * 4 + dF.numel() * 4
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if esize == 4 else "bf16",
+        "data": "synthetic (seeded N(0,1) features and 6-camera rigs with nuScenes-like shapes; no dataset)",
+        "config": {"workload": workload_desc(w), "global_batch": B * world,
+                   "parallelism": f"dp{world} (each rank its own batch, no collective)",
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "timing": "CUDA events around CUDA-graph replays of each stage, launching stream"},
+        "stages_ms": stage_ms,
+        "forward_only": {"elements_per_s": elems / (stage_ms["forward"] * 1e-3), "GB_per_s": fwd_gbs,
+                         "frac_of_hbm_peak": fwd_gbs / peak},
+        "roofline": roofline,
+        "e2e": {"value": world * elems / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "pinned host -> device copies, bev_sample_forward (NCHW) + bev_sample_backward, "
+                        "device -> pinned host copies"},
+        "gpu_launches": args.steps * sum(launches_per_step.values()),
+        "clocks": clocks.summary(),
+    }
+    for g in graphs.values():
+        g.reset()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

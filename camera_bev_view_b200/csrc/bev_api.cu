@@ -1,0 +1,291 @@
+// bev_api.cu -- host side of the C ABI declared in include/bevsample.h.
+//
+// Validates every argument before anything is enqueued, picks the launch
+// shape (channel slices, lanes per cell) and enqueues the kernels on the
+// caller's stream.  No allocation, no synchronisation, no global state.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "bev_kernels.cuh"
+#include "bevsample.h"
+
+#define BEV_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool dims_ok(int B, int N, int C, int Hf, int Wf) {
+    if (B < 1 || N < 1 || C < 1 || Hf < 1 || Wf < 1) return false;
+    if (N > BEV_MAX_CAMERAS || Hf > BEV_MAX_DIM || Wf > BEV_MAX_DIM) return false;
+    if ((long long)B * N > 65535) return false;  // grid limits of the layout kernels
+    if (C > (1 << 20)) return false;
+    return true;
+}
+
+bool grid_ok(const bev_grid_t* g) {
+    if (!g) return false;
+    if (g->X < 1 || g->Y < 1 || g->Z < 1) return false;
+    if (g->X > BEV_MAX_DIM || g->Y > BEV_MAX_DIM || g->Z > BEV_MAX_Z) return false;
+    const float v[6] = {g->xmin, g->ymin, g->zmin, g->dx, g->dy, g->dz};
+    for (float f : v)
+        if (!isfinite(f)) return false;
+    return g->dx > 0.0f && g->dy > 0.0f && g->dz > 0.0f;
+}
+
+// A pointer the kernels may dereference: device or managed memory of `dev`.
+int device_ptr(const void* p, int dev) {
+    if (!p) return BEV_ERR_INVALID_ARG;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return BEV_ERR_INVALID_ARG;
+    }
+    if (at.type == cudaMemoryTypeManaged) return BEV_OK;
+    if (at.type != cudaMemoryTypeDevice || at.device != dev) return BEV_ERR_INVALID_ARG;
+    return BEV_OK;
+}
+
+int current_device(int* dev) {
+    if (cudaGetDevice(dev) != cudaSuccess) {
+        cudaGetLastError();
+        return BEV_ERR_CUDA;
+    }
+    return BEV_OK;
+}
+
+int chan_per_chunk(int dtype) { return dtype == BEV_BF16 ? 8 : 4; }
+int elem_size(int dtype) { return dtype == BEV_BF16 ? 2 : 4; }
+int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+// Does the forward need a repacked channels-last copy of the features?
+bool needs_repack(int dtype, int layout, int C) {
+    return layout == BEV_NCHW || (C % chan_per_chunk(dtype)) != 0;
+}
+
+size_t forward_ws(int dtype, int layout, int B, int N, int C, int Hf, int Wf) {
+    if (!needs_repack(dtype, layout, C)) return 0;
+    const size_t Cp = (size_t)round_up(C, chan_per_chunk(dtype));
+    return align_up((size_t)B * N * Hf * Wf * Cp * elem_size(dtype));
+}
+
+size_t backward_ws(int B, int N, int C, int Hf, int Wf) {
+    return align_up((size_t)B * N * Hf * Wf * (size_t)round_up(C, 4) * sizeof(float));
+}
+
+// Lanes per cell L (power of two dividing 32) and chunks per lane V for a
+// slice of qs 16-byte chunks: the widest L that divides qs with V <= 8, else
+// one warp per cell.
+void pick_lanes(int qs, int* L, int* V) {
+    for (int l = 32; l >= 1; l >>= 1) {
+        if (qs % l == 0 && qs / l <= 8) {
+            *L = l;
+            *V = qs / l;
+            return;
+        }
+    }
+    *L = 32;
+    *V = (qs + 31) / 32;
+}
+
+bev::GeoParams geo(const bev_grid_t* g, int Hf, int Wf, int img_h, int img_w) {
+    bev::GeoParams p;
+    p.xmin = g->xmin;
+    p.ymin = g->ymin;
+    p.zmin = g->zmin;
+    p.dx = g->dx;
+    p.dy = g->dy;
+    p.dz = g->dz;
+    p.img_w = (float)img_w;
+    p.img_h = (float)img_h;
+    p.sW = (float)Wf / (float)img_w;
+    p.sH = (float)Hf / (float)img_h;
+    p.X = g->X;
+    p.Y = g->Y;
+    p.Z = g->Z;
+    p.Hf = Hf;
+    p.Wf = Wf;
+    return p;
+}
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return BEV_OK;
+    cudaGetLastError();
+    return BEV_ERR_CUDA;
+}
+
+}  // namespace
+
+BEV_API const char* bev_status_string(int status) {
+    switch (status) {
+        case BEV_OK: return "ok";
+        case BEV_ERR_INVALID_ARG: return "invalid argument";
+        case BEV_ERR_UNSUPPORTED: return "unsupported request";
+        case BEV_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        case BEV_ERR_CUDA: return "CUDA runtime error";
+        case BEV_ERR_INTERNAL: return "internal consistency check failed";
+        default: return "unknown status";
+    }
+}
+
+BEV_API int bev_grid_spec(const float range[6], const float res[3], bev_grid_t* out) {
+    if (!range || !res || !out) return BEV_ERR_INVALID_ARG;
+    int counts[3];
+    float cell[3];
+    for (int a = 0; a < 3; ++a) {
+        const float lo = range[2 * a], hi = range[2 * a + 1], r = res[a];
+        if (!isfinite(lo) || !isfinite(hi) || !isfinite(r) || !(hi > lo) || !(r > 0.0f))
+            return BEV_ERR_INVALID_ARG;
+        const float extent = hi - lo;
+        const double q = (double)extent / (double)r;
+        const double k = nearbyint(q);
+        const int limit = a == 2 ? BEV_MAX_Z : BEV_MAX_DIM;
+        if (fabs(q - k) > 1e-4 || k < 1.0 || k > (double)limit) return BEV_ERR_INVALID_ARG;
+        counts[a] = (int)k;
+        cell[a] = extent / (float)counts[a];
+    }
+    out->X = counts[0];
+    out->Y = counts[1];
+    out->Z = counts[2];
+    out->xmin = range[0];
+    out->xmax = range[1];
+    out->ymin = range[2];
+    out->ymax = range[3];
+    out->zmin = range[4];
+    out->zmax = range[5];
+    out->dx = cell[0];
+    out->dy = cell[1];
+    out->dz = cell[2];
+    return BEV_OK;
+}
+
+BEV_API size_t bev_workspace_size(int dtype, int layout, int B, int N, int C, int Hf, int Wf,
+                                  int for_backward) {
+    if (!dims_ok(B, N, C, Hf, Wf)) return (size_t)-1;
+    if (for_backward) return backward_ws(B, N, C, Hf, Wf);
+    if ((dtype != BEV_F32 && dtype != BEV_BF16) || (layout != BEV_NCHW && layout != BEV_NHWC))
+        return (size_t)-1;
+    return forward_ws(dtype, layout, B, N, C, Hf, Wf);
+}
+
+BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int B, int N, int C, int Hf,
+                               int Wf, const float* intrinsics, const float* ego2cam, int img_h,
+                               int img_w, const bev_grid_t* grid, float* out, uint8_t* valid_count,
+                               void* workspace, size_t workspace_bytes, bev_stream_t stream) {
+    // host-only checks first: nothing below touches CUDA until these pass
+    if (!features || !intrinsics || !ego2cam || !out || !grid) return BEV_ERR_INVALID_ARG;
+    if (!dims_ok(B, N, C, Hf, Wf) || !grid_ok(grid)) return BEV_ERR_INVALID_ARG;
+    if (img_h < 1 || img_w < 1 || img_h > BEV_MAX_DIM || img_w > BEV_MAX_DIM) return BEV_ERR_INVALID_ARG;
+    if (dtype != BEV_F32 && dtype != BEV_BF16) return BEV_ERR_UNSUPPORTED;
+    if (layout != BEV_NCHW && layout != BEV_NHWC) return BEV_ERR_UNSUPPORTED;
+    const bool repack = needs_repack(dtype, layout, C);
+    const size_t ws_need = forward_ws(dtype, layout, B, N, C, Hf, Wf);
+    if (ws_need > 0 && (!workspace || workspace_bytes < ws_need || ((uintptr_t)workspace % kAlign) != 0))
+        return BEV_ERR_WORKSPACE;
+    if (!repack && ((uintptr_t)features % 16) != 0) return BEV_ERR_INVALID_ARG;
+
+    int dev;
+    int st = current_device(&dev);
+    if (st != BEV_OK) return st;
+    const void* ptrs[5] = {features, intrinsics, ego2cam, out, valid_count};
+    for (int k = 0; k < 5; ++k) {
+        if (k == 4 && !valid_count) continue;
+        if ((st = device_ptr(ptrs[k], dev)) != BEV_OK) return st;
+    }
+    if (ws_need > 0 && (st = device_ptr(workspace, dev)) != BEV_OK) return BEV_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int cpc = chan_per_chunk(dtype);
+    const int Cp = round_up(C, cpc);
+    const void* feat = features;
+    if (repack) {
+        st = cuda_status(bev_launch_to_channels_last(features, layout, elem_size(dtype), B * N, C,
+                                                     Hf * Wf, Cp, workspace, s));
+        if (st != BEV_OK) return st;
+        feat = workspace;
+    }
+    bev::SampleArgs a;
+    memset(&a, 0, sizeof(a));
+    a.feat = feat;
+    a.K = intrinsics;
+    a.E = ego2cam;
+    a.out = out;
+    a.count = valid_count;
+    a.g = geo(grid, Hf, Wf, img_h, img_w);
+    a.B = B;
+    a.N = N;
+    a.C = C;
+    a.Qtot = Cp / cpc;
+    a.chan_per_chunk = cpc;
+    const int max_chunks = bev::kSliceMax / cpc;
+    const int slices = (a.Qtot + max_chunks - 1) / max_chunks;
+    if (slices > 65535) return BEV_ERR_UNSUPPORTED;
+    a.slice_chunks = (a.Qtot + slices - 1) / slices;
+    int V;
+    pick_lanes(a.slice_chunks, &a.L, &V);
+    a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
+    return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, V, slices, s));
+}
+
+BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, int Wf,
+                                const float* intrinsics, const float* ego2cam, int img_h, int img_w,
+                                const bev_grid_t* grid, float* dfeatures, void* workspace,
+                                size_t workspace_bytes, bev_stream_t stream) {
+    if (!dout || !intrinsics || !ego2cam || !dfeatures || !grid) return BEV_ERR_INVALID_ARG;
+    if (!dims_ok(B, N, C, Hf, Wf) || !grid_ok(grid)) return BEV_ERR_INVALID_ARG;
+    if (img_h < 1 || img_w < 1 || img_h > BEV_MAX_DIM || img_w > BEV_MAX_DIM) return BEV_ERR_INVALID_ARG;
+    const size_t ws_need = backward_ws(B, N, C, Hf, Wf);
+    if (!workspace || workspace_bytes < ws_need || ((uintptr_t)workspace % kAlign) != 0)
+        return BEV_ERR_WORKSPACE;
+
+    int dev;
+    int st = current_device(&dev);
+    if (st != BEV_OK) return st;
+    const void* ptrs[4] = {dout, intrinsics, ego2cam, dfeatures};
+    for (int k = 0; k < 4; ++k)
+        if ((st = device_ptr(ptrs[k], dev)) != BEV_OK) return st;
+    if (device_ptr(workspace, dev) != BEV_OK) return BEV_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int Cp = round_up(C, 4);
+    if ((st = cuda_status(cudaMemsetAsync(workspace, 0, ws_need, s))) != BEV_OK) return st;
+    bev::SampleArgs a;
+    memset(&a, 0, sizeof(a));
+    a.K = intrinsics;
+    a.E = ego2cam;
+    a.dout = dout;
+    a.dfeat = static_cast<float*>(workspace);
+    a.g = geo(grid, Hf, Wf, img_h, img_w);
+    a.B = B;
+    a.N = N;
+    a.C = C;
+    a.Qtot = Cp / 4;
+    a.chan_per_chunk = 4;
+    const int max_chunks = bev::kSliceMax / 4;
+    const int slices = (a.Qtot + max_chunks - 1) / max_chunks;
+    if (slices > 65535) return BEV_ERR_UNSUPPORTED;
+    a.slice_chunks = (a.Qtot + slices - 1) / slices;
+    int V;
+    pick_lanes(a.slice_chunks, &a.L, &V);
+    a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
+    if ((st = cuda_status(bev_launch_backward(a, V, slices, s))) != BEV_OK) return st;
+    return cuda_status(bev_launch_to_nchw(static_cast<const float*>(workspace), B * N, C, Hf * Wf, Cp,
+                                          dfeatures, s));
+}
+
+BEV_API int bev_features_to_channels_last(const void* features, int dtype, int B, int N, int C, int Hf,
+                                          int Wf, void* out, bev_stream_t stream) {
+    if (!features || !out) return BEV_ERR_INVALID_ARG;
+    if (!dims_ok(B, N, C, Hf, Wf)) return BEV_ERR_INVALID_ARG;
+    if (dtype != BEV_F32 && dtype != BEV_BF16) return BEV_ERR_UNSUPPORTED;
+    int dev;
+    int st = current_device(&dev);
+    if (st != BEV_OK) return st;
+    if ((st = device_ptr(features, dev)) != BEV_OK) return st;
+    if ((st = device_ptr(out, dev)) != BEV_OK) return st;
+    return cuda_status(bev_launch_to_channels_last(features, BEV_NCHW, elem_size(dtype), B * N, C, Hf * Wf,
+                                                   C, out, reinterpret_cast<cudaStream_t>(stream)));
+}

@@ -1,0 +1,118 @@
+// bev_geometry.cuh -- device-side voxel geometry for the dense Sampling-VT.
+//
+// Projection and validity follow the SparseDriveV2 notes, "Deformable
+// Aggregation" step 2 ([u v 1]^T ~ K (R p + t); keep the camera only when the
+// projection lands in [0, W] x [0, H]) with the depth test depth > 0.1 and the
+// bilinear convention align_corners=False.  Every product and sum is rounded
+// on its own (__fmul_rn / __fadd_rn never fuse into FMA) and the divide is the
+// IEEE one, in the order the public header states, so validity counts and
+// corner indices are reproducible bit for bit.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bev {
+
+// Per-camera constants staged in shared memory: E rows 0..2 then K rows 0..1.
+constexpr int kCamFloats = 18;
+
+struct GeoParams {
+    float xmin, ymin, zmin;
+    float dx, dy, dz;
+    float img_w, img_h;   // image size as float (exact for sizes < 2^24)
+    float sW, sH;         // (float)Wf / (float)img_w, (float)Hf / (float)img_h, host IEEE divide
+    int X, Y, Z;
+    int Hf, Wf;
+};
+
+__device__ __forceinline__ float voxel_centre(float lo, int i, float d) {
+    return __fadd_rn(lo, __fmul_rn(__fadd_rn((float)i, 0.5f), d));
+}
+
+// Row r of the ego-to-camera transform: ((e0 x + e1 y) + e2 z) + e3.
+__device__ __forceinline__ float cam_row(const float* e, float x, float y, float z) {
+    float t = __fadd_rn(__fmul_rn(e[0], x), __fmul_rn(e[1], y));
+    t = __fadd_rn(t, __fmul_rn(e[2], z));
+    return __fadd_rn(t, e[3]);
+}
+
+// Project one voxel centre through one camera.  On success writes the
+// feature-map sampling position (fx, fy) and returns true.
+__device__ __forceinline__ bool project_voxel(const float* cam, float x, float y, float z,
+                                              const GeoParams& g, float& fx, float& fy) {
+    const float pcx = cam_row(cam + 0, x, y, z);
+    const float pcy = cam_row(cam + 4, x, y, z);
+    const float depth = cam_row(cam + 8, x, y, z);
+    if (!(depth > 0.1f)) return false;
+    const float* k = cam + 12;
+    float uh = __fadd_rn(__fmul_rn(k[0], pcx), __fmul_rn(k[1], pcy));
+    uh = __fadd_rn(uh, __fmul_rn(k[2], depth));
+    float vh = __fadd_rn(__fmul_rn(k[3], pcx), __fmul_rn(k[4], pcy));
+    vh = __fadd_rn(vh, __fmul_rn(k[5], depth));
+    const float u = __fdiv_rn(uh, depth);
+    const float v = __fdiv_rn(vh, depth);
+    if (!(u >= 0.0f && u <= g.img_w && v >= 0.0f && v <= g.img_h)) return false;
+    fx = __fadd_rn(__fmul_rn(u, g.sW), -0.5f);
+    fy = __fadd_rn(__fmul_rn(v, g.sH), -0.5f);
+    return true;
+}
+
+// Bilinear corners of (fx, fy): top-left texel and the four weights
+// w00 (y0,x0), w01 (y0,x0+1), w10 (y0+1,x0), w11 (y0+1,x0+1).
+struct Corners {
+    int x0, y0;
+    float w00, w01, w10, w11;
+};
+
+__device__ __forceinline__ Corners bilinear_corners(float fx, float fy) {
+    const float x0f = floorf(fx), y0f = floorf(fy);
+    const float wx1 = __fsub_rn(fx, x0f), wy1 = __fsub_rn(fy, y0f);
+    const float wx0 = __fsub_rn(1.0f, wx1), wy0 = __fsub_rn(1.0f, wy1);
+    Corners c;
+    c.x0 = (int)x0f;
+    c.y0 = (int)y0f;
+    c.w00 = __fmul_rn(wy0, wx0);
+    c.w01 = __fmul_rn(wy0, wx1);
+    c.w10 = __fmul_rn(wy1, wx0);
+    c.w11 = __fmul_rn(wy1, wx1);
+    return c;
+}
+
+// Conservative visibility of an axis-aligned box of voxel centres from one
+// camera.  Returns false only when one of the five validity conditions
+// (depth > 0.1, uh >= 0, W pc_z - uh >= 0, vh >= 0, H pc_z - vh >= 0) fails at
+// every point of the box by more than a rounding margin (1e-4 of the terms'
+// magnitude, far above the fp32 evaluation error).  Each condition plus its
+// margin is convex in the point, so its maximum over the box is at a vertex.
+__device__ inline bool box_may_be_visible(const float* cam, float x_lo, float x_hi, float y_lo,
+                                          float y_hi, float z_lo, float z_hi, float img_w,
+                                          float img_h) {
+    double best[5] = {-1e300, -1e300, -1e300, -1e300, -1e300};
+    const double W = img_w, H = img_h;
+    const double k0 = cam[12], k1 = cam[13], k2 = cam[14], k3 = cam[15], k4 = cam[16], k5 = cam[17];
+    for (int v = 0; v < 8; ++v) {
+        const double p[3] = {(v & 1) ? x_hi : x_lo, (v & 2) ? y_hi : y_lo, (v & 4) ? z_hi : z_lo};
+        double pc[3], mag[3];
+        for (int r = 0; r < 3; ++r) {
+            const float* e = cam + 4 * r;
+            pc[r] = (double)e[0] * p[0] + (double)e[1] * p[1] + (double)e[2] * p[2] + (double)e[3];
+            mag[r] = fabs((double)e[0] * p[0]) + fabs((double)e[1] * p[1]) +
+                     fabs((double)e[2] * p[2]) + fabs((double)e[3]);
+        }
+        const double uh = k0 * pc[0] + k1 * pc[1] + k2 * pc[2];
+        const double vh = k3 * pc[0] + k4 * pc[1] + k5 * pc[2];
+        const double umag = fabs(k0) * mag[0] + fabs(k1) * mag[1] + fabs(k2) * mag[2];
+        const double vmag = fabs(k3) * mag[0] + fabs(k4) * mag[1] + fabs(k5) * mag[2];
+        const double t = 1e-4, a = 1e-6;
+        const double val[5] = {pc[2] - 0.1 + t * mag[2] + a, uh + t * umag + a,
+                               W * pc[2] - uh + t * (umag + W * mag[2]) + a, vh + t * vmag + a,
+                               H * pc[2] - vh + t * (vmag + H * mag[2]) + a};
+        for (int q = 0; q < 5; ++q) best[q] = fmax(best[q], val[q]);
+    }
+    for (int q = 0; q < 5; ++q)
+        if (best[q] < 0.0) return false;
+    return true;
+}
+
+}  // namespace bev

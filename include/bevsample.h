@@ -1,0 +1,157 @@
+/*
+ * bevsample.h -- C ABI of the B200-native exact dense Sampling-VT library
+ * (libbevsample.so, sm_100a).
+ *
+ * The operation (FlashBEV reading notes, arxiv cs.RO 2607.10071, "Core Idea"
+ * and "Method" items 1-4): for every BEV output element (b, c, i, j) visit
+ * each height bin k and camera n, project the voxel centre through the
+ * camera's ego-to-camera extrinsic and intrinsic (SparseDriveV2 notes,
+ * "Deformable Aggregation" step 2: [u v 1]^T ~ K (R p + t)), keep the camera
+ * when depth > 0.1 and (u, v) lies in [0, W_img] x [0, H_img], sample the
+ * feature map bilinearly (align_corners=False, zero padding), average over the
+ * valid cameras of the bin and sum the bin means over height ("Key Insight":
+ * a height sum).  No voxel grid, projected-coordinate tensor, mask or
+ * Features3D volume is written to memory; the notes' "Method" item 4 holds:
+ * results equal the materialised form up to floating-point order.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers are DEVICE pointers on the current CUDA device unless marked
+ *    "host".  All tensors are dense, row-major, without padding.
+ *  - The caller owns every buffer.  The library allocates nothing, keeps no
+ *    global state between calls and may be called from several host threads.
+ *  - Work is enqueued asynchronously on `stream` (0 = legacy default stream).
+ *    No call synchronises the device or copies between host and device.
+ *  - Errors are returned as status codes, never thrown; no call aborts.  An
+ *    argument error is detected before anything is enqueued.
+ *  - Ego frame: x forward, y left, z up.  out[b, c, i, j]: row i indexes ego x,
+ *    column j indexes ego y (the LSS tutorial's "Splat" step: x to row, y to
+ *    column).  Camera frame: x right, y down, z forward (depth = camera z).
+ *  - Geometry is evaluated in fp32 in one fixed order, each product and sum
+ *    rounded separately, with an IEEE divide:
+ *      centre   x_i = xmin + ((float)i + 0.5f) * dx   (same for y_j, z_k)
+ *      camera   pc_r = ((E_r0 x + E_r1 y) + E_r2 z) + E_r3
+ *      image    u = ((K_00 pc_x + K_01 pc_y) + K_02 pc_z) / pc_z, v likewise
+ *      feature  fx = u * ((float)Wf / (float)W_img) - 0.5f, fy likewise
+ *      weights  x0 = floor(fx), wx1 = fx - x0, wx0 = 1 - wx1; w = wy * wx
+ *    so validity counts are reproducible bit for bit by any IEEE evaluation
+ *    of the same expression.  Accumulation is fp32.
+ *  - Preconditions not checked on the device: K's last row is [0 0 1]; E's
+ *    bottom row is ignored; calibrations are finite.
+ */
+#ifndef BEVSAMPLE_H
+#define BEVSAMPLE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* CUDA stream handle (identical to cudaStream_t / CUstream). */
+typedef struct CUstream_st* bev_stream_t;
+
+/* Feature storage type. */
+enum { BEV_F32 = 0, BEV_BF16 = 1 };
+/* Feature layout: [B,N,C,Hf,Wf] (per-camera NCHW) or [B,N,Hf,Wf,C] (channels last). */
+enum { BEV_NCHW = 0, BEV_NHWC = 1 };
+
+/* Status codes. */
+enum {
+    BEV_OK = 0,
+    BEV_ERR_INVALID_ARG = -1, /* NULL pointer, bad size, bad grid, host pointer where a device one is due */
+    BEV_ERR_UNSUPPORTED = -2, /* valid request outside what this build implements */
+    BEV_ERR_WORKSPACE = -3,   /* workspace NULL, too small or misaligned */
+    BEV_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
+    BEV_ERR_INTERNAL = -5     /* a device-side consistency check failed */
+};
+
+/* Limits of this build. */
+#define BEV_MAX_CAMERAS 32  /* N; counts are stored as uint8 */
+#define BEV_MAX_DIM 16384   /* X, Y, Hf, Wf, img sizes */
+#define BEV_MAX_Z 1024
+
+/* BEV voxel grid.  X, Y, Z counts; ranges in metres; dx, dy, dz = extent /
+ * count in fp32.  Voxel centres: xmin + ((float)i + 0.5f) * dx. */
+typedef struct bev_grid_t {
+    int X, Y, Z;
+    float xmin, xmax, ymin, ymax, zmin, zmax;
+    float dx, dy, dz;
+} bev_grid_t;
+
+/* Build a grid from ranges and cell sizes (LSS tutorial, "Splat": the range
+ * divided by the cell size gives the count, e.g. [-50, 50] m at 0.5 m -> 200).
+ *   range  host float[6]: xmin, xmax, ymin, ymax, zmin, zmax (max > min, finite)
+ *   res    host float[3]: dx, dy, dz (> 0)
+ *   out    host, written on success
+ * Each extent / res must lie within 1e-4 of an integer in [1, BEV_MAX_DIM]
+ * (Z: [1, BEV_MAX_Z]); the stored cell size is recomputed as extent / count
+ * in fp32.  Returns BEV_OK or BEV_ERR_INVALID_ARG.  Host only. */
+int bev_grid_spec(const float range[6], const float res[3], bev_grid_t* out);
+
+/* Bytes of device workspace bev_sample_forward (for_backward = 0) or
+ * bev_sample_backward (for_backward = 1) needs for these sizes; 0 when none is
+ * needed.  dtype/layout are ignored for the backward.  Returns (size_t)-1 for
+ * invalid sizes. */
+size_t bev_workspace_size(int dtype, int layout, int B, int N, int C, int Hf, int Wf,
+                          int for_backward);
+
+/* Forward: out[b, c, i, j] = sum_k [cnt > 0] (1 / cnt) sum_{valid n} bilinear(F[b, n, c], u, v)
+ * (FlashBEV reading notes, "Method" items 1-2).
+ *   features     [B,N,C,Hf,Wf] (BEV_NCHW) or [B,N,Hf,Wf,C] (BEV_NHWC); dtype BEV_F32 or BEV_BF16
+ *   intrinsics   [B,N,3,3] fp32, pixel units of a W_img x H_img image
+ *   ego2cam      [B,N,4,4] fp32, maps ego coordinates into the camera frame
+ *   img_h/img_w  image size the intrinsics refer to (>= 1)
+ *   grid         host pointer, from bev_grid_spec (or filled consistently)
+ *   out          [B,C,X,Y] fp32, fully overwritten
+ *   valid_count  [B,X,Y,Z] uint8 number of valid cameras per voxel, or NULL
+ *   workspace    device scratch of at least bev_workspace_size(dtype, layout, ..., 0)
+ *                bytes, 256-byte aligned (may be NULL when that size is 0).  The
+ *                library reuses it inside the call only; do not share one
+ *                workspace between calls that may overlap on the device.
+ * 1 <= N <= BEV_MAX_CAMERAS; B, C >= 1.
+ * Returns BEV_OK, BEV_ERR_INVALID_ARG, BEV_ERR_UNSUPPORTED, BEV_ERR_WORKSPACE
+ * or BEV_ERR_CUDA.  Outputs are undefined after an error. */
+int bev_sample_forward(const void* features, int dtype, int layout,
+                       int B, int N, int C, int Hf, int Wf,
+                       const float* intrinsics, const float* ego2cam,
+                       int img_h, int img_w, const bev_grid_t* grid,
+                       float* out, uint8_t* valid_count,
+                       void* workspace, size_t workspace_bytes, bev_stream_t stream);
+
+/* Backward with respect to the features only (the operator is linear in them):
+ *   dF[b, n, c, y, x] = sum over valid (i, j, k, n) samples touching texel (y, x)
+ *                       of w * dout[b, c, i, j] / cnt_k
+ * (FlashBEV reading notes, "Method" item 4: forward and backward differ from the
+ * materialised form only by floating-point order).  No gradient flows to K, E
+ * or the grid.
+ *   dout        [B,C,X,Y] fp32
+ *   dfeatures   [B,N,C,Hf,Wf] fp32, fully overwritten
+ *   workspace   at least bev_workspace_size(.., 1) bytes, 256-byte aligned
+ * Other arguments as for bev_sample_forward.  Accumulation order across cells
+ * is not fixed (atomics), so repeated calls may differ in the last bits. */
+int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, int Wf,
+                        const float* intrinsics, const float* ego2cam,
+                        int img_h, int img_w, const bev_grid_t* grid,
+                        float* dfeatures, void* workspace, size_t workspace_bytes,
+                        bev_stream_t stream);
+
+/* Channels-last copy of the features: out[b, n, y, x, c] = features[b, n, c, y, x].
+ * The forward performs this step itself for BEV_NCHW input; calling it
+ * separately lets a caller keep one channels-last copy for several forward
+ * calls, and pass it with layout BEV_NHWC (used in place when C is a multiple
+ * of 4 for fp32 or 8 for bf16).  A bandwidth-bound tiled transpose.
+ *   features  [B,N,C,Hf,Wf], dtype BEV_F32 or BEV_BF16
+ *   out       [B,N,Hf,Wf,C], same dtype, must not overlap features
+ * Returns BEV_OK, BEV_ERR_INVALID_ARG, BEV_ERR_UNSUPPORTED or BEV_ERR_CUDA. */
+int bev_features_to_channels_last(const void* features, int dtype, int B, int N, int C, int Hf, int Wf,
+                                  void* out, bev_stream_t stream);
+
+/* Static, human-readable text for a status code. */
+const char* bev_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BEVSAMPLE_H */

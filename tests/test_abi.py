@@ -1,0 +1,137 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from camera_bev_view_b200 import build as B
+from camera_bev_view_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bevsample.h")
+FAKE = 0x10000  # non-NULL, never dereferenced by the paths tested here
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return ops.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(bev_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["bev_grid_spec", "bev_workspace_size", "bev_sample_forward", "bev_sample_backward",
+              "bev_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    assert ops.bev_status_string(0) == "ok"
+    for s in (-1, -2, -3, -4, -5):
+        assert ops.bev_status_string(s) not in ("ok", "unknown status")
+    assert ops.bev_status_string(42) == "unknown status"
+
+
+def test_grid_spec(L):
+    g = ops.bev_grid_spec((-50, 50, -50, 50, -5, 3), (0.5, 0.5, 1.0))
+    assert (g.X, g.Y, g.Z) == (200, 200, 8)
+    assert (g.dx, g.dy, g.dz) == (0.5, 0.5, 1.0)
+    g = ops.bev_grid_spec((-50, 50, -50, 50, -5, 3), (0.25, 0.25, 0.5))
+    assert (g.X, g.Y, g.Z) == (400, 400, 16)
+    g = ops.bev_grid_spec((-25, 25, -25, 25, -5, 3), (1.0, 1.0, 2.0))
+    assert (g.X, g.Y, g.Z, g.xmin, g.zmax) == (50, 50, 4, -25.0, 3.0)
+    bad = [((-50, 50, -50, 50, -5, 3), (0.3, 0.5, 1.0)),       # non-integral
+           ((50, -50, -50, 50, -5, 3), (0.5, 0.5, 1.0)),       # max < min
+           ((-50, 50, -50, 50, -5, 3), (0.0, 0.5, 1.0)),       # zero res
+           ((-50, 50, -50, 50, -5, float("nan")), (0.5, 0.5, 1.0)),
+           ((-50, 50, -50, 50, -5, 3), (1e-4, 0.5, 1.0)),      # count above the limit
+           ((-50, 50, -50, 50, -5, 3), (0.5, 0.5, 1e-3))]      # Z above the limit
+    for r, s in bad:
+        with pytest.raises(ops.BevError) as e:
+            ops.bev_grid_spec(r, s)
+        assert e.value.status == -1
+    assert L.bev_grid_spec(None, None, None) == -1
+
+
+def test_workspace_sizes(L):
+    # NCHW fp32: channels-last copy, C padded to 4, 256-byte aligned
+    assert ops.bev_workspace_size(0, 0, 1, 6, 64, 16, 44, 0) == 6 * 16 * 44 * 64 * 4
+    assert ops.bev_workspace_size(1, 0, 4, 6, 128, 32, 88, 0) == 4 * 6 * 32 * 88 * 128 * 2
+    assert ops.bev_workspace_size(0, 0, 1, 1, 3, 2, 2, 0) == 256          # 16 floats -> 256
+    # NHWC with aligned channel count: used in place
+    assert ops.bev_workspace_size(0, 1, 1, 6, 64, 16, 44, 0) == 0
+    assert ops.bev_workspace_size(1, 1, 1, 6, 120, 16, 44, 0) == 0
+    # NHWC with C not a multiple of the 16-byte chunk: repacked
+    assert ops.bev_workspace_size(1, 1, 1, 6, 12, 16, 44, 0) == 6 * 16 * 44 * 16 * 2
+    # backward: fp32 channels-last gradient
+    assert ops.bev_workspace_size(0, 0, 2, 6, 64, 16, 44, 1) == 2 * 6 * 16 * 44 * 64 * 4
+    for args in [(0, 0, 0, 6, 64, 16, 44, 0), (0, 0, 1, 33, 64, 16, 44, 0), (2, 0, 1, 6, 64, 16, 44, 0),
+                 (0, 2, 1, 6, 64, 16, 44, 0), (0, 0, 1, 6, 64, 0, 44, 1)]:
+        with pytest.raises(ops.BevError):
+            ops.bev_workspace_size(*args)
+
+
+def _fwd(L, **kw):
+    g = ops.bev_grid_spec((-50, 50, -50, 50, -5, 3), (0.5, 0.5, 1.0))
+    a = dict(features=FAKE, dtype=0, layout=0, B=1, N=6, C=64, Hf=16, Wf=44, K=FAKE, E=FAKE,
+             img_h=256, img_w=704, grid=ctypes.byref(g), out=FAKE, count=None, ws=FAKE,
+             ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.bev_sample_forward(a["features"], a["dtype"], a["layout"], a["B"], a["N"], a["C"], a["Hf"],
+                                a["Wf"], a["K"], a["E"], a["img_h"], a["img_w"], a["grid"], a["out"],
+                                a["count"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def _bwd(L, **kw):
+    g = ops.bev_grid_spec((-50, 50, -50, 50, -5, 3), (0.5, 0.5, 1.0))
+    a = dict(dout=FAKE, B=2, N=6, C=64, Hf=16, Wf=44, K=FAKE, E=FAKE, img_h=256, img_w=704,
+             grid=ctypes.byref(g), dF=FAKE, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.bev_sample_backward(a["dout"], a["B"], a["N"], a["C"], a["Hf"], a["Wf"], a["K"], a["E"],
+                                 a["img_h"], a["img_w"], a["grid"], a["dF"], a["ws"], a["ws_bytes"],
+                                 a["stream"])
+
+
+def test_forward_argument_errors(L):
+    bad_grid = ops.BevGrid(0, 10, 10, 0, 1, 0, 1, 0, 1, 0.1, 0.1, 0.1)
+    nan_grid = ops.BevGrid(10, 10, 10, float("nan"), 1, 0, 1, 0, 1, 0.1, 0.1, 0.1)
+    cases = [
+        (dict(features=None), -1), (dict(K=None), -1), (dict(E=None), -1), (dict(out=None), -1),
+        (dict(grid=None), -1), (dict(B=0), -1), (dict(N=0), -1), (dict(N=33), -1), (dict(C=0), -1),
+        (dict(Hf=0), -1), (dict(Wf=-3), -1), (dict(img_h=0), -1), (dict(img_w=0), -1),
+        (dict(grid=ctypes.byref(bad_grid)), -1), (dict(grid=ctypes.byref(nan_grid)), -1),
+        (dict(B=20000), -1),                         # B * N beyond the launch limits
+        (dict(dtype=2), -2), (dict(layout=5), -2),
+        (dict(ws=None), -3), (dict(ws_bytes=100), -3), (dict(ws=FAKE + 8), -3),
+        (dict(layout=1, features=FAKE + 4, ws=None, ws_bytes=0), -1),   # NHWC in place must be 16B aligned
+    ]
+    for kw, want in cases:
+        assert _fwd(L, **kw) == want, kw
+
+
+def test_backward_argument_errors(L):
+    cases = [(dict(dout=None), -1), (dict(dF=None), -1), (dict(K=None), -1), (dict(N=40), -1),
+             (dict(C=0), -1), (dict(grid=None), -1), (dict(img_w=-1), -1),
+             (dict(ws=None), -3), (dict(ws_bytes=1024), -3), (dict(ws=FAKE + 16), -3)]
+    for kw, want in cases:
+        assert _bwd(L, **kw) == want, kw
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_host_checks_then_cuda_error_without_device(L):
+    # every host-side check passes; the first CUDA call reports that no device is usable
+    assert _fwd(L) == -4
+    assert _bwd(L) == -4
