@@ -11,6 +11,7 @@ The functions keep the C names:
     bev_workspace_size(dtype, layout, B, N, C, Hf, Wf, for_backward) -> int
     bev_sample_forward(features, K, E, img_h, img_w, grid, ...) -> (out, count)
     bev_sample_backward(dout, K, E, img_h, img_w, grid, N, Hf, Wf, ...) -> dfeatures
+    bev_sample_backward_noalloc(dout, K, E, img_h, img_w, grid, N, Hf, Wf, out) -> dfeatures
     bev_features_to_channels_last(features, out=None) -> [B,N,Hf,Wf,C] copy
     bev_status_string(status)                        -> str
 """
@@ -75,6 +76,9 @@ def lib():
         L.bev_sample_backward.argtypes = [P, I, I, I, I, I, P, P, I, I, ctypes.POINTER(BevGrid),
                                           P, P, S, P]
         L.bev_sample_backward.restype = I
+        L.bev_sample_backward_noalloc.argtypes = [P, I, I, I, I, I, P, P, I, I, ctypes.POINTER(BevGrid),
+                                                  P, P]
+        L.bev_sample_backward_noalloc.restype = I
         L.bev_features_to_channels_last.argtypes = [P, I, I, I, I, I, I, P, P]
         L.bev_features_to_channels_last.restype = I
         L.bev_status_string.argtypes = [I]
@@ -181,4 +185,19 @@ def bev_features_to_channels_last(features: torch.Tensor, out: torch.Tensor | No
                                              out.data_ptr(), _stream_ptr(stream))
     if st != 0:
         raise BevError(st, "bev_features_to_channels_last")
+    return out
+
+
+def bev_sample_backward_noalloc(dout: torch.Tensor, K: torch.Tensor, E: torch.Tensor, img_h: int, img_w: int,
+                                grid: BevGrid, N: int, Hf: int, Wf: int, out: torch.Tensor,
+                                stream=None) -> torch.Tensor:
+    """Feature gradient without a workspace, for callers that cannot allocate:
+    the library accumulates in its own fixed 16 MiB device array.  ``out``
+    ([B,N,C,Hf,Wf] fp32) must be supplied; this wrapper allocates nothing."""
+    B, C = dout.shape[:2]
+    st = lib().bev_sample_backward_noalloc(
+        dout.data_ptr(), B, N, C, Hf, Wf, K.data_ptr(), E.data_ptr(), int(img_h), int(img_w),
+        ctypes.byref(grid), out.data_ptr(), _stream_ptr(stream))
+    if st != 0:
+        raise BevError(st, "bev_sample_backward_noalloc")
     return out

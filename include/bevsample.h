@@ -136,6 +136,37 @@ int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, int Wf,
                         float* dfeatures, void* workspace, size_t workspace_bytes,
                         bev_stream_t stream);
 
+/* Size of the built-in scratch array used by bev_sample_backward_noalloc. */
+#define BEV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* The feature gradient of bev_sample_backward for callers that cannot
+ * allocate device memory or hand the library a workspace -- for example a
+ * plugin inside an engine that pre-plans every device buffer and gives its
+ * plugins no allocator, a deployment that forbids device allocation after
+ * start-up, or a real-time loop in which cudaMalloc / cudaFree would stall the
+ * device.  (The pages have no counterpart: this is a packaging variant of the
+ * backward above, with the same arguments minus the workspace and the same
+ * results.)
+ *
+ * The accumulation buffer lives in a fixed array of BEV_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) in the library's own device memory, which every GPU that loads the
+ * library keeps until the process exits.  Shapes whose buffer,
+ * B * N * Hf * Wf * round_up(C, 4) * 4 bytes, exceeds it are rejected with
+ * BEV_ERR_UNSUPPORTED before anything is enqueued.
+ *
+ * The first call on each device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with that device current) and caches it, so make the
+ * first call on a device before capturing any stream.  All calls share the one
+ * array and leave their contents in it; each call clears what it uses before
+ * accumulating.  Calls whose work may overlap on the GPU (other streams, other
+ * host threads) race on the array: serialise them.  Nothing is allocated and
+ * no cudaMalloc / cudaFree is made.  Other arguments, results and errors as for
+ * bev_sample_backward. */
+int bev_sample_backward_noalloc(const float* dout, int B, int N, int C, int Hf, int Wf,
+                                const float* intrinsics, const float* ego2cam,
+                                int img_h, int img_w, const bev_grid_t* grid,
+                                float* dfeatures, bev_stream_t stream);
+
 /* Channels-last copy of the features: out[b, n, y, x, c] = features[b, n, c, y, x].
  * The forward performs this step itself for BEV_NCHW input; calling it
  * separately lets a caller keep one channels-last copy for several forward
