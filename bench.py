@@ -25,7 +25,6 @@ with "impl": "reference".
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -77,21 +76,27 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (earlier measurement on this pool)"
 
 
-def source_digest():
+KERNEL_SOURCES = {
+    "sample_forward_kernel": ["bev_forward.cu", "bev_tile.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
+    "sample_backward_kernel": ["bev_backward.cu", "bev_tile.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
+}
+
+
+def source_digest(kernel):
+    """Digest of the source files a kernel is built from."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "camera_bev_view_b200", "csrc", "*"))):
-        h.update(open(p, "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "camera_bev_view_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+    on the kernel's current sources; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        rec = json.load(open(p))
-        ent = rec[kernel][workload]
-        if ent.get("source_digest") == source_digest():
+        ent = json.load(open(p))[kernel][workload]
+        if ent.get("source_digest") == source_digest(kernel):
             return float(ent["dram_bytes_per_launch"])
     except Exception:
         pass
