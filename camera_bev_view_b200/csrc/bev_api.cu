@@ -76,19 +76,33 @@ size_t backward_ws(int B, int N, int C, int Hf, int Wf) {
     return align_up((size_t)B * N * Hf * Wf * (size_t)round_up(C, 4) * sizeof(float));
 }
 
-// Lanes per cell L (power of two dividing 32) and chunks per lane V for a
-// slice of qs 16-byte chunks: the widest L that divides qs with V <= 8, else
-// one warp per cell.
+// Lanes per cell L and 16-byte chunks per lane V (<= 8) for a slice of qs
+// chunks (qs <= 32).  Eight lanes per cell is preferred: each load
+// instruction then covers whole 128-byte lines of four cells, and each lane
+// keeps 2V packed accumulators busy per texel.  Wider or narrower groups are
+// used only when eight lanes would leave more than a fifth of the lanes idle.
 void pick_lanes(int qs, int* L, int* V) {
-    for (int l = 32; l >= 1; l >>= 1) {
-        if (qs % l == 0 && qs / l <= 8) {
+    const int order[4] = {8, 16, 32, 4};
+    for (int k = 0; k < 4; ++k) {
+        const int l = order[k], v = (qs + l - 1) / l;
+        if (v <= 8 && 5 * (l * v - qs) <= l * v) {
             *L = l;
-            *V = qs / l;
+            *V = v;
             return;
         }
     }
-    *L = 32;
-    *V = (qs + 31) / 32;
+    int best_l = 4, best_v = (qs + 3) / 4, best_waste = 1 << 30;
+    for (int k = 0; k < 4; ++k) {
+        const int l = order[k], v = (qs + l - 1) / l;
+        if (v > 8) continue;
+        if (l * v - qs < best_waste) {
+            best_waste = l * v - qs;
+            best_l = l;
+            best_v = v;
+        }
+    }
+    *L = best_l;
+    *V = best_v;
 }
 
 bev::GeoParams geo(const bev_grid_t* g, int Hf, int Wf, int img_h, int img_w) {
@@ -226,6 +240,7 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
     a.slice_chunks = (a.Qtot + slices - 1) / slices;
     int V;
     pick_lanes(a.slice_chunks, &a.L, &V);
+    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
     a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
     return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, V, slices, s));
 }
@@ -270,6 +285,7 @@ BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, 
     a.slice_chunks = (a.Qtot + slices - 1) / slices;
     int V;
     pick_lanes(a.slice_chunks, &a.L, &V);
+    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
     a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
     if ((st = cuda_status(bev_launch_backward(a, V, slices, s))) != BEV_OK) return st;
     return cuda_status(bev_launch_to_nchw(static_cast<const float*>(workspace), B * N, C, Hf * Wf, Cp,

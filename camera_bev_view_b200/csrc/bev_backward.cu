@@ -4,16 +4,16 @@
 // The forward is linear in F, so dL/dF is its adjoint (FlashBEV reading notes,
 // "Method" item 4: forward and backward differ from the materialised form only
 // by floating-point order):
-//   dF[b, n, c, y, x] += w * dout[b, c, i, j] / cnt_k
-// for every valid (cell, bin, camera) sample and every in-range bilinear corner
-// (y, x) it touches.
+//   dF[b, n, c, y, x] += (sum_k w_k / cnt_k) * dout[b, c, i, j]
+// over every (cell, camera) and every texel (y, x) its valid samples touch.
 //
 // One CTA = one 8x8 BEV tile of one batch item and one channel slice, with the
-// same culling and once-per-voxel geometry as the forward.  The tile's dout
-// slice is staged in shared memory (coalesced along y); each lane then owns V
-// chunks of 4 channels of one cell and scatters w / cnt * dout into the fp32
-// channels-last gradient buffer with 16-byte vector reductions
-// (red.global.add.v4.f32), one per (corner, chunk).
+// same culling, once-per-voxel geometry and merged per-(cell, camera, texel)
+// weights as the forward (bev_tile.cuh).  The tile's dout slice is staged in
+// shared memory (coalesced along y) and held in registers: each lane owns V
+// chunks of 4 channels of one cell.  Each touched texel then receives one
+// 16-byte vector reduction per chunk (red.global.add.v4.f32) into the fp32
+// channels-last gradient buffer, however many height bins hit it.
 #include "bev_tile.cuh"
 
 namespace bev {
@@ -24,112 +24,167 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
-template <int V>
-__global__ void __launch_bounds__(kThreads) sample_backward_kernel(const SampleArgs a) {
+template <int L, int V>
+__device__ __forceinline__ void scatter_texel(float* p, const float (&d)[V][4], float w, int ql,
+                                              int nchunks) {
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+        if (ql + v * L < nchunks)
+            red_add_v4(p + v * L * 4, w * d[v][0], w * d[v][1], w * d[v][2], w * d[v][3]);
+}
+
+template <int L, int V>
+__device__ __forceinline__ void scatter_patch(const float (&d)[V][4], const float* pf, const int4 pi,
+                                              float* Gn, int Wf, int tstride, int ql, int nchunks) {
+    const int h = pi.z >> 16, w = pi.z & 0xffff;
+    const float* pw = pf + pi.w;
+    float* grow = Gn + ((size_t)pi.x * Wf + pi.y) * tstride;
+    for (int r = 0; r < h; ++r, grow += (size_t)Wf * tstride, pw += w) {
+        for (int cc = 0; cc < w; ++cc) {
+            const float wt = pw[cc];
+            if (wt != 0.0f) scatter_texel<L, V>(grow + (size_t)cc * tstride, d, wt, ql, nchunks);
+        }
+    }
+}
+
+template <int L, int V>
+__device__ __forceinline__ void scatter_direct(const float (&d)[V][4], const TileSmem& s, int cell, int aa,
+                                               int zlen, float* Gn, int Hf, int Wf, int tstride, int ql,
+                                               int nchunks) {
+    for (int zl = 0; zl < zlen; ++zl) {
+        const float2 f = s.items[item_index(cell, aa, zl, zlen)];
+        if (!(f.x == f.x)) continue;
+        const float cntf = (float)cell_count(s.cnt, zl, cell);
+        const Corners c = bilinear_corners(f.x, f.y);
+        const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
+            if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
+            scatter_texel<L, V>(Gn + ((size_t)yy * Wf + xx) * tstride, d, __fdiv_rn(ws[k], cntf), ql, nchunks);
+        }
+    }
+}
+
+template <int L, int V>
+__global__ void __launch_bounds__(kThreads, 2) sample_backward_kernel(const SampleArgs a) {
+    constexpr int G = 32 / L;
+    constexpr int CG = kCellsPerWarp / G;
+    static_assert(G * CG == kCellsPerWarp, "lanes per cell must be 4, 8, 16 or 32");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const TileSmem s = carve_smem(smem_raw, a.N);
+    float* dbuf = reinterpret_cast<float*>(smem_raw + sample_smem_bytes(a.N));
     const GeoParams& g = a.g;
 
     const int b = blockIdx.y;
-    const int ti0 = (blockIdx.x / a.tiles_j) * kTileI;
-    const int tj0 = (blockIdx.x % a.tiles_j) * kTileJ;
+    int ti0, tj0;
+    tile_origin(a, ti0, tj0);
     const int chunk0 = blockIdx.z * a.slice_chunks;
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
-    const int cs = nchunks * 4;
     const int c_base = chunk0 * 4;
 
     // stage dout[b, c_base + c, tile] as [c][cell]; padding channels read as 0
-    for (int t = threadIdx.x; t < cs * kTile; t += kThreads) {
+    for (int t = threadIdx.x; t < nchunks * 4 * kTile; t += kThreads) {
         const int c = t / kTile, cell = t - c * kTile;
         const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
         float v = 0.0f;
         if (c_base + c < a.C && i < g.X && j < g.Y)
             v = a.dout[(((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + j];
-        s.obuf[c * kObufStride + cell] = v;
+        dbuf[c * kObufStride + cell] = v;
     }
     setup_tile(a, s, b, ti0, tj0);
     const int nA = s.act[32];
     if (nA == 0) return;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int L = a.L, G = 32 / L;
     const int sub = lane / L, ql = lane - sub * L;
-    const int zc = z_chunk(g.Z, nA);
+    float d[CG][V][4];
+#pragma unroll
+    for (int q = 0; q < CG; ++q) {
+        const int cell = warp * kCellsPerWarp + q * G + sub;
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            const int cq = ql + v * L;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[q][v][e] = cq < nchunks ? dbuf[(cq * 4 + e) * kObufStride + cell] : 0.0f;
+        }
+    }
     const size_t texels = (size_t)g.Hf * g.Wf;
     const int tstride = a.Qtot * 4;  // floats per texel in the gradient buffer
+    float* grad = a.dfeat + (size_t)(chunk0 + ql) * 4;
 
-    for (int z0 = 0; z0 < g.Z; z0 += zc) {
+    int zc = z_chunk(g.Z, nA);
+    int z0 = 0;
+    while (z0 < g.Z) {
         const int zlen = min(zc, g.Z - z0);
         geometry_chunk(a, s, ti0, tj0, nA, z0, zlen);
-        for (int cg = warp; cg * G < kTile; cg += kWarps) {
-            const int cell = cg * G + sub;
-            float d[V][4];
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int q = ql + v * L;
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    d[v][e] = q < nchunks ? s.obuf[(q * 4 + e) * kObufStride + cell] : 0.0f;
+        int total = layout_patches(a, s, zlen, 0, nA);
+        if (total < 0 && zlen > 1) {  // too many texels: fewer bins per chunk
+            zc = (zlen + 1) / 2;
+            continue;
+        }
+        int a0 = 0, ga = nA;
+        while (a0 < nA) {
+            const int a1 = min(nA, a0 + ga);
+            if (a0 > 0 || a1 < nA) total = layout_patches(a, s, zlen, a0, a1);
+            if (total < 0 && a1 - a0 > 1) {  // still too many: fewer cameras at once
+                ga = (a1 - a0 + 1) / 2;
+                continue;
             }
-            for (int aa = 0; aa < nA; ++aa) {
-                const int n = s.act[aa];
-                float* Gn = a.dfeat + ((size_t)b * a.N + n) * texels * tstride + (size_t)(chunk0 + ql) * 4;
-                const float2* it = s.items + (cell * nA + aa) * zlen;
-                const int* cn = s.cnt + cell * zlen;
-                for (int zl = 0; zl < zlen; ++zl) {
-                    const float2 f = it[zl];
-                    if (!(f.x == f.x)) continue;
-                    const float sc = __frcp_rn((float)cn[zl]);
-                    const Corners c = bilinear_corners(f.x, f.y);
-                    const int ys[4] = {c.y0, c.y0, c.y0 + 1, c.y0 + 1};
-                    const int xs[4] = {c.x0, c.x0 + 1, c.x0, c.x0 + 1};
-                    const float ws[4] = {c.w00 * sc, c.w01 * sc, c.w10 * sc, c.w11 * sc};
+            if (total >= 0) fill_patches(a, s, zlen, a0, a1);
+            const float* pf = s.patch;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        if ((unsigned)ys[k] >= (unsigned)g.Hf || (unsigned)xs[k] >= (unsigned)g.Wf) continue;
-                        float* p = Gn + ((size_t)ys[k] * g.Wf + xs[k]) * tstride;
-#pragma unroll
-                        for (int v = 0; v < V; ++v) {
-                            if (ql + v * L < nchunks)
-                                red_add_v4(p + v * L * 4, ws[k] * d[v][0], ws[k] * d[v][1],
-                                           ws[k] * d[v][2], ws[k] * d[v][3]);
-                        }
-                    }
+            for (int q = 0; q < CG; ++q) {
+                const int cell = warp * kCellsPerWarp + q * G + sub;
+                for (int aa = a0; aa < a1; ++aa) {
+                    float* Gn = grad + ((size_t)b * a.N + s.act[aa]) * texels * tstride;
+                    if (total >= 0)
+                        scatter_patch<L, V>(d[q], pf, s.pinfo[aa * kTile + cell], Gn, g.Wf, tstride, ql, nchunks);
+                    else
+                        scatter_direct<L, V>(d[q], s, cell, aa, zlen, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
                 }
             }
+            __syncthreads();
+            a0 = a1;
+            total = -1;
         }
+        z0 += zlen;
     }
 }
 
-static cudaError_t launch_bwd_v(const SampleArgs& a, int V, dim3 grid, size_t smem, cudaStream_t st) {
-    switch (V) {
-#define BEV_BWD_CASE(VV)                                                                        \
-    case VV: {                                                                                  \
-        auto k = sample_backward_kernel<VV>;                                                    \
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,    \
-                                             (int)smem);                                        \
-        if (e != cudaSuccess) return e;                                                         \
-        k<<<grid, kThreads, smem, st>>>(a);                                                     \
-        return cudaGetLastError();                                                              \
-    }
-        BEV_BWD_CASE(1)
-        BEV_BWD_CASE(2)
-        BEV_BWD_CASE(3)
-        BEV_BWD_CASE(4)
-        BEV_BWD_CASE(5)
-        BEV_BWD_CASE(6)
-        BEV_BWD_CASE(7)
-        BEV_BWD_CASE(8)
-#undef BEV_BWD_CASE
-        default:
-            return cudaErrorInvalidValue;
+template <int L, int V>
+static cudaError_t launch_one(const SampleArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
+    auto k = sample_backward_kernel<L, V>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_bwd(const SampleArgs& a, int V, dim3 grid, size_t smem, cudaStream_t st) {
+    switch (a.L * 16 + V) {
+        case 32 * 16 + 1: return launch_one<32, 1>(a, grid, smem, st);
+        case 16 * 16 + 1: return launch_one<16, 1>(a, grid, smem, st);
+        case 16 * 16 + 2: return launch_one<16, 2>(a, grid, smem, st);
+        case 8 * 16 + 1: return launch_one<8, 1>(a, grid, smem, st);
+        case 8 * 16 + 2: return launch_one<8, 2>(a, grid, smem, st);
+        case 8 * 16 + 3: return launch_one<8, 3>(a, grid, smem, st);
+        case 8 * 16 + 4: return launch_one<8, 4>(a, grid, smem, st);
+        case 4 * 16 + 1: return launch_one<4, 1>(a, grid, smem, st);
+        case 4 * 16 + 2: return launch_one<4, 2>(a, grid, smem, st);
+        case 4 * 16 + 3: return launch_one<4, 3>(a, grid, smem, st);
+        case 4 * 16 + 4: return launch_one<4, 4>(a, grid, smem, st);
+        case 4 * 16 + 5: return launch_one<4, 5>(a, grid, smem, st);
+        case 4 * 16 + 6: return launch_one<4, 6>(a, grid, smem, st);
+        case 4 * 16 + 7: return launch_one<4, 7>(a, grid, smem, st);
+        case 4 * 16 + 8: return launch_one<4, 8>(a, grid, smem, st);
+        default: return cudaErrorInvalidValue;
     }
 }
 
 }  // namespace bev
 
 cudaError_t bev_launch_backward(const bev::SampleArgs& a, int V, int slices, cudaStream_t stream) {
-    const int tiles_i = (a.g.X + bev::kTileI - 1) / bev::kTileI;
-    const dim3 grid(tiles_i * a.tiles_j, a.B, slices);
-    return bev::launch_bwd_v(a, V, grid, bev::sample_smem_bytes(a.N), stream);
+    const dim3 grid(a.tiles_i * a.tiles_j, a.B, slices);
+    return bev::launch_bwd(a, V, grid, bev::sample_smem_bytes_bwd(a.N), stream);
 }

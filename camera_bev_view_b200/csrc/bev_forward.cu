@@ -4,138 +4,284 @@
 // (FlashBEV reading notes, "Method" items 1-2: per-bin valid mean over cameras,
 // then a sum over height, in one kernel with nothing intermediate in HBM).
 //
-// One CTA = one 8x8 BEV tile of one batch item and one channel slice.
-//   1. camera constants to shared memory; cameras that cannot see the tile
-//      are culled (conservative box test);
-//   2. per chunk of height bins: (fx, fy) of every (cell, active camera, bin)
-//      and the per-(cell, bin) valid count, computed once, in shared memory;
-//   3. each warp takes G = 32 / L cells at a time; the L lanes of a cell sweep
-//      the channel slice with 16-byte loads from the channels-last feature
-//      buffer (V chunks per lane) and accumulate w / cnt * F in fp32 registers;
-//   4. the per-cell partial sums are folded into a [channel][cell] staging tile
-//      in shared memory, which is finally stored along y (the contiguous axis
-//      of out) in coalesced rows.
+// One CTA = one 8x8 BEV tile of one batch item and one channel slice; warp w
+// owns tile row w.  Per tile (bev_tile.cuh): cameras are culled, every
+// (cell, camera, bin) voxel is projected once, and the weights w / cnt of all
+// bins are merged per (cell, camera, texel).  The channel loop then visits
+// each touched texel of a (cell, camera) once: the L lanes of a cell read its
+// channel vector with 16-byte loads (V chunks per lane) from the channels-last
+// feature buffer and accumulate in fp32 registers, which persist across
+// height chunks.  The tile is finally stored along y, the contiguous axis of
+// out, through a [channel][cell] shared-memory staging tile.
 #include "bev_tile.cuh"
 
 namespace bev {
 
+// Channel chunks of 16 bytes: 4 fp32 or 8 bf16 channels, accumulated in fp32
+// pairs with the packed fp32x2 FMA of sm_100 (each half is an IEEE fma.rn).
 template <bool BF16>
 struct Chunk;
 
 template <>
 struct Chunk<false> {
-    static constexpr int kCh = 4;
-    __device__ __forceinline__ static void fma(float (&acc)[4], const uint4& d, float w) {
-        acc[0] = fmaf(w, __uint_as_float(d.x), acc[0]);
-        acc[1] = fmaf(w, __uint_as_float(d.y), acc[1]);
-        acc[2] = fmaf(w, __uint_as_float(d.z), acc[2]);
-        acc[3] = fmaf(w, __uint_as_float(d.w), acc[3]);
+    static constexpr int kPairs = 2;
+    __device__ __forceinline__ static void fma(float2 (&acc)[2], const uint4& d, float w) {
+        const float2 ww = make_float2(w, w);
+        acc[0] = __ffma2_rn(ww, make_float2(__uint_as_float(d.x), __uint_as_float(d.y)), acc[0]);
+        acc[1] = __ffma2_rn(ww, make_float2(__uint_as_float(d.z), __uint_as_float(d.w)), acc[1]);
     }
 };
 
 template <>
 struct Chunk<true> {
-    static constexpr int kCh = 8;
+    static constexpr int kPairs = 4;
     // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word.
-    __device__ __forceinline__ static void fma(float (&acc)[8], const uint4& d, float w) {
-        acc[0] = fmaf(w, __uint_as_float(d.x << 16), acc[0]);
-        acc[1] = fmaf(w, __uint_as_float(d.x & 0xffff0000u), acc[1]);
-        acc[2] = fmaf(w, __uint_as_float(d.y << 16), acc[2]);
-        acc[3] = fmaf(w, __uint_as_float(d.y & 0xffff0000u), acc[3]);
-        acc[4] = fmaf(w, __uint_as_float(d.z << 16), acc[4]);
-        acc[5] = fmaf(w, __uint_as_float(d.z & 0xffff0000u), acc[5]);
-        acc[6] = fmaf(w, __uint_as_float(d.w << 16), acc[6]);
-        acc[7] = fmaf(w, __uint_as_float(d.w & 0xffff0000u), acc[7]);
+    __device__ __forceinline__ static void fma(float2 (&acc)[4], const uint4& d, float w) {
+        const float2 ww = make_float2(w, w);
+        acc[0] = __ffma2_rn(ww, make_float2(__uint_as_float(d.x << 16), __uint_as_float(d.x & 0xffff0000u)), acc[0]);
+        acc[1] = __ffma2_rn(ww, make_float2(__uint_as_float(d.y << 16), __uint_as_float(d.y & 0xffff0000u)), acc[1]);
+        acc[2] = __ffma2_rn(ww, make_float2(__uint_as_float(d.z << 16), __uint_as_float(d.z & 0xffff0000u)), acc[2]);
+        acc[3] = __ffma2_rn(ww, make_float2(__uint_as_float(d.w << 16), __uint_as_float(d.w & 0xffff0000u)), acc[3]);
     }
 };
 
 template <bool BF16, int V>
-__global__ void __launch_bounds__(kThreads) sample_forward_kernel(const SampleArgs a) {
-    using CK = Chunk<BF16>;
-    constexpr int CH = CK::kCh;
+using Acc = float2[V][Chunk<BF16>::kPairs];
+
+// One texel: acc += w * F[texel, lane chunks].
+template <bool BF16, int L, int V>
+__device__ __forceinline__ void accumulate_texel(Acc<BF16, V>& acc, const uint4* p, float w, int ql,
+                                                 int nchunks) {
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+        if (ql + v * L < nchunks) Chunk<BF16>::fma(acc[v], __ldg(p + v * L), w);
+}
+
+// Texels visited per step of the merged walk: their loads are all issued
+// before any of their FMAs, so each lane keeps kUnroll * V loads in flight.
+constexpr int kUnroll = 4;
+
+// Merged path: walk the (cell, camera) patch in row-major order.  The trip
+// count is the warp's longest patch; shorter patches of the other cells of
+// the warp are predicated off.
+template <bool BF16, int L, int V>
+__device__ __forceinline__ void gather_patch(Acc<BF16, V>& acc, const float* pf, const int4 pi,
+                                             const uint4* Fn, int Wf, int Qtot, int ql, int nchunks) {
+    const int w = pi.z & 0xffff;
+    const int n = (pi.z >> 16) * w;
+    const int nmax = __reduce_max_sync(0xffffffffu, n);
+    const float inv_w = 1.0f / (float)max(w, 1);
+    const float* pw = pf + pi.w;
+    const uint4* base = Fn + ((size_t)pi.x * Wf + pi.y) * Qtot;
+    for (int e0 = 0; e0 < nmax; e0 += kUnroll) {
+        float wt[kUnroll];
+        const uint4* pp[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int e = e0 + u;
+            const int r = __float2int_rz(((float)e + 0.5f) * inv_w);  // e / w, exact for e < 2^16
+            wt[u] = e < n ? pw[e] : 0.0f;
+            pp[u] = base + ((size_t)r * Wf + (e - r * w)) * Qtot;
+        }
+        uint4 d[kUnroll][V];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+            for (int v = 0; v < V; ++v)
+                d[u][v] = (wt[u] != 0.0f && ql + v * L < nchunks) ? __ldg(pp[u] + v * L) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+            for (int v = 0; v < V; ++v) Chunk<BF16>::fma(acc[v], d[u][v], wt[u]);
+    }
+}
+
+// Merged path over the shared-memory copy of the camera's texel window
+// (window origin (wy0, wx0), ww texels wide, Q chunks per texel).
+template <bool BF16, int L, int V>
+__device__ __forceinline__ void gather_patch_staged(Acc<BF16, V>& acc, const float* pf, const int4 pi,
+                                                    const uint4* st, int wy0, int wx0, int ww, int Q, int ql,
+                                                    int nchunks) {
+    const int w = pi.z & 0xffff;
+    const int n = (pi.z >> 16) * w;
+    const int nmax = __reduce_max_sync(0xffffffffu, n);
+    const float inv_w = 1.0f / (float)max(w, 1);
+    const float* pw = pf + pi.w;
+    const uint4* base = st + ((pi.x - wy0) * ww + (pi.y - wx0)) * Q + ql;
+    for (int e0 = 0; e0 < nmax; e0 += kUnroll) {
+        float wt[kUnroll];
+        const uint4* pp[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int e = e0 + u;
+            const int r = __float2int_rz(((float)e + 0.5f) * inv_w);
+            wt[u] = e < n ? pw[e] : 0.0f;
+            pp[u] = base + (r * ww + (e - r * w)) * Q;
+        }
+        uint4 d[kUnroll][V];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+            for (int v = 0; v < V; ++v)
+                d[u][v] = (wt[u] != 0.0f && ql + v * L < nchunks) ? pp[u][v * L] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+            for (int v = 0; v < V; ++v) Chunk<BF16>::fma(acc[v], d[u][v], wt[u]);
+    }
+}
+
+// Copy the texel window [wn.x, wn.y] x [wn.z, wn.w] of one camera (all Q
+// chunks of each texel; rows are contiguous in the channels-last map) into
+// shared memory with 16-byte asynchronous copies that bypass L1.  Ends with a
+// CTA barrier once every copy has landed.
+__device__ __forceinline__ void stage_window(uint4* st, const uint4* Fn, const int4 wn, int Wf, int Q) {
+    const int ww = wn.w - wn.z + 1;
+    const int rowchunks = ww * Q;
+    const int total = (wn.y - wn.x + 1) * rowchunks;
+    const float inv_row = 1.0f / (float)rowchunks;
+    for (int k = threadIdx.x; k < total; k += kThreads) {
+        const int r = __float2int_rz(((float)k + 0.5f) * inv_row);  // k / rowchunks, exact here
+        const uint4* src = Fn + ((size_t)(wn.x + r) * Wf + wn.z) * Q + (k - r * rowchunks);
+        const unsigned dst = (unsigned)__cvta_generic_to_shared(st + k);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+}
+
+// Unmerged path for a camera whose patches do not fit: corners straight from (fx, fy).
+template <bool BF16, int L, int V>
+__device__ __forceinline__ void gather_direct(Acc<BF16, V>& acc, const TileSmem& s, int cell, int aa,
+                                              int zlen, const uint4* Fn, int Hf, int Wf, int Qtot, int ql,
+                                              int nchunks) {
+    for (int zl = 0; zl < zlen; ++zl) {
+        const float2 f = s.items[item_index(cell, aa, zl, zlen)];
+        if (!(f.x == f.x)) continue;
+        const float cntf = (float)cell_count(s.cnt, zl, cell);
+        const Corners c = bilinear_corners(f.x, f.y);
+        const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
+            if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
+            accumulate_texel<BF16, L, V>(acc, Fn + ((size_t)yy * Wf + xx) * Qtot, __fdiv_rn(ws[k], cntf), ql,
+                                         nchunks);
+        }
+    }
+}
+
+template <bool BF16, int L, int V>
+__global__ void __launch_bounds__(kThreads, 3) sample_forward_kernel(const SampleArgs a) {
+    constexpr int P = Chunk<BF16>::kPairs;
+    constexpr int G = 32 / L;                // cells a warp works on at once
+    constexpr int CG = kCellsPerWarp / G;    // rounds of cells per warp
+    static_assert(G * CG == kCellsPerWarp, "lanes per cell must be 4, 8, 16 or 32");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const TileSmem s = carve_smem(smem_raw, a.N);
     const GeoParams& g = a.g;
 
     const int b = blockIdx.y;
-    const int ti0 = (blockIdx.x / a.tiles_j) * kTileI;
-    const int tj0 = (blockIdx.x % a.tiles_j) * kTileJ;
+    int ti0, tj0;
+    tile_origin(a, ti0, tj0);
     const int chunk0 = blockIdx.z * a.slice_chunks;
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
-    const int cs = nchunks * CH;
 
-    for (int t = threadIdx.x; t < cs * kObufStride; t += kThreads) s.obuf[t] = 0.0f;
     setup_tile(a, s, b, ti0, tj0);
     const int nA = s.act[32];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int L = a.L, G = 32 / L;
     const int sub = lane / L, ql = lane - sub * L;
     const bool write_count = a.count != nullptr && blockIdx.z == 0;
+    const size_t texels = (size_t)g.Hf * g.Wf;
+    const uint4* feat = reinterpret_cast<const uint4*>(a.feat) + chunk0 + ql;
+
+    float2 acc[CG][V][P];
+#pragma unroll
+    for (int q = 0; q < CG; ++q)
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+#pragma unroll
+            for (int e = 0; e < P; ++e) acc[q][v][e] = make_float2(0.0f, 0.0f);
 
     if (nA == 0) {
         if (write_count) store_counts(a, nullptr, b, ti0, tj0, 0, g.Z);
     } else {
-        const int zc = z_chunk(g.Z, nA);
-        const size_t texels = (size_t)g.Hf * g.Wf;
-        for (int z0 = 0; z0 < g.Z; z0 += zc) {
+        int zc = z_chunk(g.Z, nA);
+        int z0 = 0;
+        while (z0 < g.Z) {
             const int zlen = min(zc, g.Z - z0);
             geometry_chunk(a, s, ti0, tj0, nA, z0, zlen);
+            int total = layout_patches(a, s, zlen, 0, nA);
+            if (total < 0 && zlen > 1) {  // too many texels: fewer bins per chunk
+                zc = (zlen + 1) / 2;
+                continue;
+            }
             if (write_count) store_counts(a, s.cnt, b, ti0, tj0, z0, zlen);
-
-            for (int cg = warp; cg * G < kTile; cg += kWarps) {
-                const int cell = cg * G + sub;
-                float acc[V][CH];
-#pragma unroll
-                for (int v = 0; v < V; ++v)
-#pragma unroll
-                    for (int e = 0; e < CH; ++e) acc[v][e] = 0.0f;
-
-                for (int aa = 0; aa < nA; ++aa) {
-                    const int n = s.act[aa];
-                    const uint4* Fn = reinterpret_cast<const uint4*>(a.feat) +
-                                      ((size_t)b * a.N + n) * texels * a.Qtot + chunk0 + ql;
-                    const float2* it = s.items + (cell * nA + aa) * zlen;
-                    const int* cn = s.cnt + cell * zlen;
-                    for (int zl = 0; zl < zlen; ++zl) {
-                        const float2 f = it[zl];
-                        if (!(f.x == f.x)) continue;  // camera not valid for this voxel
-                        const float sc = __frcp_rn((float)cn[zl]);
-                        const Corners c = bilinear_corners(f.x, f.y);
-                        const bool x0in = (unsigned)c.x0 < (unsigned)g.Wf;
-                        const bool x1in = (unsigned)(c.x0 + 1) < (unsigned)g.Wf;
-                        const bool y0in = (unsigned)c.y0 < (unsigned)g.Hf;
-                        const bool y1in = (unsigned)(c.y0 + 1) < (unsigned)g.Hf;
-                        const uint4* p00 = Fn + ((long long)c.y0 * g.Wf + c.x0) * a.Qtot;
-                        const size_t row = (size_t)g.Wf * a.Qtot;
-#pragma unroll
-                        for (int v = 0; v < V; ++v) {
-                            if (ql + v * L < nchunks) {
-                                const int o = v * L;
-                                if (y0in && x0in) CK::fma(acc[v], __ldg(p00 + o), c.w00 * sc);
-                                if (y0in && x1in) CK::fma(acc[v], __ldg(p00 + a.Qtot + o), c.w01 * sc);
-                                if (y1in && x0in) CK::fma(acc[v], __ldg(p00 + row + o), c.w10 * sc);
-                                if (y1in && x1in)
-                                    CK::fma(acc[v], __ldg(p00 + row + a.Qtot + o), c.w11 * sc);
-                            }
-                        }
-                    }
+            int a0 = 0, ga = nA;
+            while (a0 < nA) {
+                const int a1 = min(nA, a0 + ga);
+                if (a0 > 0 || a1 < nA) total = layout_patches(a, s, zlen, a0, a1);
+                if (total < 0 && a1 - a0 > 1) {  // still too many: fewer cameras at once
+                    ga = (a1 - a0 + 1) / 2;
+                    continue;
                 }
-                // fold into the staging tile; each (channel, cell) has exactly one owner lane
+                if (total >= 0) fill_patches(a, s, zlen, a0, a1);
+                const float* pf = s.patch;
+                for (int aa = a0; aa < a1; ++aa) {
+                    const uint4* Fn = feat + ((size_t)b * a.N + s.act[aa]) * texels * a.Qtot;
+                    const int4 wn = s.win[aa];
+                    const int wh = wn.y - wn.x + 1, ww = wn.w - wn.z + 1;
+                    // whole channel vectors of the window fit in shared memory: gather from there
+                    const bool staged = total >= 0 && nchunks == a.Qtot && wh > 0 &&
+                                        wh * ww * a.Qtot <= kStageChunks;
+                    if (staged)
+                        stage_window(s.stage, reinterpret_cast<const uint4*>(a.feat) +
+                                                  ((size_t)b * a.N + s.act[aa]) * texels * a.Qtot,
+                                     wn, g.Wf, a.Qtot);
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    const int q = ql + v * L;
-                    if (q < nchunks) {
-#pragma unroll
-                        for (int e = 0; e < CH; ++e) s.obuf[(q * CH + e) * kObufStride + cell] += acc[v][e];
+                    for (int q = 0; q < CG; ++q) {
+                        const int cell = warp * kCellsPerWarp + q * G + sub;
+                        if (staged)
+                            gather_patch_staged<BF16, L, V>(acc[q], pf, s.pinfo[aa * kTile + cell], s.stage, wn.x,
+                                                            wn.z, ww, a.Qtot, ql, nchunks);
+                        else if (total >= 0)
+                            gather_patch<BF16, L, V>(acc[q], pf, s.pinfo[aa * kTile + cell], Fn, g.Wf, a.Qtot,
+                                                     ql, nchunks);
+                        else
+                            gather_direct<BF16, L, V>(acc[q], s, cell, aa, zlen, Fn, g.Hf, g.Wf, a.Qtot, ql,
+                                                      nchunks);
                     }
+                    if (staged) __syncthreads();  // the next camera reuses the window buffer
+                }
+                __syncthreads();  // patches are rebuilt by the next camera group / chunk
+                a0 = a1;
+                total = -1;
+            }
+            z0 += zlen;
+        }
+    }
+    __syncthreads();
+    // stage [channel][cell] (aliases the geometry buffers), then store rows along y
+#pragma unroll
+    for (int q = 0; q < CG; ++q) {
+        const int cell = warp * kCellsPerWarp + q * G + sub;
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            const int cq = ql + v * L;
+            if (cq < nchunks) {
+#pragma unroll
+                for (int e = 0; e < P; ++e) {
+                    s.obuf[(cq * 2 * P + 2 * e) * kObufStride + cell] = acc[q][v][e].x;
+                    s.obuf[(cq * 2 * P + 2 * e + 1) * kObufStride + cell] = acc[q][v][e].y;
                 }
             }
         }
     }
     __syncthreads();
-    const int c_base = chunk0 * CH;
-    const int c_real = max(0, min(cs, a.C - c_base));
+    const int c_base = chunk0 * 2 * P;
+    const int c_real = max(0, min(nchunks * 2 * P, a.C - c_base));
     for (int t = threadIdx.x; t < c_real * kTile; t += kThreads) {
         const int c = t / kTile, cell = t - c * kTile;
         const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
@@ -144,29 +290,48 @@ __global__ void __launch_bounds__(kThreads) sample_forward_kernel(const SampleAr
     }
 }
 
-template <bool BF16>
-static cudaError_t launch_fwd_v(const SampleArgs& a, int V, dim3 grid, size_t smem, cudaStream_t st) {
-    switch (V) {
-#define BEV_FWD_CASE(VV)                                                                        \
-    case VV: {                                                                                  \
-        auto k = sample_forward_kernel<BF16, VV>;                                               \
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,    \
-                                             (int)smem);                                        \
-        if (e != cudaSuccess) return e;                                                         \
-        k<<<grid, kThreads, smem, st>>>(a);                                                     \
-        return cudaGetLastError();                                                              \
+template <bool BF16, int L, int V>
+static cudaError_t launch_one(const SampleArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
+    auto k = sample_forward_kernel<BF16, L, V>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+// (L, V) combinations the host's lane picker can produce: L * V <= 32 chunks
+// for fp32 slices, <= 16 for bf16 slices (128 channels either way).
+static cudaError_t launch_fwd_f32(const SampleArgs& a, int V, dim3 grid, size_t smem, cudaStream_t st) {
+    switch (a.L * 16 + V) {
+        case 32 * 16 + 1: return launch_one<false, 32, 1>(a, grid, smem, st);
+        case 16 * 16 + 1: return launch_one<false, 16, 1>(a, grid, smem, st);
+        case 16 * 16 + 2: return launch_one<false, 16, 2>(a, grid, smem, st);
+        case 8 * 16 + 1: return launch_one<false, 8, 1>(a, grid, smem, st);
+        case 8 * 16 + 2: return launch_one<false, 8, 2>(a, grid, smem, st);
+        case 8 * 16 + 3: return launch_one<false, 8, 3>(a, grid, smem, st);
+        case 8 * 16 + 4: return launch_one<false, 8, 4>(a, grid, smem, st);
+        case 4 * 16 + 1: return launch_one<false, 4, 1>(a, grid, smem, st);
+        case 4 * 16 + 2: return launch_one<false, 4, 2>(a, grid, smem, st);
+        case 4 * 16 + 3: return launch_one<false, 4, 3>(a, grid, smem, st);
+        case 4 * 16 + 4: return launch_one<false, 4, 4>(a, grid, smem, st);
+        case 4 * 16 + 5: return launch_one<false, 4, 5>(a, grid, smem, st);
+        case 4 * 16 + 6: return launch_one<false, 4, 6>(a, grid, smem, st);
+        case 4 * 16 + 7: return launch_one<false, 4, 7>(a, grid, smem, st);
+        case 4 * 16 + 8: return launch_one<false, 4, 8>(a, grid, smem, st);
+        default: return cudaErrorInvalidValue;
     }
-        BEV_FWD_CASE(1)
-        BEV_FWD_CASE(2)
-        BEV_FWD_CASE(3)
-        BEV_FWD_CASE(4)
-        BEV_FWD_CASE(5)
-        BEV_FWD_CASE(6)
-        BEV_FWD_CASE(7)
-        BEV_FWD_CASE(8)
-#undef BEV_FWD_CASE
-        default:
-            return cudaErrorInvalidValue;
+}
+
+static cudaError_t launch_fwd_bf16(const SampleArgs& a, int V, dim3 grid, size_t smem, cudaStream_t st) {
+    switch (a.L * 16 + V) {
+        case 16 * 16 + 1: return launch_one<true, 16, 1>(a, grid, smem, st);
+        case 8 * 16 + 1: return launch_one<true, 8, 1>(a, grid, smem, st);
+        case 8 * 16 + 2: return launch_one<true, 8, 2>(a, grid, smem, st);
+        case 4 * 16 + 1: return launch_one<true, 4, 1>(a, grid, smem, st);
+        case 4 * 16 + 2: return launch_one<true, 4, 2>(a, grid, smem, st);
+        case 4 * 16 + 3: return launch_one<true, 4, 3>(a, grid, smem, st);
+        case 4 * 16 + 4: return launch_one<true, 4, 4>(a, grid, smem, st);
+        default: return cudaErrorInvalidValue;
     }
 }
 
@@ -174,9 +339,8 @@ static cudaError_t launch_fwd_v(const SampleArgs& a, int V, dim3 grid, size_t sm
 
 cudaError_t bev_launch_forward(const bev::SampleArgs& a, bool bf16, int V, int slices,
                                cudaStream_t stream) {
-    const int tiles_i = (a.g.X + bev::kTileI - 1) / bev::kTileI;
-    const dim3 grid(tiles_i * a.tiles_j, a.B, slices);
+    const dim3 grid(a.tiles_i * a.tiles_j, a.B, slices);
     const size_t smem = bev::sample_smem_bytes(a.N);
-    return bf16 ? bev::launch_fwd_v<true>(a, V, grid, smem, stream)
-                : bev::launch_fwd_v<false>(a, V, grid, smem, stream);
+    return bf16 ? bev::launch_fwd_bf16(a, V, grid, smem, stream)
+                : bev::launch_fwd_f32(a, V, grid, smem, stream);
 }

@@ -90,7 +90,7 @@ def test_forward_channels_last_input(name):
     K, E = I.make_rigs(w)
     out_nhwc, _ = gpu_forward(F, K, E, w.img_h, w.img_w, w.ranges, w.res, layout=ops.NHWC)
     out_nchw, _ = gpu_forward(F, K, E, w.img_h, w.img_w, w.ranges, w.res, layout=ops.NCHW)
-    assert torch.equal(out_nhwc, out_nchw)
+    assert torch.equal(out_nhwc, out_nchw)   # same kernel, same order: bitwise equal
 
 
 def test_backward_workload_full_size():
@@ -186,6 +186,21 @@ def test_thirty_two_cameras_force_height_chunks():
     assert cnt.max() >= 4
     dout = torch.randn((1, 8, 24, 24), generator=torch.Generator().manual_seed(33))
     check_backward(dout, K, E, 64, 160, ranges, res, 32, 8, 20)
+
+
+def test_tall_patches_take_the_unmerged_path():
+    """One camera close to a fine column of 32 bins with a tall feature map:
+    each cell's bins span the whole map height, so the merged patches of a
+    tile exceed shared memory and the kernels fall back to unmerged taps."""
+    K = np.array([[[[448.0, 0, 320], [0, 448.0, 128], [0, 0, 1]]]], np.float32)
+    E = np.array([[[[0, -1, 0, 0], [0, 0, -1, 0], [1, 0, 0, 0], [0, 0, 0, 1]]]], np.float32)
+    K, E = torch.from_numpy(K), torch.from_numpy(E)
+    F = torch.randn((1, 1, 8, 64, 160), generator=torch.Generator().manual_seed(41))
+    ranges, res = (1.5, 5.5, -1.0, 1.0, -2.0, 2.0), (0.25, 0.25, 0.125)
+    out, ref, cnt, _ = check_forward(F, K, E, 256, 640, ranges, res, 1e-5)
+    assert cnt.sum() > 1000
+    dout = torch.randn((1, 8, 16, 8), generator=torch.Generator().manual_seed(42))
+    check_backward(dout, K, E, 256, 640, ranges, res, 1, 64, 160)
 
 
 def test_empty_view_gives_zeros():
