@@ -67,46 +67,58 @@ __device__ __forceinline__ void scatter_direct(const float (&d)[V][4], const Til
 }
 
 template <int L, int V>
-__global__ void __launch_bounds__(kThreads, 2) sample_backward_kernel(const SampleArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(const SampleArgs a) {
     constexpr int G = 32 / L;
     constexpr int CG = kCellsPerWarp / G;
     static_assert(G * CG == kCellsPerWarp, "lanes per cell must be 4, 8, 16 or 32");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const TileSmem s = carve_smem(smem_raw, a.N);
-    float* dbuf = reinterpret_cast<float*>(smem_raw + sample_smem_bytes(a.N));
     const GeoParams& g = a.g;
 
     const int b = blockIdx.y;
     int ti0, tj0;
-    tile_origin(a, ti0, tj0);
+    tile_origin(a, s.act + 40, ti0, tj0);
     const int chunk0 = blockIdx.z * a.slice_chunks;
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
     const int c_base = chunk0 * 4;
 
-    // stage dout[b, c_base + c, tile] as [c][cell]; padding channels read as 0
-    for (int t = threadIdx.x; t < nchunks * 4 * kTile; t += kThreads) {
-        const int c = t / kTile, cell = t - c * kTile;
-        const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
-        float v = 0.0f;
-        if (c_base + c < a.C && i < g.X && j < g.Y)
-            v = a.dout[(((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + j];
-        dbuf[c * kObufStride + cell] = v;
-    }
     setup_tile(a, s, b, ti0, tj0);
     const int nA = s.act[32];
     if (nA == 0) return;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / L, ql = lane - sub * L;
+    // Upstream gradient of the tile into registers, kGroupCh channels at a time
+    // through the [channel][cell] staging tile (loads coalesced along y).
     float d[CG][V][4];
 #pragma unroll
-    for (int q = 0; q < CG; ++q) {
-        const int cell = warp * kCellsPerWarp + q * G + sub;
+    for (int q = 0; q < CG; ++q)
 #pragma unroll
-        for (int v = 0; v < V; ++v) {
-            const int cq = ql + v * L;
+        for (int v = 0; v < V; ++v)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) d[q][v][e] = cq < nchunks ? dbuf[(cq * 4 + e) * kObufStride + cell] : 0.0f;
+            for (int e = 0; e < 4; ++e) d[q][v][e] = 0.0f;
+    for (int g0 = 0; g0 < nchunks * 4; g0 += kGroupCh) {
+        __syncthreads();
+        for (int t = threadIdx.x; t < kGroupCh * kTile; t += kThreads) {
+            const int c = t / kTile, cell = t - c * kTile;
+            const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
+            float v = 0.0f;
+            if (g0 + c < nchunks * 4 && c_base + g0 + c < a.C && i < g.X && j < g.Y)
+                v = a.dout[(((size_t)b * a.C + c_base + g0 + c) * g.X + i) * g.Y + j];
+            s.obuf[c * kObufStride + cell] = v;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < CG; ++q) {
+            const int cell = warp * kCellsPerWarp + q * G + sub;
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const int c0 = (ql + v * L) * 4 - g0;
+                if (c0 >= 0 && c0 < kGroupCh) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) d[q][v][e] = s.obuf[(c0 + e) * kObufStride + cell];
+                }
+            }
         }
     }
     const size_t texels = (size_t)g.Hf * g.Wf;
@@ -156,6 +168,8 @@ template <int L, int V>
 static cudaError_t launch_one(const SampleArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
     auto k = sample_backward_kernel<L, V>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, carveout_percent(smem));
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, smem, st>>>(a);
     return cudaGetLastError();
@@ -186,5 +200,5 @@ static cudaError_t launch_bwd(const SampleArgs& a, int V, dim3 grid, size_t smem
 
 cudaError_t bev_launch_backward(const bev::SampleArgs& a, int V, int slices, cudaStream_t stream) {
     const dim3 grid(a.tiles_i * a.tiles_j, a.B, slices);
-    return bev::launch_bwd(a, V, grid, bev::sample_smem_bytes_bwd(a.N), stream);
+    return bev::launch_bwd(a, V, grid, bev::sample_smem_bytes(a.N), stream);
 }

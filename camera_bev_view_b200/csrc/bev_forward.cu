@@ -57,98 +57,38 @@ __device__ __forceinline__ void accumulate_texel(Acc<BF16, V>& acc, const uint4*
         if (ql + v * L < nchunks) Chunk<BF16>::fma(acc[v], __ldg(p + v * L), w);
 }
 
-// Texels visited per step of the merged walk: their loads are all issued
-// before any of their FMAs, so each lane keeps kUnroll * V loads in flight.
-constexpr int kUnroll = 4;
-
-// Merged path: walk the (cell, camera) patch in row-major order.  The trip
-// count is the warp's longest patch; shorter patches of the other cells of
-// the warp are predicated off.
+// Merged path: walk the (cell, camera) patch two rows by two columns per
+// step (patches are mostly two texels wide: a vertical column of voxels
+// projects to a near-vertical line).  The trip counts are the warp's largest
+// patch; the other cells of the warp are predicated off past their own.
 template <bool BF16, int L, int V>
 __device__ __forceinline__ void gather_patch(Acc<BF16, V>& acc, const float* pf, const int4 pi,
                                              const uint4* Fn, int Wf, int Qtot, int ql, int nchunks) {
-    const int w = pi.z & 0xffff;
-    const int n = (pi.z >> 16) * w;
-    const int nmax = __reduce_max_sync(0xffffffffu, n);
-    const float inv_w = 1.0f / (float)max(w, 1);
-    const float* pw = pf + pi.w;
-    const uint4* base = Fn + ((size_t)pi.x * Wf + pi.y) * Qtot;
-    for (int e0 = 0; e0 < nmax; e0 += kUnroll) {
-        float wt[kUnroll];
-        const uint4* pp[kUnroll];
+    const int h = pi.z >> 16, w = pi.z & 0xffff;
+    const int hmax = __reduce_max_sync(0xffffffffu, h);
+    const int wmax = __reduce_max_sync(0xffffffffu, w);
+    const size_t rstride = (size_t)Wf * Qtot;
+    for (int c0 = 0; c0 < wmax; c0 += 2) {
+        const bool c0in = c0 < w, c1in = c0 + 1 < w;
+        const float* pw = pf + pi.w + c0;
+        const uint4* rp = Fn + ((size_t)pi.x * Wf + pi.y + c0) * Qtot;
+        for (int r0 = 0; r0 < hmax; r0 += 2, pw += 2 * w, rp += 2 * rstride) {
+            const bool r0in = r0 < h, r1in = r0 + 1 < h;
+            const float wt[4] = {(r0in && c0in) ? pw[0] : 0.0f, (r0in && c1in) ? pw[1] : 0.0f,
+                                 (r1in && c0in) ? pw[w] : 0.0f, (r1in && c1in) ? pw[w + 1] : 0.0f};
+            const uint4* pp[4] = {rp, rp + Qtot, rp + rstride, rp + rstride + Qtot};
+            uint4 d[4][V];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int e = e0 + u;
-            const int r = __float2int_rz(((float)e + 0.5f) * inv_w);  // e / w, exact for e < 2^16
-            wt[u] = e < n ? pw[e] : 0.0f;
-            pp[u] = base + ((size_t)r * Wf + (e - r * w)) * Qtot;
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < V; ++v)
+                    d[u][v] = (wt[u] != 0.0f && ql + v * L < nchunks) ? __ldg(pp[u] + v * L) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < V; ++v) Chunk<BF16>::fma(acc[v], d[u][v], wt[u]);
         }
-        uint4 d[kUnroll][V];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-#pragma unroll
-            for (int v = 0; v < V; ++v)
-                d[u][v] = (wt[u] != 0.0f && ql + v * L < nchunks) ? __ldg(pp[u] + v * L) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-#pragma unroll
-            for (int v = 0; v < V; ++v) Chunk<BF16>::fma(acc[v], d[u][v], wt[u]);
     }
-}
-
-// Merged path over the shared-memory copy of the camera's texel window
-// (window origin (wy0, wx0), ww texels wide, Q chunks per texel).
-template <bool BF16, int L, int V>
-__device__ __forceinline__ void gather_patch_staged(Acc<BF16, V>& acc, const float* pf, const int4 pi,
-                                                    const uint4* st, int wy0, int wx0, int ww, int Q, int ql,
-                                                    int nchunks) {
-    const int w = pi.z & 0xffff;
-    const int n = (pi.z >> 16) * w;
-    const int nmax = __reduce_max_sync(0xffffffffu, n);
-    const float inv_w = 1.0f / (float)max(w, 1);
-    const float* pw = pf + pi.w;
-    const uint4* base = st + ((pi.x - wy0) * ww + (pi.y - wx0)) * Q + ql;
-    for (int e0 = 0; e0 < nmax; e0 += kUnroll) {
-        float wt[kUnroll];
-        const uint4* pp[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int e = e0 + u;
-            const int r = __float2int_rz(((float)e + 0.5f) * inv_w);
-            wt[u] = e < n ? pw[e] : 0.0f;
-            pp[u] = base + (r * ww + (e - r * w)) * Q;
-        }
-        uint4 d[kUnroll][V];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-#pragma unroll
-            for (int v = 0; v < V; ++v)
-                d[u][v] = (wt[u] != 0.0f && ql + v * L < nchunks) ? pp[u][v * L] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-#pragma unroll
-            for (int v = 0; v < V; ++v) Chunk<BF16>::fma(acc[v], d[u][v], wt[u]);
-    }
-}
-
-// Copy the texel window [wn.x, wn.y] x [wn.z, wn.w] of one camera (all Q
-// chunks of each texel; rows are contiguous in the channels-last map) into
-// shared memory with 16-byte asynchronous copies that bypass L1.  Ends with a
-// CTA barrier once every copy has landed.
-__device__ __forceinline__ void stage_window(uint4* st, const uint4* Fn, const int4 wn, int Wf, int Q) {
-    const int ww = wn.w - wn.z + 1;
-    const int rowchunks = ww * Q;
-    const int total = (wn.y - wn.x + 1) * rowchunks;
-    const float inv_row = 1.0f / (float)rowchunks;
-    for (int k = threadIdx.x; k < total; k += kThreads) {
-        const int r = __float2int_rz(((float)k + 0.5f) * inv_row);  // k / rowchunks, exact here
-        const uint4* src = Fn + ((size_t)(wn.x + r) * Wf + wn.z) * Q + (k - r * rowchunks);
-        const unsigned dst = (unsigned)__cvta_generic_to_shared(st + k);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
 }
 
 // Unmerged path for a camera whose patches do not fit: corners straight from (fx, fy).
@@ -173,7 +113,7 @@ __device__ __forceinline__ void gather_direct(Acc<BF16, V>& acc, const TileSmem&
 }
 
 template <bool BF16, int L, int V>
-__global__ void __launch_bounds__(kThreads, 3) sample_forward_kernel(const SampleArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(const SampleArgs a) {
     constexpr int P = Chunk<BF16>::kPairs;
     constexpr int G = 32 / L;                // cells a warp works on at once
     constexpr int CG = kCellsPerWarp / G;    // rounds of cells per warp
@@ -184,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 3) sample_forward_kernel(const Sampl
 
     const int b = blockIdx.y;
     int ti0, tj0;
-    tile_origin(a, ti0, tj0);
+    tile_origin(a, s.act + 40, ti0, tj0);
     const int chunk0 = blockIdx.z * a.slice_chunks;
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
 
@@ -227,33 +167,24 @@ __global__ void __launch_bounds__(kThreads, 3) sample_forward_kernel(const Sampl
                     ga = (a1 - a0 + 1) / 2;
                     continue;
                 }
-                if (total >= 0) fill_patches(a, s, zlen, a0, a1);
+                if (total >= 0) {
+                    prefetch_windows(s, reinterpret_cast<const uint4*>(a.feat) + (size_t)b * a.N * texels * a.Qtot,
+                                     texels * a.Qtot, g.Wf, a.Qtot, chunk0, nchunks, a0, a1);
+                    fill_patches(a, s, zlen, a0, a1);
+                }
                 const float* pf = s.patch;
-                for (int aa = a0; aa < a1; ++aa) {
-                    const uint4* Fn = feat + ((size_t)b * a.N + s.act[aa]) * texels * a.Qtot;
-                    const int4 wn = s.win[aa];
-                    const int wh = wn.y - wn.x + 1, ww = wn.w - wn.z + 1;
-                    // whole channel vectors of the window fit in shared memory: gather from there
-                    const bool staged = total >= 0 && nchunks == a.Qtot && wh > 0 &&
-                                        wh * ww * a.Qtot <= kStageChunks;
-                    if (staged)
-                        stage_window(s.stage, reinterpret_cast<const uint4*>(a.feat) +
-                                                  ((size_t)b * a.N + s.act[aa]) * texels * a.Qtot,
-                                     wn, g.Wf, a.Qtot);
 #pragma unroll
-                    for (int q = 0; q < CG; ++q) {
-                        const int cell = warp * kCellsPerWarp + q * G + sub;
-                        if (staged)
-                            gather_patch_staged<BF16, L, V>(acc[q], pf, s.pinfo[aa * kTile + cell], s.stage, wn.x,
-                                                            wn.z, ww, a.Qtot, ql, nchunks);
-                        else if (total >= 0)
+                for (int q = 0; q < CG; ++q) {
+                    const int cell = warp * kCellsPerWarp + q * G + sub;
+                    for (int aa = a0; aa < a1; ++aa) {
+                        const uint4* Fn = feat + ((size_t)b * a.N + s.act[aa]) * texels * a.Qtot;
+                        if (total >= 0)
                             gather_patch<BF16, L, V>(acc[q], pf, s.pinfo[aa * kTile + cell], Fn, g.Wf, a.Qtot,
                                                      ql, nchunks);
                         else
                             gather_direct<BF16, L, V>(acc[q], s, cell, aa, zlen, Fn, g.Hf, g.Wf, a.Qtot, ql,
                                                       nchunks);
                     }
-                    if (staged) __syncthreads();  // the next camera reuses the window buffer
                 }
                 __syncthreads();  // patches are rebuilt by the next camera group / chunk
                 a0 = a1;
@@ -262,31 +193,36 @@ __global__ void __launch_bounds__(kThreads, 3) sample_forward_kernel(const Sampl
             z0 += zlen;
         }
     }
-    __syncthreads();
-    // stage [channel][cell] (aliases the geometry buffers), then store rows along y
+    // Store: kGroupCh channels at a time through the [channel][cell] staging
+    // tile (it aliases the geometry buffers), rows along y, the contiguous
+    // axis of out.  A 16-byte chunk (2P channels) never straddles a group.
+    const int c_base = chunk0 * 2 * P;
+    const int c_real = max(0, min(nchunks * 2 * P, a.C - c_base));
+    for (int g0 = 0; g0 < c_real; g0 += kGroupCh) {
+        __syncthreads();
 #pragma unroll
-    for (int q = 0; q < CG; ++q) {
-        const int cell = warp * kCellsPerWarp + q * G + sub;
+        for (int q = 0; q < CG; ++q) {
+            const int cell = warp * kCellsPerWarp + q * G + sub;
 #pragma unroll
-        for (int v = 0; v < V; ++v) {
-            const int cq = ql + v * L;
-            if (cq < nchunks) {
+            for (int v = 0; v < V; ++v) {
+                const int c0 = (ql + v * L) * 2 * P - g0;
+                if (ql + v * L < nchunks && c0 >= 0 && c0 < kGroupCh) {
 #pragma unroll
-                for (int e = 0; e < P; ++e) {
-                    s.obuf[(cq * 2 * P + 2 * e) * kObufStride + cell] = acc[q][v][e].x;
-                    s.obuf[(cq * 2 * P + 2 * e + 1) * kObufStride + cell] = acc[q][v][e].y;
+                    for (int e = 0; e < P; ++e) {
+                        s.obuf[(c0 + 2 * e) * kObufStride + cell] = acc[q][v][e].x;
+                        s.obuf[(c0 + 2 * e + 1) * kObufStride + cell] = acc[q][v][e].y;
+                    }
                 }
             }
         }
-    }
-    __syncthreads();
-    const int c_base = chunk0 * 2 * P;
-    const int c_real = max(0, min(nchunks * 2 * P, a.C - c_base));
-    for (int t = threadIdx.x; t < c_real * kTile; t += kThreads) {
-        const int c = t / kTile, cell = t - c * kTile;
-        const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
-        if (i < g.X && j < g.Y)
-            a.out[(((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + j] = s.obuf[c * kObufStride + cell];
+        __syncthreads();
+        const int gc = min(kGroupCh, c_real - g0);
+        for (int t = threadIdx.x; t < gc * kTile; t += kThreads) {
+            const int c = t / kTile, cell = t - c * kTile;
+            const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
+            if (i < g.X && j < g.Y)
+                a.out[(((size_t)b * a.C + c_base + g0 + c) * g.X + i) * g.Y + j] = s.obuf[c * kObufStride + cell];
+        }
     }
 }
 
@@ -294,6 +230,8 @@ template <bool BF16, int L, int V>
 static cudaError_t launch_one(const SampleArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
     auto k = sample_forward_kernel<BF16, L, V>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, carveout_percent(smem));
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, smem, st>>>(a);
     return cudaGetLastError();

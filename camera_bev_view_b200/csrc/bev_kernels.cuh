@@ -17,17 +17,24 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCellsPerWarp = kTile / kWarps;
 static_assert(kCellsPerWarp == kTileJ, "one warp per tile row");
-// (fx, fy) slots per height chunk: kTile * active cameras * bins.
+// (fx, fy) slots per height chunk: kTile * active cameras * bins.  At least one
+// bin of every camera must fit (a chunk never has fewer than one bin).
 constexpr int kItemCap = 2048;
+static_assert(kItemCap >= kTile * 32, "one height bin of 32 cameras must fit");
 // Merged-weight patch entries per height chunk (fp32 each).
-constexpr int kPatchCap = 4096;
+constexpr int kPatchCap = 2048;
 // Height bins per chunk at most (valid counts are packed one byte per cell).
 constexpr int kZChunkMax = 32;
-// Channels per CTA slice (the output staging tile holds kTile x kSliceMax floats).
+// Channels per CTA slice.
 constexpr int kSliceMax = 128;
-constexpr int kObufStride = kTile + 1;  // padded row of the [channel][cell] staging tile
-// Shared-memory copy of one camera's texel window for the tile, in 16-byte chunks.
-constexpr int kStageChunks = 2048;
+// The [channel][cell] staging tile used to move a tile's channel vectors
+// between registers and the y-contiguous rows of [B,C,X,Y] covers kGroupCh
+// channels at a time (it aliases the geometry buffers).
+constexpr int kGroupCh = 32;
+constexpr int kObufStride = kTile + 1;  // padded row of the staging tile
+// Shared memory per CTA stays small (~26 KB for 6 cameras) so that most of
+// the SM's 256 KB on-chip array serves as L1 for the tile's texel windows.
+constexpr int kCtasPerSm = 3;
 
 struct SampleArgs {
     const void* feat;       // channels-last [B*N][Hf*Wf][Qtot chunks of 16 bytes]
@@ -47,23 +54,41 @@ struct SampleArgs {
 };
 
 // Bytes of dynamic shared memory of one CTA (see carve_smem).
-__host__ __device__ inline size_t sample_smem_bytes(int N) {
+// Byte offsets of the per-CTA shared-memory regions (one source of truth for
+// the kernels' carve-up and the launch size).
+struct SmemLayout {
+    size_t items, patch, cnt, pinfo, win, cams, act, scan, total;
+};
+
+__host__ __device__ inline SmemLayout smem_layout(int N) {
+    SmemLayout l;
     size_t b = 0;
-    b += sizeof(float2) * kItemCap;                      // geometry slots
-    b += sizeof(float) * kPatchCap;                      // merged weights
-    b += (size_t)16 * kStageChunks;                      // texel window copy
-    b += sizeof(int) * (kTile / 4) * kZChunkMax;         // valid counts, one byte per (bin, cell)
-    b += sizeof(int4) * kTile * N;                       // patch box per (cell, active camera)
-    b += sizeof(int4) * 32;                              // texel window per active camera
-    b += sizeof(float) * ((N * kCamFloats + 3) & ~3);    // camera constants
-    b += sizeof(int) * 64;                               // active camera list, flags
-    b += sizeof(int) * 64;                               // scan scratch
-    return b;
+    l.items = b;  b += sizeof(float2) * kItemCap;                     // geometry slots
+    l.patch = b;  b += sizeof(float) * kPatchCap;                     // merged weights
+    l.cnt = b;    b += sizeof(int) * (kTile / 4) * kZChunkMax;        // valid counts, a byte per (bin, cell)
+    l.pinfo = b;  b += sizeof(int4) * kTile * N;                      // patch box per (cell, active camera)
+    l.win = b;    b += sizeof(int4) * 32;                             // texel window per active camera
+    l.cams = b;   b += sizeof(float) * ((N * kCamFloats + 3) & ~3);   // camera constants
+    l.act = b;    b += sizeof(int) * 64;                              // active camera list
+    l.scan = b;   b += sizeof(int) * 64;                              // scan scratch
+    l.total = b;
+    return l;
 }
 
-// The backward adds a [channel][cell] staging tile of its upstream gradient.
-__host__ __device__ inline size_t sample_smem_bytes_bwd(int N) {
-    return sample_smem_bytes(N) + sizeof(float) * kSliceMax * kObufStride;
+__host__ __device__ inline size_t sample_smem_bytes(int N) { return smem_layout(N).total; }
+
+static_assert(sizeof(float) * kGroupCh * kObufStride <= sizeof(float2) * kItemCap + sizeof(float) * kPatchCap,
+              "the staging tile aliases the geometry slots and the patches");
+
+// Preferred shared-memory carveout for kCtasPerSm CTAs of `smem` bytes each:
+// the smallest shared-memory configuration of the SM (KB) that holds them,
+// as a percentage of the 228 KB maximum; the rest of the array is L1.
+inline int carveout_percent(size_t smem) {
+    const int sizes_kb[] = {0, 8, 16, 32, 64, 100, 132, 164, 196, 228};
+    const size_t need = (size_t)kCtasPerSm * (smem + 1024);
+    for (int kb : sizes_kb)
+        if ((size_t)kb * 1024 >= need) return (100 * kb + 227) / 228;
+    return 100;
 }
 
 }  // namespace bev

@@ -28,11 +28,10 @@ namespace bev {
 struct TileSmem {
     float2* items;  // [kItemCap] (fx, fy) per (camera aa, bin zl, cell); fx = NaN: invalid
     float* patch;   // [kPatchCap] merged weights
-    uint4* stage;   // [kStageChunks] one camera's texel window, channels last
-    float* obuf;    // [kSliceMax][kObufStride], aliases items + patch + stage (forward epilogue)
+    float* obuf;    // [kGroupCh][kObufStride] channel-major staging tile, aliases items + patch
     int* cnt;       // [zl][cell / 4] valid cameras per (cell, bin), one byte each
     int4* pinfo;    // [aa][cell] patch (y0, x0, h << 16 | w, offset)
-    int4* win;      // [aa] texel window (ymin, ymax, xmin, xmax) of the tile
+    int4* win;      // [aa] union of the camera's texel boxes over the tile (ymin, ymax, xmin, xmax)
     float* cams;    // [N][kCamFloats]
     int* act;       // [0..nA) active camera ids; act[32] = nA
     int* scan;      // [64] block-scan scratch
@@ -44,47 +43,71 @@ __device__ __forceinline__ int cell_count(const int* cnt, int zl, int cell) {
 }
 
 __device__ __forceinline__ TileSmem carve_smem(unsigned char* smem, int N) {
+    const SmemLayout l = smem_layout(N);
     TileSmem s;
-    s.items = reinterpret_cast<float2*>(smem);
-    s.obuf = reinterpret_cast<float*>(smem);
-    smem += sizeof(float2) * kItemCap;
-    s.patch = reinterpret_cast<float*>(smem);
-    smem += sizeof(float) * kPatchCap;
-    s.stage = reinterpret_cast<uint4*>(smem);
-    smem += (size_t)16 * kStageChunks;
-    s.cnt = reinterpret_cast<int*>(smem);
-    smem += sizeof(int) * (kTile / 4) * kZChunkMax;
-    s.pinfo = reinterpret_cast<int4*>(smem);
-    smem += sizeof(int4) * kTile * N;
-    s.win = reinterpret_cast<int4*>(smem);
-    smem += sizeof(int4) * 32;
-    s.cams = reinterpret_cast<float*>(smem);
-    smem += sizeof(float) * ((N * kCamFloats + 3) & ~3);
-    s.act = reinterpret_cast<int*>(smem);
-    smem += sizeof(int) * 64;
-    s.scan = reinterpret_cast<int*>(smem);
+    s.items = reinterpret_cast<float2*>(smem + l.items);
+    s.obuf = reinterpret_cast<float*>(smem + l.items);
+    s.patch = reinterpret_cast<float*>(smem + l.patch);
+    s.cnt = reinterpret_cast<int*>(smem + l.cnt);
+    s.pinfo = reinterpret_cast<int4*>(smem + l.pinfo);
+    s.win = reinterpret_cast<int4*>(smem + l.win);
+    s.cams = reinterpret_cast<float*>(smem + l.cams);
+    s.act = reinterpret_cast<int*>(smem + l.act);
+    s.scan = reinterpret_cast<int*>(smem + l.scan);
     return s;
 }
 
-// k-th index of [0, T) in order of distance from the middle (middle first).
-__device__ __forceinline__ int middle_out(int k, int T) {
-    if (T & 1) {
-        const int m = T >> 1;
-        return (k & 1) ? m + ((k + 1) >> 1) : m - (k >> 1);
+// Tile of this CTA.  Tiles are issued in rings of increasing Chebyshev
+// distance from the centre tile of the grid: for rigs mounted near the grid
+// centre the nearest voxels see the most texels, so the heaviest tiles start
+// first and the light outer ring fills the tail of the launch.  Any order
+// gives the same results.  Warp 0 maps the block index (the rank) to its
+// ring, then finds the position inside the ring with ballots over 32 ring
+// positions at a time; the result is shared through `slot`.
+__device__ inline void tile_origin(const SampleArgs& a, int* slot, int& ti0, int& tj0) {
+    const int Ti = a.tiles_i, Tj = a.tiles_j;
+    if (threadIdx.x < 32) {
+        const int ci = (Ti - 1) >> 1, cj = (Tj - 1) >> 1;
+        auto area = [&](int r) -> int {  // tiles within Chebyshev distance r of the centre
+            if (r < 0) return 0;
+            const int h = min(ci + r, Ti - 1) - max(ci - r, 0) + 1;
+            const int w = min(cj + r, Tj - 1) - max(cj - r, 0) + 1;
+            return h * w;
+        };
+        int k = blockIdx.x, r = 0;
+        while (k >= area(r) - area(r - 1)) {
+            k -= area(r) - area(r - 1);
+            ++r;
+        }
+        // positions of ring r: p = 0 .. 8r - 1 (or just the centre for r = 0)
+        const int ring = r == 0 ? 1 : 8 * r;
+        int found = -1;
+        for (int p0 = 0; p0 < ring && found < 0; p0 += 32) {
+            const int p = p0 + (int)threadIdx.x;
+            int di = 0, dj = 0;
+            if (r > 0 && p < ring) {
+                const int side = p / (2 * r), t = p - side * 2 * r;
+                if (side == 0)      { di = -r;     dj = -r + t; }
+                else if (side == 1) { di = -r + t; dj = r; }
+                else if (side == 2) { di = r;      dj = r - t; }
+                else                { di = r - t;  dj = -r; }
+            }
+            const bool inside = p < ring && ci + di >= 0 && ci + di < Ti && cj + dj >= 0 && cj + dj < Tj;
+            const unsigned m = __ballot_sync(0xffffffffu, inside);
+            if (k < __popc(m)) {
+                if (inside && __popc(m & ((1u << threadIdx.x) - 1u)) == k) {
+                    slot[0] = (ci + di) * kTileI;
+                    slot[1] = (cj + dj) * kTileJ;
+                }
+                found = 1;
+            } else {
+                k -= __popc(m);
+            }
+        }
     }
-    const int m = (T >> 1) - 1;
-    return (k & 1) ? m + 1 + (k >> 1) : m - (k >> 1);
-}
-
-// Tile of this CTA.  Tile rows and columns are issued from the middle of the
-// grid outwards: for rigs mounted near the grid centre the nearest voxels see
-// the most texels, so the heaviest tiles start first and the light outer ones
-// fill the tail of the launch.  Any order gives the same results.
-__device__ __forceinline__ void tile_origin(const SampleArgs& a, int& ti0, int& tj0) {
-    const int k = blockIdx.x;
-    const int ri = k / a.tiles_j, rj = k - ri * a.tiles_j;
-    ti0 = middle_out(ri, a.tiles_i) * kTileI;
-    tj0 = middle_out(rj, a.tiles_j) * kTileJ;
+    __syncthreads();
+    ti0 = slot[0];
+    tj0 = slot[1];
 }
 
 // Stage camera constants of batch item b and cull cameras against the tile.
@@ -222,8 +245,7 @@ __device__ __forceinline__ int4 texel_box(const TileSmem& s, int cell, int aa, i
 // Lay out the patches of cameras [a0, a1) over their texel boxes.  Returns the
 // number of patch entries, or -1 (uniformly) if they would not fit in
 // kPatchCap.  On success s.pinfo[aa][cell] holds (y0, x0, h << 16 | w, offset)
-// and s.win[aa] the union of the camera's boxes over the tile.  Ends with a CTA
-// barrier.
+// and s.win[aa] the union of camera aa's boxes.  Ends with a CTA barrier.
 __device__ inline int layout_patches(const SampleArgs& a, const TileSmem& s, int zlen, int a0, int a1) {
     const int pairs = kTile * (a1 - a0);  // <= kTile * BEV_MAX_CAMERAS = 8 * kThreads
     int4 box[8];
@@ -239,7 +261,7 @@ __device__ inline int layout_patches(const SampleArgs& a, const TileSmem& s, int
     }
     if (threadIdx.x < a1 - a0) s.win[a0 + threadIdx.x] = make_int4(INT_MAX, -1, INT_MAX, -1);
     int total;
-    int off = block_exclusive_scan(sizes, s.scan, &total);  // (its barriers order the window reset)
+    int off = block_exclusive_scan(sizes, s.scan, &total);  // its barriers order the reset above
     if (total > kPatchCap) return -1;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -264,6 +286,30 @@ __device__ inline int layout_patches(const SampleArgs& a, const TileSmem& s, int
     return total;
 }
 
+// Ask L1 for the texel windows of cameras [a0, a1): every 128-byte line of
+// their channel vectors (channels-last rows [xmin, xmax] of rows [ymin, ymax],
+// chunks [chunk0, chunk0 + nchunks)).  Issued before the patches are filled,
+// so the lines are on chip when the channel loop reaches them.
+__device__ inline void prefetch_windows(const TileSmem& s, const uint4* feat_b, size_t cam_stride, int Wf,
+                                        int Qtot, int chunk0, int nchunks, int a0, int a1) {
+    for (int aa = a0; aa < a1; ++aa) {
+        const int4 wn = s.win[aa];
+        if (wn.y < wn.x) continue;
+        const uint4* Fn = feat_b + (size_t)s.act[aa] * cam_stride;
+        const int ww = wn.w - wn.z + 1;
+        // bytes of one window row, from the first texel's first chunk to the last texel's last chunk
+        const int span = ((ww - 1) * Qtot + nchunks) * 16;
+        const int lines = (span + 127) / 128 + 1;
+        const int rows = wn.y - wn.x + 1;
+        for (int t = threadIdx.x; t < rows * lines; t += kThreads) {
+            const int r = t / lines, l = t - r * lines;
+            const char* row = reinterpret_cast<const char*>(Fn + ((size_t)(wn.x + r) * Wf + wn.z) * Qtot + chunk0);
+            const char* p = row + 128 * l;
+            if (p < row + span) asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+        }
+    }
+}
+
 // Merge w / cnt of the valid voxels of cameras [a0, a1) into their patches.
 // One thread per (cell, camera): it clears its own patch, then adds the four
 // corner weights of each valid bin in increasing bin order (fp32 sums in a
@@ -281,14 +327,14 @@ __device__ inline void fill_patches(const SampleArgs& a, const TileSmem& s, int 
         for (int zl = 0; zl < zlen; ++zl) {
             const float2 f = s.items[item_index(cell, aa, zl, zlen)];
             if (!(f.x == f.x)) continue;
-            const float cntf = (float)cell_count(s.cnt, zl, cell);
+            const float rc = __frcp_rn((float)cell_count(s.cnt, zl, cell));
             const Corners c = bilinear_corners(f.x, f.y);
             const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
                 if ((unsigned)yy >= (unsigned)g.Hf || (unsigned)xx >= (unsigned)g.Wf) continue;
-                pw[(yy - pi.x) * w + (xx - pi.y)] += __fdiv_rn(ws[k], cntf);
+                pw[(yy - pi.x) * w + (xx - pi.y)] += ws[k] * rc;
             }
         }
     }
