@@ -77,8 +77,8 @@ def hbm_peak():
 
 
 KERNEL_SOURCES = {
-    "sample_forward_kernel": ["bev_forward.cu", "bev_tile.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
-    "sample_backward_kernel": ["bev_backward.cu", "bev_tile.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
+    "sample_forward_kernel": ["bev_forward.cu", "bev_warp.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
+    "sample_backward_kernel": ["bev_backward.cu", "bev_warp.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
 }
 
 

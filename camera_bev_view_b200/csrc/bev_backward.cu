@@ -9,12 +9,12 @@
 //
 // One CTA = one 8x8 BEV tile of one batch item and one channel slice, with the
 // same culling, once-per-voxel geometry and merged per-(cell, camera, texel)
-// weights as the forward (bev_tile.cuh).  The tile's dout slice is staged in
-// shared memory (coalesced along y) and held in registers: each lane owns V
-// chunks of 4 channels of one cell.  Each touched texel then receives one
-// 16-byte vector reduction per chunk (red.global.add.v4.f32) into the fp32
-// channels-last gradient buffer, however many height bins hit it.
-#include "bev_tile.cuh"
+// weights as the forward (bev_warp.cuh).  Each warp loads its row's dout slice
+// through its own shared-memory region (coalesced along y) into registers:
+// each lane owns V chunks of 4 channels of one cell.  Each touched texel then
+// receives one 16-byte vector reduction per chunk (red.global.add.v4.f32) into
+// the fp32 channels-last gradient buffer, however many height bins hit it.
+#include "bev_warp.cuh"
 
 namespace bev {
 
@@ -34,11 +34,11 @@ __device__ __forceinline__ void scatter_texel(float* p, const float (&d)[V][4], 
 }
 
 template <int L, int V>
-__device__ __forceinline__ void scatter_patch(const float (&d)[V][4], const float* pf, const int4 pi,
-                                              float* Gn, int Wf, int tstride, int ql, int nchunks) {
-    const int h = pi.z >> 16, w = pi.z & 0xffff;
-    const float* pw = pf + pi.w;
-    float* grow = Gn + ((size_t)pi.x * Wf + pi.y) * tstride;
+__device__ __forceinline__ void scatter_patch(const float (&d)[V][4], const float* pf, const Patch& pt, float* Gn,
+                                              int Wf, int tstride, int ql, int nchunks) {
+    const int h = pt.h, w = pt.w;
+    const float* pw = pf + pt.off;
+    float* grow = Gn + ((size_t)pt.y0 * Wf + pt.x0) * tstride;
     for (int r = 0; r < h; ++r, grow += (size_t)Wf * tstride, pw += w) {
         for (int cc = 0; cc < w; ++cc) {
             const float wt = pw[cc];
@@ -48,20 +48,27 @@ __device__ __forceinline__ void scatter_patch(const float (&d)[V][4], const floa
 }
 
 template <int L, int V>
-__device__ __forceinline__ void scatter_direct(const float (&d)[V][4], const TileSmem& s, int cell, int aa,
-                                               int zlen, float* Gn, int Hf, int Wf, int tstride, int ql,
-                                               int nchunks) {
-    for (int zl = 0; zl < zlen; ++zl) {
-        const float2 f = s.items[item_index(cell, aa, zl, zlen)];
-        if (!(f.x == f.x)) continue;
-        const float cntf = (float)cell_count(s.cnt, zl, cell);
-        const Corners c = bilinear_corners(f.x, f.y);
-        const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+__device__ __forceinline__ void scatter_direct(const float (&d)[V][4], const Items& it,
+                                               const float (&rc)[kZPerLaneMax], int zn, bool mine, int sub,
+                                               float* Gn, int Hf, int Wf, int tstride, int ql, int nchunks) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
-            if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
-            scatter_texel<L, V>(Gn + ((size_t)yy * Wf + xx) * tstride, d, __fdiv_rn(ws[k], cntf), ql, nchunks);
+    for (int t = 0; t < kZPerLaneMax; ++t) {
+        if (t >= zn) break;
+        for (int zz = 0; zz < L; ++zz) {
+            const int src = sub * L + zz;
+            const float fx = __shfl_sync(0xffffffffu, it.fx[t], src);
+            const float fy = __shfl_sync(0xffffffffu, it.fy[t], src);
+            const bool ok = (__shfl_sync(0xffffffffu, it.ok, src) >> t) & 1u;
+            const float r = __shfl_sync(0xffffffffu, rc[t], src);
+            if (!(mine && ok)) continue;
+            const Corners c = bilinear_corners(fx, fy);
+            const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
+                if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
+                scatter_texel<L, V>(Gn + ((size_t)yy * Wf + xx) * tstride, d, ws[k] * r, ql, nchunks);
+            }
         }
     }
 }
@@ -72,7 +79,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(c
     constexpr int CG = kCellsPerWarp / G;
     static_assert(G * CG == kCellsPerWarp, "lanes per cell must be 4, 8, 16 or 32");
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const TileSmem s = carve_smem(smem_raw, a.N);
+    const CtaSmem s = carve_smem(smem_raw, a.N);
     const GeoParams& g = a.g;
 
     const int b = blockIdx.y;
@@ -81,86 +88,76 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(c
     const int chunk0 = blockIdx.z * a.slice_chunks;
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
     const int c_base = chunk0 * 4;
-
     setup_tile(a, s, b, ti0, tj0);
     const int nA = s.act[32];
     if (nA == 0) return;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / L, ql = lane - sub * L;
-    // Upstream gradient of the tile into registers, kGroupCh channels at a time
-    // through the [channel][cell] staging tile (loads coalesced along y).
+    int* region = reinterpret_cast<int*>(s.warps + (size_t)warp * (kWarpBytes + 512));
+    const int i = ti0 + warp;
+
+    // dout of the warp's row -> [channel][cell] staging -> registers
+    float* stage = reinterpret_cast<float*>(region);
+    for (int t = lane; t < nchunks * 4 * kCellsPerWarp; t += 32) {
+        const int c = t >> 3, jc = t & 7;
+        float v = 0.0f;
+        if (c_base + c < a.C && i < g.X && tj0 + jc < g.Y)
+            v = a.dout[(((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0 + jc];
+        stage[c * kStageStride + jc] = v;
+    }
+    __syncwarp();
     float d[CG][V][4];
 #pragma unroll
-    for (int q = 0; q < CG; ++q)
+    for (int q = 0; q < CG; ++q) {
+        const int jc = q * G + sub;
 #pragma unroll
-        for (int v = 0; v < V; ++v)
+        for (int v = 0; v < V; ++v) {
+            const int c0 = (ql + v * L) * 4;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) d[q][v][e] = 0.0f;
-    for (int g0 = 0; g0 < nchunks * 4; g0 += kGroupCh) {
-        __syncthreads();
-        for (int t = threadIdx.x; t < kGroupCh * kTile; t += kThreads) {
-            const int c = t / kTile, cell = t - c * kTile;
-            const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
-            float v = 0.0f;
-            if (g0 + c < nchunks * 4 && c_base + g0 + c < a.C && i < g.X && j < g.Y)
-                v = a.dout[(((size_t)b * a.C + c_base + g0 + c) * g.X + i) * g.Y + j];
-            s.obuf[c * kObufStride + cell] = v;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int q = 0; q < CG; ++q) {
-            const int cell = warp * kCellsPerWarp + q * G + sub;
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int c0 = (ql + v * L) * 4 - g0;
-                if (c0 >= 0 && c0 < kGroupCh) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) d[q][v][e] = s.obuf[(c0 + e) * kObufStride + cell];
-                }
-            }
+            for (int e = 0; e < 4; ++e) d[q][v][e] = ql + v * L < nchunks ? stage[(c0 + e) * kStageStride + jc] : 0.0f;
         }
     }
+    __syncwarp();
+
     const size_t texels = (size_t)g.Hf * g.Wf;
     const int tstride = a.Qtot * 4;  // floats per texel in the gradient buffer
-    float* grad = a.dfeat + (size_t)(chunk0 + ql) * 4;
+    float* grad = a.dfeat + (size_t)(chunk0 + ql) * 4 + (size_t)b * a.N * texels * tstride;
+    const float x = voxel_centre(g.xmin, i, g.dx);
+    const int zn = min(kZPerLaneMax, (g.Z + L - 1) / L);
 
-    int zc = z_chunk(g.Z, nA);
-    int z0 = 0;
-    while (z0 < g.Z) {
-        const int zlen = min(zc, g.Z - z0);
-        geometry_chunk(a, s, ti0, tj0, nA, z0, zlen);
-        int total = layout_patches(a, s, zlen, 0, nA);
-        if (total < 0 && zlen > 1) {  // too many texels: fewer bins per chunk
-            zc = (zlen + 1) / 2;
-            continue;
-        }
-        int a0 = 0, ga = nA;
-        while (a0 < nA) {
-            const int a1 = min(nA, a0 + ga);
-            if (a0 > 0 || a1 < nA) total = layout_patches(a, s, zlen, a0, a1);
-            if (total < 0 && a1 - a0 > 1) {  // still too many: fewer cameras at once
-                ga = (a1 - a0 + 1) / 2;
-                continue;
-            }
-            if (total >= 0) fill_patches(a, s, zlen, a0, a1);
-            const float* pf = s.patch;
 #pragma unroll
-            for (int q = 0; q < CG; ++q) {
-                const int cell = warp * kCellsPerWarp + q * G + sub;
-                for (int aa = a0; aa < a1; ++aa) {
-                    float* Gn = grad + ((size_t)b * a.N + s.act[aa]) * texels * tstride;
-                    if (total >= 0)
-                        scatter_patch<L, V>(d[q], pf, s.pinfo[aa * kTile + cell], Gn, g.Wf, tstride, ql, nchunks);
-                    else
-                        scatter_direct<L, V>(d[q], s, cell, aa, zlen, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
-                }
+    for (int q = 0; q < CG; ++q) {
+        const int j = tj0 + q * G + sub;
+        const bool in_grid = i < g.X && j < g.Y;
+        const float y = voxel_centre(g.ymin, j, g.dy);
+        for (int z0 = 0; z0 < g.Z; z0 += L * zn) {
+            // valid cameras per bin of this lane, over all active cameras; the
+            // projections of the first two cameras are kept for the merge pass
+            int cnt[kZPerLaneMax] = {0, 0, 0, 0};
+            Items keep0, keep1;
+            for (int aa = 0; aa < nA; ++aa) {
+                const Items it = project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
+                if (aa == 0) keep0 = it;
+                if (aa == 1) keep1 = it;
+#pragma unroll
+                for (int t = 0; t < kZPerLaneMax; ++t) cnt[t] += (it.ok >> t) & 1u;
             }
-            __syncthreads();
-            a0 = a1;
-            total = -1;
+            float rc[kZPerLaneMax];
+#pragma unroll
+            for (int t = 0; t < kZPerLaneMax; ++t) rc[t] = cnt[t] > 0 ? __frcp_rn((float)cnt[t]) : 0.0f;
+            for (int aa = 0; aa < nA; ++aa) {
+                const Items it = aa == 0 ? keep0
+                               : aa == 1 ? keep1
+                                         : project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
+                const Patch pt = merge_patches<L>(it, rc, zn, sub, ql, g.Hf, g.Wf, region);
+                float* Gn = grad + (size_t)s.act[aa] * texels * tstride;
+                scatter_patch<L, V>(d[q], reinterpret_cast<const float*>(region), pt, Gn, g.Wf, tstride, ql, nchunks);
+                if (__any_sync(0xffffffffu, pt.overflow))
+                    scatter_direct<L, V>(d[q], it, rc, zn, pt.overflow, sub, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
+                __syncwarp();
+            }
         }
-        z0 += zlen;
     }
 }
 

@@ -5,15 +5,15 @@
 // then a sum over height, in one kernel with nothing intermediate in HBM).
 //
 // One CTA = one 8x8 BEV tile of one batch item and one channel slice; warp w
-// owns tile row w.  Per tile (bev_tile.cuh): cameras are culled, every
-// (cell, camera, bin) voxel is projected once, and the weights w / cnt of all
-// bins are merged per (cell, camera, texel).  The channel loop then visits
-// each touched texel of a (cell, camera) once: the L lanes of a cell read its
-// channel vector with 16-byte loads (V chunks per lane) from the channels-last
-// feature buffer and accumulate in fp32 registers, which persist across
-// height chunks.  The tile is finally stored along y, the contiguous axis of
-// out, through a [channel][cell] shared-memory staging tile.
-#include "bev_tile.cuh"
+// owns tile row w (bev_warp.cuh: cameras culled per tile, every (cell, camera,
+// bin) voxel projected once, the weights w / cnt of all bins merged per
+// (cell, camera, texel)).  The channel loop then visits each touched texel of
+// a (cell, camera) once: the L lanes of a cell read its channel vector with
+// 16-byte loads (V chunks per lane) from the channels-last feature buffer and
+// accumulate in fp32 registers, which persist across height chunks.  The warp
+// finally stores its row along y, the contiguous axis of out, through a
+// [channel][cell] staging tile in its own shared-memory region.
+#include "bev_warp.cuh"
 
 namespace bev {
 
@@ -57,32 +57,36 @@ __device__ __forceinline__ void accumulate_texel(Acc<BF16, V>& acc, const uint4*
         if (ql + v * L < nchunks) Chunk<BF16>::fma(acc[v], __ldg(p + v * L), w);
 }
 
-// Merged path: walk the (cell, camera) patch two rows by two columns per
-// step (patches are mostly two texels wide: a vertical column of voxels
-// projects to a near-vertical line).  The trip counts are the warp's largest
-// patch; the other cells of the warp are predicated off past their own.
+// Merged path: walk the cell's patch two rows by two columns per step
+// (patches are mostly two texels wide: a vertical column of voxels projects
+// to a near-vertical line).  The trip counts are the warp's largest patch;
+// the other cells of the warp are predicated off past their own.
 template <bool BF16, int L, int V>
-__device__ __forceinline__ void gather_patch(Acc<BF16, V>& acc, const float* pf, const int4 pi,
+__device__ __forceinline__ void gather_patch(Acc<BF16, V>& acc, const float* pf, const Patch& pt,
                                              const uint4* Fn, int Wf, int Qtot, int ql, int nchunks) {
-    const int h = pi.z >> 16, w = pi.z & 0xffff;
+    const int h = pt.h, w = pt.w;
     const int hmax = __reduce_max_sync(0xffffffffu, h);
     const int wmax = __reduce_max_sync(0xffffffffu, w);
     const size_t rstride = (size_t)Wf * Qtot;
+    bool lane_ok[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) lane_ok[v] = ql + v * L < nchunks;
     for (int c0 = 0; c0 < wmax; c0 += 2) {
         const bool c0in = c0 < w, c1in = c0 + 1 < w;
-        const float* pw = pf + pi.w + c0;
-        const uint4* rp = Fn + ((size_t)pi.x * Wf + pi.y + c0) * Qtot;
+        const float* pw = pf + pt.off + c0;
+        const uint4* rp = Fn + ((size_t)pt.y0 * Wf + pt.x0 + c0) * Qtot;
         for (int r0 = 0; r0 < hmax; r0 += 2, pw += 2 * w, rp += 2 * rstride) {
             const bool r0in = r0 < h, r1in = r0 + 1 < h;
-            const float wt[4] = {(r0in && c0in) ? pw[0] : 0.0f, (r0in && c1in) ? pw[1] : 0.0f,
-                                 (r1in && c0in) ? pw[w] : 0.0f, (r1in && c1in) ? pw[w + 1] : 0.0f};
+            const bool in[4] = {r0in && c0in, r0in && c1in, r1in && c0in, r1in && c1in};
+            const float wt[4] = {in[0] ? pw[0] : 0.0f, in[1] ? pw[1] : 0.0f, in[2] ? pw[w] : 0.0f,
+                                 in[3] ? pw[w + 1] : 0.0f};
             const uint4* pp[4] = {rp, rp + Qtot, rp + rstride, rp + rstride + Qtot};
             uint4 d[4][V];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
 #pragma unroll
                 for (int v = 0; v < V; ++v)
-                    d[u][v] = (wt[u] != 0.0f && ql + v * L < nchunks) ? __ldg(pp[u] + v * L) : make_uint4(0, 0, 0, 0);
+                    d[u][v] = (in[u] && wt[u] != 0.0f && lane_ok[v]) ? __ldg(pp[u] + v * L) : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -91,23 +95,30 @@ __device__ __forceinline__ void gather_patch(Acc<BF16, V>& acc, const float* pf,
     }
 }
 
-// Unmerged path for a camera whose patches do not fit: corners straight from (fx, fy).
+// Unmerged path for cells whose patches did not fit: each bin's four corners,
+// broadcast from the lane that projected it.  Called by the whole warp.
 template <bool BF16, int L, int V>
-__device__ __forceinline__ void gather_direct(Acc<BF16, V>& acc, const TileSmem& s, int cell, int aa,
-                                              int zlen, const uint4* Fn, int Hf, int Wf, int Qtot, int ql,
-                                              int nchunks) {
-    for (int zl = 0; zl < zlen; ++zl) {
-        const float2 f = s.items[item_index(cell, aa, zl, zlen)];
-        if (!(f.x == f.x)) continue;
-        const float cntf = (float)cell_count(s.cnt, zl, cell);
-        const Corners c = bilinear_corners(f.x, f.y);
-        const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+__device__ __forceinline__ void gather_direct(Acc<BF16, V>& acc, const Items& it,
+                                              const float (&rc)[kZPerLaneMax], int zn, bool mine, int sub,
+                                              const uint4* Fn, int Hf, int Wf, int Qtot, int ql, int nchunks) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
-            if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
-            accumulate_texel<BF16, L, V>(acc, Fn + ((size_t)yy * Wf + xx) * Qtot, __fdiv_rn(ws[k], cntf), ql,
-                                         nchunks);
+    for (int t = 0; t < kZPerLaneMax; ++t) {
+        if (t >= zn) break;
+        for (int zz = 0; zz < L; ++zz) {
+            const int src = sub * L + zz;
+            const float fx = __shfl_sync(0xffffffffu, it.fx[t], src);
+            const float fy = __shfl_sync(0xffffffffu, it.fy[t], src);
+            const bool ok = (__shfl_sync(0xffffffffu, it.ok, src) >> t) & 1u;
+            const float r = __shfl_sync(0xffffffffu, rc[t], src);
+            if (!(mine && ok)) continue;
+            const Corners c = bilinear_corners(fx, fy);
+            const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
+                if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
+                accumulate_texel<BF16, L, V>(acc, Fn + ((size_t)yy * Wf + xx) * Qtot, ws[k] * r, ql, nchunks);
+            }
         }
     }
 }
@@ -119,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
     constexpr int CG = kCellsPerWarp / G;    // rounds of cells per warp
     static_assert(G * CG == kCellsPerWarp, "lanes per cell must be 4, 8, 16 or 32");
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const TileSmem s = carve_smem(smem_raw, a.N);
+    const CtaSmem s = carve_smem(smem_raw, a.N);
     const GeoParams& g = a.g;
 
     const int b = blockIdx.y;
@@ -127,15 +138,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
     tile_origin(a, s.act + 40, ti0, tj0);
     const int chunk0 = blockIdx.z * a.slice_chunks;
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
-
     setup_tile(a, s, b, ti0, tj0);
     const int nA = s.act[32];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / L, ql = lane - sub * L;
-    const bool write_count = a.count != nullptr && blockIdx.z == 0;
+    int* region = reinterpret_cast<int*>(s.warps + (size_t)warp * (kWarpBytes + 512));
     const size_t texels = (size_t)g.Hf * g.Wf;
-    const uint4* feat = reinterpret_cast<const uint4*>(a.feat) + chunk0 + ql;
+    const uint4* feat = reinterpret_cast<const uint4*>(a.feat) + chunk0 + ql + (size_t)b * a.N * texels * a.Qtot;
+    const int i = ti0 + warp;
+    const float x = voxel_centre(g.xmin, i, g.dx);
+    const bool write_count = a.count != nullptr && blockIdx.z == 0;
+    const int zn = min(kZPerLaneMax, (g.Z + L - 1) / L);  // bins per lane per chunk
 
     float2 acc[CG][V][P];
 #pragma unroll
@@ -145,83 +159,85 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
 #pragma unroll
             for (int e = 0; e < P; ++e) acc[q][v][e] = make_float2(0.0f, 0.0f);
 
-    if (nA == 0) {
-        if (write_count) store_counts(a, nullptr, b, ti0, tj0, 0, g.Z);
-    } else {
-        int zc = z_chunk(g.Z, nA);
-        int z0 = 0;
-        while (z0 < g.Z) {
-            const int zlen = min(zc, g.Z - z0);
-            geometry_chunk(a, s, ti0, tj0, nA, z0, zlen);
-            int total = layout_patches(a, s, zlen, 0, nA);
-            if (total < 0 && zlen > 1) {  // too many texels: fewer bins per chunk
-                zc = (zlen + 1) / 2;
-                continue;
-            }
-            if (write_count) store_counts(a, s.cnt, b, ti0, tj0, z0, zlen);
-            int a0 = 0, ga = nA;
-            while (a0 < nA) {
-                const int a1 = min(nA, a0 + ga);
-                if (a0 > 0 || a1 < nA) total = layout_patches(a, s, zlen, a0, a1);
-                if (total < 0 && a1 - a0 > 1) {  // still too many: fewer cameras at once
-                    ga = (a1 - a0 + 1) / 2;
-                    continue;
-                }
-                if (total >= 0) {
-                    prefetch_windows(s, reinterpret_cast<const uint4*>(a.feat) + (size_t)b * a.N * texels * a.Qtot,
-                                     texels * a.Qtot, g.Wf, a.Qtot, chunk0, nchunks, a0, a1);
-                    fill_patches(a, s, zlen, a0, a1);
-                }
-                const float* pf = s.patch;
 #pragma unroll
-                for (int q = 0; q < CG; ++q) {
-                    const int cell = warp * kCellsPerWarp + q * G + sub;
-                    for (int aa = a0; aa < a1; ++aa) {
-                        const uint4* Fn = feat + ((size_t)b * a.N + s.act[aa]) * texels * a.Qtot;
-                        if (total >= 0)
-                            gather_patch<BF16, L, V>(acc[q], pf, s.pinfo[aa * kTile + cell], Fn, g.Wf, a.Qtot,
-                                                     ql, nchunks);
-                        else
-                            gather_direct<BF16, L, V>(acc[q], s, cell, aa, zlen, Fn, g.Hf, g.Wf, a.Qtot, ql,
-                                                      nchunks);
-                    }
-                }
-                __syncthreads();  // patches are rebuilt by the next camera group / chunk
-                a0 = a1;
-                total = -1;
+    for (int q = 0; q < CG; ++q) {
+        const int j = tj0 + q * G + sub;
+        const bool in_grid = i < g.X && j < g.Y;
+        const float y = voxel_centre(g.ymin, j, g.dy);
+        for (int z0 = 0; z0 < g.Z; z0 += L * zn) {
+            // valid cameras per bin of this lane, over all active cameras
+            // valid cameras per bin of this lane, over all active cameras; the
+            // projections of the first two cameras are kept for the merge pass
+            int cnt[kZPerLaneMax] = {0, 0, 0, 0};
+            Items keep0, keep1;
+            for (int aa = 0; aa < nA; ++aa) {
+                const Items it = project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
+                if (aa == 0) keep0 = it;
+                if (aa == 1) keep1 = it;
+#pragma unroll
+                for (int t = 0; t < kZPerLaneMax; ++t) cnt[t] += (it.ok >> t) & 1u;
             }
-            z0 += zlen;
+            float rc[kZPerLaneMax];
+#pragma unroll
+            for (int t = 0; t < kZPerLaneMax; ++t) {
+                rc[t] = cnt[t] > 0 ? __frcp_rn((float)cnt[t]) : 0.0f;
+                const int z = z0 + ql + L * t;
+                if (write_count && t < zn && in_grid && z < g.Z)
+                    a.count[(((size_t)b * g.X + i) * g.Y + j) * g.Z + z] = (uint8_t)cnt[t];
+            }
+            for (int aa = 0; aa < nA; ++aa) {
+                const Items it = aa == 0 ? keep0
+                               : aa == 1 ? keep1
+                                         : project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
+                const Patch pt = merge_patches<L>(it, rc, zn, sub, ql, g.Hf, g.Wf, region);
+                const uint4* Fn = feat + (size_t)s.act[aa] * texels * a.Qtot;
+                gather_patch<BF16, L, V>(acc[q], reinterpret_cast<const float*>(region), pt, Fn, g.Wf, a.Qtot, ql,
+                                         nchunks);
+                if (__any_sync(0xffffffffu, pt.overflow))
+                    gather_direct<BF16, L, V>(acc[q], it, rc, zn, pt.overflow, sub, Fn, g.Hf, g.Wf, a.Qtot, ql,
+                                              nchunks);
+                __syncwarp();  // the region is rebuilt for the next camera
+            }
         }
     }
-    // Store: kGroupCh channels at a time through the [channel][cell] staging
-    // tile (it aliases the geometry buffers), rows along y, the contiguous
-    // axis of out.  A 16-byte chunk (2P channels) never straddles a group.
+
+    // Store the warp's row: [channel][cell] staging tile in the warp's region,
+    // then rows of 8 cells along y.  Lanes of absent cameras still write 0.
+    float* stage = reinterpret_cast<float*>(region);
     const int c_base = chunk0 * 2 * P;
     const int c_real = max(0, min(nchunks * 2 * P, a.C - c_base));
-    for (int g0 = 0; g0 < c_real; g0 += kGroupCh) {
-        __syncthreads();
 #pragma unroll
-        for (int q = 0; q < CG; ++q) {
-            const int cell = warp * kCellsPerWarp + q * G + sub;
+    for (int q = 0; q < CG; ++q) {
+        const int jc = q * G + sub;
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int c0 = (ql + v * L) * 2 * P - g0;
-                if (ql + v * L < nchunks && c0 >= 0 && c0 < kGroupCh) {
+        for (int v = 0; v < V; ++v) {
+            const int c0 = (ql + v * L) * 2 * P;
+            if (ql + v * L < nchunks) {
 #pragma unroll
-                    for (int e = 0; e < P; ++e) {
-                        s.obuf[(c0 + 2 * e) * kObufStride + cell] = acc[q][v][e].x;
-                        s.obuf[(c0 + 2 * e + 1) * kObufStride + cell] = acc[q][v][e].y;
-                    }
+                for (int e = 0; e < P; ++e) {
+                    stage[(c0 + 2 * e) * kStageStride + jc] = acc[q][v][e].x;
+                    stage[(c0 + 2 * e + 1) * kStageStride + jc] = acc[q][v][e].y;
                 }
             }
         }
-        __syncthreads();
-        const int gc = min(kGroupCh, c_real - g0);
-        for (int t = threadIdx.x; t < gc * kTile; t += kThreads) {
-            const int c = t / kTile, cell = t - c * kTile;
-            const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
-            if (i < g.X && j < g.Y)
-                a.out[(((size_t)b * a.C + c_base + g0 + c) * g.X + i) * g.Y + j] = s.obuf[c * kObufStride + cell];
+    }
+    __syncwarp();
+    if (i < g.X) {
+        if ((g.Y & 3) == 0) {  // rows of 8 cells start 16-byte aligned: two float4 per channel
+            for (int t = lane; t < c_real * 2; t += 32) {
+                const int c = t >> 1, jc = (t & 1) * 4;
+                if (tj0 + jc < g.Y) {
+                    const float* sp = stage + c * kStageStride + jc;
+                    *reinterpret_cast<float4*>(a.out + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0 + jc) =
+                        make_float4(sp[0], sp[1], sp[2], sp[3]);
+                }
+            }
+        } else {
+            for (int t = lane; t < c_real * kCellsPerWarp; t += 32) {
+                const int c = t >> 3, jc = t & 7;
+                if (tj0 + jc < g.Y)
+                    a.out[(((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0 + jc] = stage[c * kStageStride + jc];
+            }
         }
     }
 }

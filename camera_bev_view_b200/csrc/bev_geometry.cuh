@@ -80,30 +80,29 @@ __device__ __forceinline__ Corners bilinear_corners(float fx, float fy) {
 }
 
 // Conservative visibility of an axis-aligned box of voxel centres from one
-// camera, evaluated one box corner at a time.  For a corner p this writes, in
-// fp64, each of the five validity conditions (depth > 0.1, uh >= 0,
-// W pc_z - uh >= 0, vh >= 0, H pc_z - vh >= 0) plus a rounding margin of 1e-4
-// of the terms' magnitude (far above the fp32 evaluation error).  Each such
-// quantity is convex in p, so its maximum over the box is at a corner: a
-// camera can be skipped for the box when one of the five maxima is negative.
+// camera, evaluated one box corner at a time.  For a corner p this writes
+// each of the five validity conditions (depth > 0.1, uh >= 0,
+// W pc_z - uh >= 0, vh >= 0, H pc_z - vh >= 0) plus a margin of 1e-3 of the
+// terms' magnitude (four orders above the fp32 evaluation error of both this
+// test and the projection it stands for).  Each such quantity is convex in p,
+// so its maximum over the box is at a corner: a camera can be skipped for the
+// box when one of the five maxima is negative.
 __device__ inline void corner_margins(const float* cam, float px, float py, float pz, float img_w,
-                                      float img_h, double m[5]) {
-    const double W = img_w, H = img_h;
-    const double p[3] = {px, py, pz};
-    double pc[3], mag[3];
+                                      float img_h, float m[5]) {
+    const float W = img_w, H = img_h;
+    float pc[3], mag[3];
     for (int r = 0; r < 3; ++r) {
         const float* e = cam + 4 * r;
-        pc[r] = (double)e[0] * p[0] + (double)e[1] * p[1] + (double)e[2] * p[2] + (double)e[3];
-        mag[r] = fabs((double)e[0] * p[0]) + fabs((double)e[1] * p[1]) + fabs((double)e[2] * p[2]) +
-                 fabs((double)e[3]);
+        pc[r] = e[0] * px + e[1] * py + e[2] * pz + e[3];
+        mag[r] = fabsf(e[0] * px) + fabsf(e[1] * py) + fabsf(e[2] * pz) + fabsf(e[3]);
     }
-    const double k0 = cam[12], k1 = cam[13], k2 = cam[14], k3 = cam[15], k4 = cam[16], k5 = cam[17];
-    const double uh = k0 * pc[0] + k1 * pc[1] + k2 * pc[2];
-    const double vh = k3 * pc[0] + k4 * pc[1] + k5 * pc[2];
-    const double umag = fabs(k0) * mag[0] + fabs(k1) * mag[1] + fabs(k2) * mag[2];
-    const double vmag = fabs(k3) * mag[0] + fabs(k4) * mag[1] + fabs(k5) * mag[2];
-    const double t = 1e-4, a = 1e-6;
-    m[0] = pc[2] - 0.1 + t * mag[2] + a;
+    const float k0 = cam[12], k1 = cam[13], k2 = cam[14], k3 = cam[15], k4 = cam[16], k5 = cam[17];
+    const float uh = k0 * pc[0] + k1 * pc[1] + k2 * pc[2];
+    const float vh = k3 * pc[0] + k4 * pc[1] + k5 * pc[2];
+    const float umag = fabsf(k0) * mag[0] + fabsf(k1) * mag[1] + fabsf(k2) * mag[2];
+    const float vmag = fabsf(k3) * mag[0] + fabsf(k4) * mag[1] + fabsf(k5) * mag[2];
+    const float t = 1e-3f, a = 1e-4f;
+    m[0] = pc[2] - 0.1f + t * mag[2] + a;
     m[1] = uh + t * umag + a;
     m[2] = W * pc[2] - uh + t * (umag + W * mag[2]) + a;
     m[3] = vh + t * vmag + a;

@@ -9,31 +9,31 @@
 namespace bev {
 
 // BEV tile owned by one CTA: kTileI rows (ego x) by kTileJ columns (ego y).
-// Warp w owns tile row w (kTileJ = 8 cells).
+// Warp w owns tile row w (kTileJ = 8 cells) and works on it on its own: after
+// the CTA has staged the calibrations and culled the cameras, no CTA-wide
+// barrier is needed.
 constexpr int kTileI = 8;
 constexpr int kTileJ = 8;
 constexpr int kTile = kTileI * kTileJ;
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCellsPerWarp = kTile / kWarps;
-static_assert(kCellsPerWarp == kTileJ, "one warp per tile row");
-// (fx, fy) slots per height chunk: kTile * active cameras * bins.  At least one
-// bin of every camera must fit (a chunk never has fewer than one bin).
-constexpr int kItemCap = 2048;
-static_assert(kItemCap >= kTile * 32, "one height bin of 32 cameras must fit");
-// Merged-weight patch entries per height chunk (fp32 each).
-constexpr int kPatchCap = 2048;
-// Height bins per chunk at most (valid counts are packed one byte per cell).
-constexpr int kZChunkMax = 32;
-// Channels per CTA slice.
+static_assert(kCellsPerWarp == kTileJ && kWarps == kTileI, "one warp per tile row");
+// Height bins a lane projects per chunk (chunk = lanes per cell * this).
+constexpr int kZPerLaneMax = 4;
+// Merged-weight entries of one warp for one (camera, height chunk): the
+// patches of the cells the warp works on at once.  Each entry is an exact
+// fixed-point sum split over two 32-bit words (see merge_patches).
+constexpr int kWarpPatchCap = 512;
+// Per-warp shared-memory region: the patch words, reused as the
+// [channel][cell] staging tile of the warp's row (kSliceMax x kStageStride).
 constexpr int kSliceMax = 128;
-// The [channel][cell] staging tile used to move a tile's channel vectors
-// between registers and the y-contiguous rows of [B,C,X,Y] covers kGroupCh
-// channels at a time (it aliases the geometry buffers).
-constexpr int kGroupCh = 32;
-constexpr int kObufStride = kTile + 1;  // padded row of the staging tile
-// Shared memory per CTA stays small (~26 KB for 6 cameras) so that most of
-// the SM's 256 KB on-chip array serves as L1 for the tile's texel windows.
+constexpr int kStageStride = kCellsPerWarp + 1;
+constexpr int kWarpBytes = 2 * sizeof(int) * kWarpPatchCap;
+static_assert((int)sizeof(float) * kSliceMax * kStageStride <= kWarpBytes + 512,
+              "staging tile must fit the warp region");
+// CTAs kept resident per SM; shared memory stays small (~34 KB) so that most
+// of the SM's on-chip array serves as L1 for the tiles' texel windows.
 constexpr int kCtasPerSm = 3;
 
 struct SampleArgs {
@@ -57,28 +57,20 @@ struct SampleArgs {
 // Byte offsets of the per-CTA shared-memory regions (one source of truth for
 // the kernels' carve-up and the launch size).
 struct SmemLayout {
-    size_t items, patch, cnt, pinfo, win, cams, act, scan, total;
+    size_t warps, cams, act, total;
 };
 
 __host__ __device__ inline SmemLayout smem_layout(int N) {
     SmemLayout l;
     size_t b = 0;
-    l.items = b;  b += sizeof(float2) * kItemCap;                     // geometry slots
-    l.patch = b;  b += sizeof(float) * kPatchCap;                     // merged weights
-    l.cnt = b;    b += sizeof(int) * (kTile / 4) * kZChunkMax;        // valid counts, a byte per (bin, cell)
-    l.pinfo = b;  b += sizeof(int4) * kTile * N;                      // patch box per (cell, active camera)
-    l.win = b;    b += sizeof(int4) * 32;                             // texel window per active camera
+    l.warps = b;  b += (size_t)kWarps * (kWarpBytes + 512);           // per-warp patch / staging regions
     l.cams = b;   b += sizeof(float) * ((N * kCamFloats + 3) & ~3);   // camera constants
-    l.act = b;    b += sizeof(int) * 64;                              // active camera list
-    l.scan = b;   b += sizeof(int) * 64;                              // scan scratch
+    l.act = b;    b += sizeof(int) * 128;                             // active cameras, tile slot, flags
     l.total = b;
     return l;
 }
 
 __host__ __device__ inline size_t sample_smem_bytes(int N) { return smem_layout(N).total; }
-
-static_assert(sizeof(float) * kGroupCh * kObufStride <= sizeof(float2) * kItemCap + sizeof(float) * kPatchCap,
-              "the staging tile aliases the geometry slots and the patches");
 
 // Preferred shared-memory carveout for kCtasPerSm CTAs of `smem` bytes each:
 // the smallest shared-memory configuration of the SM (KB) that holds them,

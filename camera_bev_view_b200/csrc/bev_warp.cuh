@@ -1,0 +1,293 @@
+// bev_warp.cuh -- BEV tile machinery shared by the forward and backward kernels.
+//
+// FlashBEV's reading notes ("Method" item 3) recompute the channel-independent
+// geometry for every channel and name that recompute as the cost that grows
+// with C ("Limitation", second point; their "Takeaway" 4 proposes block-level
+// geometry reuse).  Here a CTA owns an 8x8 tile of BEV cells: it stages the
+// calibrations once and culls the cameras that cannot see any voxel of the
+// tile; from then on each warp works on its own tile row, with no CTA-wide
+// barrier.  For G = 32 / L cells at a time a warp
+//   1. projects each (cell, camera, height bin) voxel once -- lanes of a cell
+//      take consecutive bins -- and counts the valid cameras of each bin in
+//      registers;
+//   2. per camera, reduces the box of texels the cell's valid voxels touch and
+//      lays a patch over it in the warp's shared-memory region;
+//   3. merges the bilinear weights w / cnt of all bins into the patch with
+//      integer atomics on an exact fixed-point representation, so the merged
+//      weight does not depend on the order of the additions, then rounds each
+//      merged weight once to fp32;
+//   4. hands the patch to the channel loop (lanes of a cell now take channel
+//      chunks), which visits each touched texel once, whatever the number of
+//      bins that hit it.  Patches that do not fit fall back to visiting the
+//      four bilinear corners of each bin.
+#pragma once
+
+#include <limits.h>
+
+#include "bev_kernels.cuh"
+
+namespace bev {
+
+struct CtaSmem {
+    unsigned char* warps;  // kWarps regions of kWarpBytes + 512
+    float* cams;           // [N][kCamFloats]
+    int* act;              // [0..nA) active camera ids, [32] nA, [40..41] tile origin, [64..95] flags
+};
+
+__device__ __forceinline__ CtaSmem carve_smem(unsigned char* smem, int N) {
+    const SmemLayout l = smem_layout(N);
+    CtaSmem s;
+    s.warps = smem + l.warps;
+    s.cams = reinterpret_cast<float*>(smem + l.cams);
+    s.act = reinterpret_cast<int*>(smem + l.act);
+    return s;
+}
+
+// Tile of this CTA.  Tiles are issued in rings of increasing Chebyshev
+// distance from the centre tile of the grid: for rigs mounted near the grid
+// centre the nearest voxels see the most texels, so the heaviest tiles start
+// first and the light outer ring fills the tail of the launch.  Any order
+// gives the same results.  Warp 0 maps the block index (the rank) to its
+// ring, then finds the position inside the ring with ballots over 32 ring
+// positions at a time.
+__device__ inline void tile_origin(const SampleArgs& a, int* slot, int& ti0, int& tj0) {
+    const int Ti = a.tiles_i, Tj = a.tiles_j;
+    if (threadIdx.x < 32) {
+        const int ci = (Ti - 1) >> 1, cj = (Tj - 1) >> 1;
+        auto area = [&](int r) -> int {  // tiles within Chebyshev distance r of the centre
+            if (r < 0) return 0;
+            const int h = min(ci + r, Ti - 1) - max(ci - r, 0) + 1;
+            const int w = min(cj + r, Tj - 1) - max(cj - r, 0) + 1;
+            return h * w;
+        };
+        // ring r of rank k: the smallest r with area(r) > k (binary search)
+        int lo = 0, hi = max(max(ci, Ti - 1 - ci), max(cj, Tj - 1 - cj));
+        const int rank = blockIdx.x;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (area(mid) > rank) hi = mid; else lo = mid + 1;
+        }
+        const int r = lo;
+        int k = rank - area(r - 1);
+        const int ring = r == 0 ? 1 : 8 * r;
+        int found = -1;
+        for (int p0 = 0; p0 < ring && found < 0; p0 += 32) {
+            const int p = p0 + (int)threadIdx.x;
+            int di = 0, dj = 0;
+            if (r > 0 && p < ring) {
+                const int side = p / (2 * r), t = p - side * 2 * r;
+                if (side == 0)      { di = -r;     dj = -r + t; }
+                else if (side == 1) { di = -r + t; dj = r; }
+                else if (side == 2) { di = r;      dj = r - t; }
+                else                { di = r - t;  dj = -r; }
+            }
+            const bool inside = p < ring && ci + di >= 0 && ci + di < Ti && cj + dj >= 0 && cj + dj < Tj;
+            const unsigned m = __ballot_sync(0xffffffffu, inside);
+            if (k < __popc(m)) {
+                if (inside && __popc(m & ((1u << threadIdx.x) - 1u)) == k) {
+                    slot[0] = (ci + di) * kTileI;
+                    slot[1] = (cj + dj) * kTileJ;
+                }
+                found = 1;
+            } else {
+                k -= __popc(m);
+            }
+        }
+    }
+    __syncthreads();
+    ti0 = slot[0];
+    tj0 = slot[1];
+}
+
+// Stage camera constants of batch item b and cull cameras against the tile.
+// One thread per (camera, corner of the tile's voxel-centre box); the five
+// visibility margins are max-reduced over the eight corners with shuffles.
+__device__ inline void setup_tile(const SampleArgs& a, const CtaSmem& s, int b, int ti0, int tj0) {
+    const int tid = threadIdx.x;
+    for (int t = tid; t < a.N * kCamFloats; t += kThreads) {
+        const int n = t / kCamFloats, r = t - n * kCamFloats;
+        s.cams[t] = r < 12 ? a.E[((size_t)b * a.N + n) * 16 + r]
+                           : a.K[((size_t)b * a.N + n) * 9 + (r - 12)];
+    }
+    __syncthreads();
+    const GeoParams& g = a.g;
+    const int n = tid >> 3, v = tid & 7;  // kThreads == 8 * BEV_MAX_CAMERAS
+    if ((tid >> 5) * 4 < a.N) {           // warps holding at least one camera
+        float m[5] = {-1e30f, -1e30f, -1e30f, -1e30f, -1e30f};
+        if (n < a.N) {
+            const int i1 = min(ti0 + kTileI, g.X) - 1, j1 = min(tj0 + kTileJ, g.Y) - 1;
+            const float px = voxel_centre(g.xmin, (v & 1) ? i1 : ti0, g.dx);
+            const float py = voxel_centre(g.ymin, (v & 2) ? j1 : tj0, g.dy);
+            const float pz = voxel_centre(g.zmin, (v & 4) ? g.Z - 1 : 0, g.dz);
+            corner_margins(s.cams + n * kCamFloats, px, py, pz, g.img_w, g.img_h, m);
+        }
+#pragma unroll
+        for (int q = 0; q < 5; ++q) {
+            m[q] = fmaxf(m[q], __shfl_xor_sync(0xffffffffu, m[q], 1));
+            m[q] = fmaxf(m[q], __shfl_xor_sync(0xffffffffu, m[q], 2));
+            m[q] = fmaxf(m[q], __shfl_xor_sync(0xffffffffu, m[q], 4));
+        }
+        if (v == 0) s.act[64 + n] = (n < a.N) && m[0] >= 0.0f && m[1] >= 0.0f && m[2] >= 0.0f &&
+                                    m[3] >= 0.0f && m[4] >= 0.0f;
+    } else if (v == 0) {
+        s.act[64 + n] = 0;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        const bool vis = s.act[64 + tid] != 0;
+        const unsigned mask = __ballot_sync(0xffffffffu, vis);
+        if (vis) s.act[__popc(mask & ((1u << tid) - 1u))] = tid;
+        if (tid == 0) s.act[32] = __popc(mask);
+    }
+    __syncthreads();
+}
+
+// Lanes of one cell: L consecutive lanes (sub = lane / L, ql = lane % L).
+template <int L>
+__device__ __forceinline__ int group_min(int v) {
+#pragma unroll
+    for (int o = 1; o < L; o <<= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+template <int L>
+__device__ __forceinline__ int group_max(int v) {
+#pragma unroll
+    for (int o = 1; o < L; o <<= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Exclusive prefix of a per-group value (uniform within each group) over the
+// G = 32 / L groups of the warp; *total receives the sum over all groups.
+template <int L>
+__device__ __forceinline__ int group_prefix(int size, int sub, int* total) {
+    constexpr int G = 32 / L;
+    int before = 0, all = 0;
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+        const int sz = __shfl_sync(0xffffffffu, size, gg * L);
+        before += gg < sub ? sz : 0;
+        all += sz;
+    }
+    *total = all;
+    return before;
+}
+
+// Exact fixed point of the merged weights.  A contribution v = w / cnt (<= 1,
+// fp32) is split into hi = floor(v * 2^20) and lo = round((v - hi 2^-20) 2^40)
+// (the subtraction is exact, lo < 2^20); the halves are summed with 32-bit
+// integer atomics (at most kZPerLaneMax * 32 contributions reach one entry, so
+// neither overflows), and the total hi 2^-20 + lo 2^-40 is independent of the
+// order of the additions.  It is rounded to fp32 once.
+constexpr float kTwo20 = 1048576.0f;
+constexpr float kTwoM20 = 9.5367431640625e-07f;
+constexpr float kTwo40 = 1099511627776.0f;
+constexpr float kTwoM40 = 9.094947017729282379150390625e-13f;
+
+// One cell group's projections for one camera in one height chunk.
+struct Items {
+    float fx[kZPerLaneMax], fy[kZPerLaneMax];
+    unsigned ok;  // bit t: item t is a valid voxel
+};
+
+// Project this lane's bins z = z0 + ql + L t (t < zn) of voxel column (x, y)
+// through one camera.
+template <int L>
+__device__ __forceinline__ Items project_items(const float* cam, float x, float y, bool in_grid, int z0,
+                                               int zn, int ql, const GeoParams& g) {
+    Items it;
+    it.ok = 0;
+#pragma unroll
+    for (int t = 0; t < kZPerLaneMax; ++t) {
+        it.fx[t] = 0.0f;
+        it.fy[t] = 0.0f;
+        const int z = z0 + ql + L * t;
+        if (t < zn && in_grid && z < g.Z) {
+            float fx, fy;
+            if (project_voxel(cam, x, y, voxel_centre(g.zmin, z, g.dz), g, fx, fy)) {
+                it.fx[t] = fx;
+                it.fy[t] = fy;
+                it.ok |= 1u << t;
+            }
+        }
+    }
+    return it;
+}
+
+// Patch of one cell group for one camera: box origin, height, width and
+// offset in the warp's region; h == 0 when the cell has no valid voxel or the
+// patches of the warp do not fit (then `overflow` is set for the cell).
+struct Patch {
+    int y0, x0, h, w, off;
+    bool overflow;
+};
+
+// Box, placement, exact merge and fp32 rounding of one camera's weights for
+// the warp's current cells.  rc[t] = 1 / cnt of item t.  Ends with the patch
+// values readable by all lanes of the warp (fp32 at words [off, off + h * w)
+// of `region`).
+template <int L>
+__device__ __forceinline__ Patch merge_patches(const Items& it, const float (&rc)[kZPerLaneMax], int zn,
+                                               int sub, int ql, int Hf, int Wf, int* region) {
+    int ylo = INT_MAX, yhi = -1, xlo = INT_MAX, xhi = -1;
+#pragma unroll
+    for (int t = 0; t < kZPerLaneMax; ++t) {
+        if (t < zn && (it.ok >> t & 1u)) {
+            const int x0 = (int)floorf(it.fx[t]), y0 = (int)floorf(it.fy[t]);
+            ylo = min(ylo, max(y0, 0));
+            yhi = max(yhi, min(y0 + 1, Hf - 1));
+            xlo = min(xlo, max(x0, 0));
+            xhi = max(xhi, min(x0 + 1, Wf - 1));
+        }
+    }
+    ylo = group_min<L>(ylo);
+    yhi = group_max<L>(yhi);
+    xlo = group_min<L>(xlo);
+    xhi = group_max<L>(xhi);
+    Patch p;
+    p.y0 = ylo;
+    p.x0 = xlo;
+    p.h = yhi >= ylo ? yhi - ylo + 1 : 0;
+    p.w = yhi >= ylo ? xhi - xlo + 1 : 0;
+    int total;
+    p.off = group_prefix<L>(p.h * p.w, sub, &total);
+    p.overflow = p.off + p.h * p.w > kWarpPatchCap;
+    if (p.overflow) p.h = 0;
+    int* lo = region;
+    int* hi = region + kWarpPatchCap;
+    const int n = p.h * p.w;
+    for (int e = ql; e < n; e += L) {
+        lo[p.off + e] = 0;
+        hi[p.off + e] = 0;
+    }
+    __syncwarp();
+    if (n > 0) {
+#pragma unroll
+        for (int t = 0; t < kZPerLaneMax; ++t) {
+            if (t < zn && (it.ok >> t & 1u)) {
+                const Corners c = bilinear_corners(it.fx[t], it.fy[t]);
+                const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
+                    if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
+                    const float v = ws[k] * rc[t];
+                    const int qh = __float2int_rd(v * kTwo20);
+                    const int ql_ = __float2int_rn(__fmul_rn(__fsub_rn(v, (float)qh * kTwoM20), kTwo40));
+                    const int e = p.off + (yy - p.y0) * p.w + (xx - p.x0);
+                    if (ql_ != 0) atomicAdd(&lo[e], ql_);
+                    if (qh != 0) atomicAdd(&hi[e], qh);
+                }
+            }
+        }
+    }
+    __syncwarp();
+    float* pf = reinterpret_cast<float*>(region);
+    for (int e = ql; e < n; e += L) {
+        pf[p.off + e] = __fadd_rn((float)hi[p.off + e] * kTwoM20, (float)lo[p.off + e] * kTwoM40);
+    }
+    __syncwarp();
+    return p;
+}
+
+}  // namespace bev
