@@ -160,6 +160,23 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Units per second for the whole job: every rank processes its own
+    batch each step, and the slowest rank sets the step time."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -305,15 +322,9 @@ def run_ours(args):
         per = {name: [ev[k][s].elapsed_time(ev[k][s + 1]) for k in range(args.steps)]
                for s, name in enumerate(names)}
     stage_ms = {name: sum(v) / len(v) for name, v in per.items()}
-    ms_local = sum(stage_ms.values())
-    ms = ms_local
-    if world > 1:
-        t = torch.tensor([ms_local], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-
+    ms = max_over_ranks(sum(stage_ms.values()), world, dev)
     elems = B * C * X * Y
-    value = world * elems / (ms * 1e-3)
+    value = whole_job_rate(elems, world, ms)
 
     # roofline of the dominant kernel (by time)
     peak, peak_src = hbm_peak()
@@ -356,11 +367,7 @@ def run_ours(args):
             e1.synchronize()
             if k >= 5:
                 e2e_times.append(e0.elapsed_time(e1))
-    e2e_ms = statistics.median(e2e_times)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(statistics.median(e2e_times), world, dev)
     h2d = sum(t.numel() * t.element_size() for t in (F_h, K_h, E_h, dout_h))
     d2h = out.numel() * 4 + dF.numel() * 4
 
@@ -377,7 +384,7 @@ def run_ours(args):
         "forward_only": {"elements_per_s": elems / (stage_ms["forward"] * 1e-3), "GB_per_s": fwd_gbs,
                          "frac_of_hbm_peak": fwd_gbs / peak},
         "roofline": roofline,
-        "e2e": {"value": world * elems / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+        "e2e": {"value": whole_job_rate(elems, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "pinned host -> device copies, bev_sample_forward (NCHW) + bev_sample_backward, "
                         "device -> pinned host copies"},
