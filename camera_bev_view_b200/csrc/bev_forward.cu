@@ -95,30 +95,46 @@ __device__ __forceinline__ void gather_patch(Acc<BF16, V>& acc, const float* pf,
     }
 }
 
-// Unmerged path for cells whose patches did not fit: each bin's four corners,
-// broadcast from the lane that projected it.  Called by the whole warp.
+// Unmerged path: each bin of the cell (projected by lane zz of the cell's
+// lanes) is broadcast to the cell's lanes, which load its four bilinear
+// corners and accumulate.  Branch-free: corners outside the map, invalid bins
+// and cells with mine == false carry weight 0 and their loads are predicated
+// off.  Called by the whole warp.
 template <bool BF16, int L, int V>
-__device__ __forceinline__ void gather_direct(Acc<BF16, V>& acc, const Items& it,
-                                              const float (&rc)[kZPerLaneMax], int zn, bool mine, int sub,
-                                              const uint4* Fn, int Hf, int Wf, int Qtot, int ql, int nchunks) {
+__device__ __forceinline__ void gather_bins(Acc<BF16, V>& acc, const Items& it, const float (&rc)[kZPerLaneMax],
+                                            int zn, bool mine, int sub, const uint4* Fn, int Hf, int Wf, int Qtot,
+                                            int ql, int nchunks) {
+    bool lane_ok[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) lane_ok[v] = ql + v * L < nchunks;
+    const ptrdiff_t rs = (ptrdiff_t)Wf * Qtot;
 #pragma unroll
     for (int t = 0; t < kZPerLaneMax; ++t) {
         if (t >= zn) break;
+        const float rct = (mine && (it.ok >> t & 1u)) ? rc[t] : 0.0f;
+#pragma unroll 2
         for (int zz = 0; zz < L; ++zz) {
             const int src = sub * L + zz;
             const float fx = __shfl_sync(0xffffffffu, it.fx[t], src);
             const float fy = __shfl_sync(0xffffffffu, it.fy[t], src);
-            const bool ok = (__shfl_sync(0xffffffffu, it.ok, src) >> t) & 1u;
-            const float r = __shfl_sync(0xffffffffu, rc[t], src);
-            if (!(mine && ok)) continue;
+            const float r = __shfl_sync(0xffffffffu, rct, src);
             const Corners c = bilinear_corners(fx, fy);
-            const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+            const bool cx0 = (unsigned)c.x0 < (unsigned)Wf, cx1 = (unsigned)(c.x0 + 1) < (unsigned)Wf;
+            const bool cy0 = (unsigned)c.y0 < (unsigned)Hf, cy1 = (unsigned)(c.y0 + 1) < (unsigned)Hf;
+            const float wt[4] = {(cy0 && cx0) ? c.w00 * r : 0.0f, (cy0 && cx1) ? c.w01 * r : 0.0f,
+                                 (cy1 && cx0) ? c.w10 * r : 0.0f, (cy1 && cx1) ? c.w11 * r : 0.0f};
+            const uint4* p = Fn + (ptrdiff_t)(c.y0 * Wf + c.x0) * Qtot;
+            const uint4* pp[4] = {p, p + Qtot, p + rs, p + rs + Qtot};
+            uint4 d[4][V];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
-                if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
-                accumulate_texel<BF16, L, V>(acc, Fn + ((size_t)yy * Wf + xx) * Qtot, ws[k] * r, ql, nchunks);
-            }
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < V; ++v)
+                    d[u][v] = (wt[u] != 0.0f && lane_ok[v]) ? __ldg(pp[u] + v * L) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < V; ++v) Chunk<BF16>::fma(acc[v], d[u][v], wt[u]);
         }
     }
 }
@@ -165,7 +181,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
         const bool in_grid = i < g.X && j < g.Y;
         const float y = voxel_centre(g.ymin, j, g.dy);
         for (int z0 = 0; z0 < g.Z; z0 += L * zn) {
-            // valid cameras per bin of this lane, over all active cameras
             // valid cameras per bin of this lane, over all active cameras; the
             // projections of the first two cameras are kept for the merge pass
             int cnt[kZPerLaneMax] = {0, 0, 0, 0};
@@ -189,14 +204,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
                 const Items it = aa == 0 ? keep0
                                : aa == 1 ? keep1
                                          : project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
-                const Patch pt = merge_patches<L>(it, rc, zn, sub, ql, g.Hf, g.Wf, region);
                 const uint4* Fn = feat + (size_t)s.act[aa] * texels * a.Qtot;
-                gather_patch<BF16, L, V>(acc[q], reinterpret_cast<const float*>(region), pt, Fn, g.Wf, a.Qtot, ql,
-                                         nchunks);
-                if (__any_sync(0xffffffffu, pt.overflow))
-                    gather_direct<BF16, L, V>(acc[q], it, rc, zn, pt.overflow, sub, Fn, g.Hf, g.Wf, a.Qtot, ql,
-                                              nchunks);
-                __syncwarp();  // the region is rebuilt for the next camera
+                Patch pt = patch_box<L>(it, zn, g.Hf, g.Wf);
+                if (merge_pays<L>(pt, zn, kMergeStepsFwd)) {
+                    merge_patches<L>(pt, it, rc, zn, sub, ql, g.Hf, g.Wf, region);
+                    gather_patch<BF16, L, V>(acc[q], reinterpret_cast<const float*>(region), pt, Fn, g.Wf, a.Qtot,
+                                             ql, nchunks);
+                    if (__any_sync(0xffffffffu, pt.overflow))
+                        gather_bins<BF16, L, V>(acc[q], it, rc, zn, pt.overflow, sub, Fn, g.Hf, g.Wf, a.Qtot, ql,
+                                                nchunks);
+                    __syncwarp();  // the region is rebuilt for the next camera
+                } else {
+                    gather_bins<BF16, L, V>(acc[q], it, rc, zn, true, sub, Fn, g.Hf, g.Wf, a.Qtot, ql, nchunks);
+                }
             }
         }
     }

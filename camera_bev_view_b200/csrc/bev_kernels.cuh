@@ -25,6 +25,11 @@ constexpr int kZPerLaneMax = 4;
 // patches of the cells the warp works on at once.  Each entry is an exact
 // fixed-point sum split over two 32-bit words (see merge_patches).
 constexpr int kWarpPatchCap = 512;
+// Forward: merging the weights of one (cell group, camera) pays when the
+// merged patch walk takes fewer steps (four texels of every lane's chunks)
+// than the bins' corners unmerged, plus this margin for the merge itself.
+// The backward always merges: there a step costs global reductions.
+constexpr int kMergeStepsFwd = 0;
 // Per-warp shared-memory region: the patch words, reused as the
 // [channel][cell] staging tile of the warp's row (kSliceMax x kStageStride).
 constexpr int kSliceMax = 128;

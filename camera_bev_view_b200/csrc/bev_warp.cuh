@@ -143,17 +143,19 @@ __device__ inline void setup_tile(const SampleArgs& a, const CtaSmem& s, int b, 
 }
 
 // Lanes of one cell: L consecutive lanes (sub = lane / L, ql = lane % L).
+// Per-halfword unsigned min / max over the cell's lanes (two 16-bit fields
+// reduced at once).
 template <int L>
-__device__ __forceinline__ int group_min(int v) {
+__device__ __forceinline__ unsigned group_min2(unsigned v) {
 #pragma unroll
-    for (int o = 1; o < L; o <<= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    for (int o = 1; o < L; o <<= 1) v = __vminu2(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 
 template <int L>
-__device__ __forceinline__ int group_max(int v) {
+__device__ __forceinline__ unsigned group_max2(unsigned v) {
 #pragma unroll
-    for (int o = 1; o < L; o <<= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    for (int o = 1; o < L; o <<= 1) v = __vmaxu2(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 
@@ -222,33 +224,56 @@ struct Patch {
     bool overflow;
 };
 
-// Box, placement, exact merge and fp32 rounding of one camera's weights for
-// the warp's current cells.  rc[t] = 1 / cnt of item t.  Ends with the patch
-// values readable by all lanes of the warp (fp32 at words [off, off + h * w)
-// of `region`).
+// Box of texels the valid voxels of this lane's cell touch through one
+// camera (uniform over the cell's lanes); h == 0 when the cell has no valid
+// voxel.  `off` and `overflow` are set by merge_patches.
 template <int L>
-__device__ __forceinline__ Patch merge_patches(const Items& it, const float (&rc)[kZPerLaneMax], int zn,
-                                               int sub, int ql, int Hf, int Wf, int* region) {
-    int ylo = INT_MAX, yhi = -1, xlo = INT_MAX, xhi = -1;
+__device__ __forceinline__ Patch patch_box(const Items& it, int zn, int Hf, int Wf) {
+    // lo = (ylo, xlo), hi = (yhi + 1, xhi + 1) as 16-bit fields (dimensions
+    // are below 2^15); an empty cell keeps lo = (0xffff, 0xffff), hi = 0
+    unsigned lo = 0xffffffffu, hi = 0u;
 #pragma unroll
     for (int t = 0; t < kZPerLaneMax; ++t) {
         if (t < zn && (it.ok >> t & 1u)) {
             const int x0 = (int)floorf(it.fx[t]), y0 = (int)floorf(it.fy[t]);
-            ylo = min(ylo, max(y0, 0));
-            yhi = max(yhi, min(y0 + 1, Hf - 1));
-            xlo = min(xlo, max(x0, 0));
-            xhi = max(xhi, min(x0 + 1, Wf - 1));
+            const unsigned l = ((unsigned)max(y0, 0) << 16) | (unsigned)max(x0, 0);
+            const unsigned h = ((unsigned)min(y0 + 2, Hf) << 16) | (unsigned)min(x0 + 2, Wf);
+            lo = __vminu2(lo, l);
+            hi = __vmaxu2(hi, h);
         }
     }
-    ylo = group_min<L>(ylo);
-    yhi = group_max<L>(yhi);
-    xlo = group_min<L>(xlo);
-    xhi = group_max<L>(xhi);
+    lo = group_min2<L>(lo);
+    hi = group_max2<L>(hi);
     Patch p;
-    p.y0 = ylo;
-    p.x0 = xlo;
-    p.h = yhi >= ylo ? yhi - ylo + 1 : 0;
-    p.w = yhi >= ylo ? xhi - xlo + 1 : 0;
+    p.y0 = (int)(lo >> 16);
+    p.x0 = (int)(lo & 0xffffu);
+    const bool any = hi != 0u;
+    p.h = any ? (int)(hi >> 16) - p.y0 : 0;
+    p.w = any ? (int)(hi & 0xffffu) - p.x0 : 0;
+    p.off = 0;
+    p.overflow = false;
+    return p;
+}
+
+// Whether merging pays for one camera: the channel loop then walks the warp's
+// largest patch two rows by two columns, against L * zn bin positions (four
+// corners each) unmerged; merging itself costs about kMergeSteps such steps.
+// Warp-uniform.
+template <int L>
+__device__ __forceinline__ bool merge_pays(const Patch& p, int zn, int merge_steps) {
+    const int hmax = __reduce_max_sync(0xffffffffu, p.h);
+    const int wmax = __reduce_max_sync(0xffffffffu, p.w);
+    return ((hmax + 1) >> 1) * ((wmax + 1) >> 1) + merge_steps < L * zn;
+}
+
+// Placement, exact merge and fp32 rounding of one camera's weights for the
+// warp's current cells into the boxes of patch_box.  rc[t] = 1 / cnt of item
+// t.  Cells whose patches do not fit the region get h = 0 and `overflow`.
+// Ends with the patch values readable by all lanes of the warp (fp32 at words
+// [off, off + h * w) of `region`).
+template <int L>
+__device__ __forceinline__ void merge_patches(Patch& p, const Items& it, const float (&rc)[kZPerLaneMax], int zn,
+                                              int sub, int ql, int Hf, int Wf, int* region) {
     int total;
     p.off = group_prefix<L>(p.h * p.w, sub, &total);
     p.overflow = p.off + p.h * p.w > kWarpPatchCap;
@@ -287,7 +312,6 @@ __device__ __forceinline__ Patch merge_patches(const Items& it, const float (&rc
         pf[p.off + e] = __fadd_rn((float)hi[p.off + e] * kTwoM20, (float)lo[p.off + e] * kTwoM40);
     }
     __syncwarp();
-    return p;
 }
 
 }  // namespace bev
