@@ -47,34 +47,31 @@ __device__ __forceinline__ void scatter_patch(const float (&d)[V][4], const floa
     }
 }
 
-// Unmerged path: each bin of the cell is broadcast to the cell's lanes, which
-// reduce w * dout into its four bilinear corners.  Corners outside the map,
-// invalid bins and cells with mine == false carry weight 0 and are skipped.
+// Fallback for cells whose patches did not fit: each valid bin's four
+// corners, broadcast from the lane that projected it.  Called by the whole
+// warp.
 template <int L, int V>
-__device__ __forceinline__ void scatter_bins(const float (&d)[V][4], const Items& it,
-                                             const float (&rc)[kZPerLaneMax], int zn, bool mine, int sub,
-                                             float* Gn, int Hf, int Wf, int tstride, int ql, int nchunks) {
-    const ptrdiff_t rs = (ptrdiff_t)Wf * tstride;
+__device__ __forceinline__ void scatter_direct(const float (&d)[V][4], const Items& it,
+                                               const float (&rc)[kZPerLaneMax], int zn, bool mine, int sub,
+                                               float* Gn, int Hf, int Wf, int tstride, int ql, int nchunks) {
 #pragma unroll
     for (int t = 0; t < kZPerLaneMax; ++t) {
         if (t >= zn) break;
-        const float rct = (mine && (it.ok >> t & 1u)) ? rc[t] : 0.0f;
-#pragma unroll 2
         for (int zz = 0; zz < L; ++zz) {
             const int src = sub * L + zz;
             const float fx = __shfl_sync(0xffffffffu, it.fx[t], src);
             const float fy = __shfl_sync(0xffffffffu, it.fy[t], src);
-            const float r = __shfl_sync(0xffffffffu, rct, src);
+            const bool ok = (__shfl_sync(0xffffffffu, it.ok, src) >> t) & 1u;
+            const float r = __shfl_sync(0xffffffffu, rc[t], src);
+            if (!(mine && ok)) continue;
             const Corners c = bilinear_corners(fx, fy);
-            const bool cx0 = (unsigned)c.x0 < (unsigned)Wf, cx1 = (unsigned)(c.x0 + 1) < (unsigned)Wf;
-            const bool cy0 = (unsigned)c.y0 < (unsigned)Hf, cy1 = (unsigned)(c.y0 + 1) < (unsigned)Hf;
-            const float wt[4] = {(cy0 && cx0) ? c.w00 * r : 0.0f, (cy0 && cx1) ? c.w01 * r : 0.0f,
-                                 (cy1 && cx0) ? c.w10 * r : 0.0f, (cy1 && cx1) ? c.w11 * r : 0.0f};
-            float* p = Gn + (ptrdiff_t)(c.y0 * Wf + c.x0) * tstride;
-            float* pp[4] = {p, p + tstride, p + rs, p + rs + tstride};
+            const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (wt[u] != 0.0f) scatter_texel<L, V>(pp[u], d, wt[u], ql, nchunks);
+            for (int k = 0; k < 4; ++k) {
+                const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
+                if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
+                scatter_texel<L, V>(Gn + ((size_t)yy * Wf + xx) * tstride, d, ws[k] * r, ql, nchunks);
+            }
         }
     }
 }
@@ -163,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(c
                 merge_patches<L>(pt, it, rc, zn, sub, ql, g.Hf, g.Wf, region);
                 scatter_patch<L, V>(d[q], reinterpret_cast<const float*>(region), pt, Gn, g.Wf, tstride, ql, nchunks);
                 if (__any_sync(0xffffffffu, pt.overflow))
-                    scatter_bins<L, V>(d[q], it, rc, zn, pt.overflow, sub, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
+                    scatter_direct<L, V>(d[q], it, rc, zn, pt.overflow, sub, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
                 __syncwarp();  // the region is rebuilt for the next camera
             }
         }
