@@ -131,6 +131,24 @@ int cuda_status(cudaError_t e) {
     return BEV_ERR_CUDA;
 }
 
+// Backward tile width: kTileJ cells, or half that when kTileJ-wide tiles
+// would not fill two waves of resident CTAs (the launch would then end on a
+// short second wave of the heaviest, near-rig tiles).  Must be a multiple
+// of the 32 / L cells a warp works on at once.
+int backward_tile_j(int L, int X, int Y, int B, int slices, int sms) {
+    const long long slots = (long long)sms * bev::kCtasPerSm;
+    const long long tiles = (long long)((X + bev::kTileI - 1) / bev::kTileI) *
+                            ((Y + bev::kTileJ - 1) / bev::kTileJ) * B * slices;
+    const int half = bev::kTileJ / 2;
+    return (tiles < 2 * slots && half % (32 / L) == 0) ? half : bev::kTileJ;
+}
+
+int sm_count(int dev, int* sms) {
+    if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *sms < 1)
+        return cuda_status(cudaErrorInvalidDevice);
+    return BEV_OK;
+}
+
 }  // namespace
 
 BEV_API const char* bev_status_string(int status) {
@@ -240,6 +258,7 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
     a.slice_chunks = (a.Qtot + slices - 1) / slices;
     int V;
     pick_lanes(a.slice_chunks, &a.L, &V);
+    a.tile_j = bev::kTileJ;
     a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
     a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
     return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, V, slices, s));
@@ -285,8 +304,11 @@ BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, 
     a.slice_chunks = (a.Qtot + slices - 1) / slices;
     int V;
     pick_lanes(a.slice_chunks, &a.L, &V);
+    int sms;
+    if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
+    a.tile_j = backward_tile_j(a.L, grid->X, grid->Y, B, slices, sms);
     a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
-    a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
+    a.tiles_j = (grid->Y + a.tile_j - 1) / a.tile_j;
     if ((st = cuda_status(bev_launch_backward(a, V, slices, s))) != BEV_OK) return st;
     return cuda_status(bev_launch_to_nchw(static_cast<const float*>(workspace), B * N, C, Hf * Wf, Cp,
                                           dfeatures, s));

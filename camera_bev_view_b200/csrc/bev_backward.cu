@@ -7,13 +7,15 @@
 //   dF[b, n, c, y, x] += (sum_k w_k / cnt_k) * dout[b, c, i, j]
 // over every (cell, camera) and every texel (y, x) its valid samples touch.
 //
-// One CTA = one 8x8 BEV tile of one batch item and one channel slice, with the
-// same culling, once-per-voxel geometry and merged per-(cell, camera, texel)
-// weights as the forward (bev_warp.cuh).  Each warp loads its row's dout slice
-// through its own shared-memory region (coalesced along y) into registers:
-// each lane owns V chunks of 4 channels of one cell.  Each touched texel then
-// receives one 16-byte vector reduction per chunk (red.global.add.v4.f32) into
-// the fp32 channels-last gradient buffer, however many height bins hit it.
+// One CTA = one tile of 8 BEV rows of one batch item and one channel slice,
+// with the same culling, once-per-voxel geometry and merged per-(cell,
+// camera, texel) weights as the forward (bev_warp.cuh).  Each lane holds
+// dout of V chunks of 4 channels of its cell in registers; each touched
+// texel then receives one 16-byte vector reduction per chunk
+// (red.global.add.v4.f32) into the fp32 channels-last gradient buffer,
+// however many height bins hit it.  The tile width is chosen per launch:
+// narrower tiles when the grid gives few tiles, so that the launch does not
+// end on a short second wave of heavy tiles.
 #include "bev_warp.cuh"
 
 namespace bev {
@@ -79,8 +81,7 @@ __device__ __forceinline__ void scatter_direct(const float (&d)[V][4], const Ite
 template <int L, int V>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(const SampleArgs a) {
     constexpr int G = 32 / L;
-    constexpr int CG = kCellsPerWarp / G;
-    static_assert(G * CG == kCellsPerWarp, "lanes per cell must be 4, 8, 16 or 32");
+    static_assert(G * L == 32, "lanes per cell must divide the warp");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const CtaSmem s = carve_smem(smem_raw, a.N);
     const GeoParams& g = a.g;
@@ -99,41 +100,29 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(c
     const int sub = lane / L, ql = lane - sub * L;
     int* region = reinterpret_cast<int*>(s.warps + (size_t)warp * (kWarpBytes + 512));
     const int i = ti0 + warp;
-
-    // dout of the warp's row -> [channel][cell] staging -> registers
-    float* stage = reinterpret_cast<float*>(region);
-    for (int t = lane; t < nchunks * 4 * kCellsPerWarp; t += 32) {
-        const int c = t >> 3, jc = t & 7;
-        float v = 0.0f;
-        if (c_base + c < a.C && i < g.X && tj0 + jc < g.Y)
-            v = a.dout[(((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0 + jc];
-        stage[c * kStageStride + jc] = v;
-    }
-    __syncwarp();
-    float d[CG][V][4];
-#pragma unroll
-    for (int q = 0; q < CG; ++q) {
-        const int jc = q * G + sub;
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-            const int c0 = (ql + v * L) * 4;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d[q][v][e] = ql + v * L < nchunks ? stage[(c0 + e) * kStageStride + jc] : 0.0f;
-        }
-    }
-    __syncwarp();
-
     const size_t texels = (size_t)g.Hf * g.Wf;
     const int tstride = a.Qtot * 4;  // floats per texel in the gradient buffer
     float* grad = a.dfeat + (size_t)(chunk0 + ql) * 4 + (size_t)b * a.N * texels * tstride;
     const float x = voxel_centre(g.xmin, i, g.dx);
     const int zn = min(kZPerLaneMax, (g.Z + L - 1) / L);
+    const size_t cstride = (size_t)g.X * g.Y;
 
-#pragma unroll
-    for (int q = 0; q < CG; ++q) {
-        const int j = tj0 + q * G + sub;
+    // G cells at a time along the warp's row of tile_j cells
+    for (int j1 = tj0; j1 < tj0 + a.tile_j; j1 += G) {
+        const int j = j1 + sub;
         const bool in_grid = i < g.X && j < g.Y;
         const float y = voxel_centre(g.ymin, j, g.dy);
+        // dout of this lane's cell and channel chunks (for one channel the G
+        // cells of the group are consecutive along y)
+        float d[V][4];
+        const float* dp = a.dout + ((size_t)b * a.C + c_base) * cstride + (size_t)i * g.Y + j;
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            const int c0 = (ql + v * L) * 4;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                d[v][e] = (in_grid && ql + v * L < nchunks && c_base + c0 + e < a.C) ? dp[(c0 + e) * cstride] : 0.0f;
+        }
         for (int z0 = 0; z0 < g.Z; z0 += L * zn) {
             // valid cameras per bin of this lane, over all active cameras; the
             // projections of the first two cameras are kept for the merge pass
@@ -158,9 +147,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(c
                 // instead of one per bin that touches it
                 Patch pt = patch_box<L>(it, zn, g.Hf, g.Wf);
                 merge_patches<L>(pt, it, rc, zn, sub, ql, g.Hf, g.Wf, region);
-                scatter_patch<L, V>(d[q], reinterpret_cast<const float*>(region), pt, Gn, g.Wf, tstride, ql, nchunks);
+                scatter_patch<L, V>(d, reinterpret_cast<const float*>(region), pt, Gn, g.Wf, tstride, ql, nchunks);
                 if (__any_sync(0xffffffffu, pt.overflow))
-                    scatter_direct<L, V>(d[q], it, rc, zn, pt.overflow, sub, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
+                    scatter_direct<L, V>(d, it, rc, zn, pt.overflow, sub, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
                 __syncwarp();  // the region is rebuilt for the next camera
             }
         }

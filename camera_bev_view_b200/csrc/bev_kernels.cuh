@@ -55,6 +55,7 @@ struct SampleArgs {
     int chan_per_chunk;     // 4 (fp32) or 8 (bf16)
     int slice_chunks;       // chunks per CTA channel slice
     int L;                  // lanes per cell (4, 8, 16 or 32)
+    int tile_j;             // cells per tile row: kTileJ (forward) or a multiple of 32 / L (backward)
     int tiles_i, tiles_j;   // tiles along X and Y
 };
 

@@ -86,7 +86,7 @@ __device__ inline void tile_origin(const SampleArgs& a, int* slot, int& ti0, int
             if (k < __popc(m)) {
                 if (inside && __popc(m & ((1u << threadIdx.x) - 1u)) == k) {
                     slot[0] = (ci + di) * kTileI;
-                    slot[1] = (cj + dj) * kTileJ;
+                    slot[1] = (cj + dj) * a.tile_j;
                 }
                 found = 1;
             } else {
@@ -115,7 +115,7 @@ __device__ inline void setup_tile(const SampleArgs& a, const CtaSmem& s, int b, 
     if ((tid >> 5) * 4 < a.N) {           // warps holding at least one camera
         float m[5] = {-1e30f, -1e30f, -1e30f, -1e30f, -1e30f};
         if (n < a.N) {
-            const int i1 = min(ti0 + kTileI, g.X) - 1, j1 = min(tj0 + kTileJ, g.Y) - 1;
+            const int i1 = min(ti0 + kTileI, g.X) - 1, j1 = min(tj0 + a.tile_j, g.Y) - 1;
             const float px = voxel_centre(g.xmin, (v & 1) ? i1 : ti0, g.dx);
             const float py = voxel_centre(g.ymin, (v & 2) ? j1 : tj0, g.dy);
             const float pz = voxel_centre(g.zmin, (v & 4) ? g.Z - 1 : 0, g.dz);
