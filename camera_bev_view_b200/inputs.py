@@ -15,6 +15,18 @@ Workloads (shapes after the LSS tutorial's worked sizes, "Lift" section:
   large       B1 N6 C80  32x88 (img 512x1408)  400x400x16 over +-50 m fp32
   backward    nuscenes shapes with B2, upstream gradient N(0,1)
 
+Deformable-aggregation workloads (SparseDriveV2 notes, "Deformable
+Aggregation": Nq queries of K keypoints each, with Nq ~ 10^2-10^3 and K in
+the tens, over six surround cameras):
+
+  deform_tiny  B1 N6 C16  8x22   (img 128x352)  Q32  K4   fp32
+  deform       B1 N6 C256 64x176 (img 512x1408) Q900 K13  fp32
+  deform_bf16  B4 N6 C256 64x176 (img 512x1408) Q900 K13  bf16
+
+Anchors are uniform over x, y in [-50, 50] m and z in [-2, 2] m; keypoint
+offsets uniform in [-2, 2] m per axis; weights uniform in [0, 1) / (N K);
+the upstream gradient is N(0, 1).
+
 z always spans [-5, 3] m.  Rig: camera n has nominal yaw 60 deg * n, sits at
 (cos yaw, sin yaw, 1.5) m plus U(-0.05, 0.05) m jitter per axis, and looks
 horizontally along yaw + U(-2, 2) deg with no pitch or roll.  Ego frame:
@@ -83,6 +95,53 @@ WORKLOADS = {
     "backward": Workload("backward", 4, 2, 6, 64, 16, 44, 256, 704, 200, 200, 8,
                          (-50.0, 50.0), (-50.0, 50.0), (-5.0, 3.0), "f32", backward=True),
 }
+
+
+@dataclasses.dataclass(frozen=True)
+class DeformWorkload:
+    name: str
+    index: int            # seed family
+    B: int
+    N: int
+    C: int
+    Hf: int
+    Wf: int
+    img_h: int
+    img_w: int
+    Q: int                # queries per batch item
+    Kp: int               # keypoints per query
+    dtype: str            # "f32" or "bf16" feature storage
+
+    @property
+    def out_elems(self):
+        return self.B * self.Q * self.C
+
+    def scaled(self, **kw):
+        return dataclasses.replace(self, **kw)
+
+
+DEFORM_WORKLOADS = {
+    "deform_tiny": DeformWorkload("deform_tiny", 10, 1, 6, 16, 8, 22, 128, 352, 32, 4, "f32"),
+    "deform": DeformWorkload("deform", 11, 1, 6, 256, 64, 176, 512, 1408, 900, 13, "f32"),
+    "deform_bf16": DeformWorkload("deform_bf16", 12, 4, 6, 256, 64, 176, 512, 1408, 900, 13, "bf16"),
+}
+
+
+def make_queries(w: DeformWorkload, shard: int = 0):
+    """(anchors [B,Q,3], offsets [B,Q,Kp,3], weights [B,Q,N,Kp]) float32 torch (CPU)."""
+    rng = np.random.default_rng(5000 + w.index + 100003 * shard)
+    anchors = np.stack([rng.uniform(-50.0, 50.0, size=(w.B, w.Q)), rng.uniform(-50.0, 50.0, size=(w.B, w.Q)),
+                        rng.uniform(-2.0, 2.0, size=(w.B, w.Q))], axis=-1)
+    offsets = rng.uniform(-2.0, 2.0, size=(w.B, w.Q, w.Kp, 3))
+    weights = rng.uniform(0.0, 1.0, size=(w.B, w.Q, w.N, w.Kp)) / (w.N * w.Kp)
+    return (torch.from_numpy(anchors.astype(np.float32)), torch.from_numpy(offsets.astype(np.float32)),
+            torch.from_numpy(weights.astype(np.float32)))
+
+
+def make_query_dout(w: DeformWorkload, shard: int = 0) -> torch.Tensor:
+    """Upstream gradient [B,Q,C] float32, i.i.d. N(0,1)."""
+    g = torch.Generator().manual_seed(6000 + w.index + 100003 * shard)
+    return torch.randn((w.B, w.Q, w.C), generator=g, dtype=torch.float32)
 
 
 def pinhole_intrinsics(img_h: int, img_w: int) -> np.ndarray:

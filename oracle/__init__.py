@@ -9,6 +9,10 @@ loop nest (FlashBEV reading notes, "Method" items 1 and 4): per height bin the
 mean over valid cameras of the bilinear samples, summed over height.  See the
 header comment of ``bev_oracle.c`` for every reading it takes.
 
+Also the deformable aggregation of the SparseDriveV2 notes ("Deformable
+Aggregation", steps 1-3): ``deform_forward`` / ``deform_backward`` (pins in
+``tests/test_oracle_deform.py``).
+
 Pins (in ``tests/test_oracle.py``): a materialised tensorized evaluation with
 ``torch.nn.functional.grid_sample`` on tiny grids, a hand-derived worked example
 (``tests/golden/``), affine and constant feature closed forms, camera
@@ -56,6 +60,11 @@ def _load():
         lib.oracle_forward.restype = None
         lib.oracle_backward.argtypes = [P, I, I, I, I, I, P, P, I, I, I, I, I, P, P, P, P, I]
         lib.oracle_backward.restype = None
+        lib.oracle_deform_forward.argtypes = [P, I, I, I, I, I, P, P, I, I, P, P, P, I, I, P, P, I]
+        lib.oracle_deform_forward.restype = None
+        lib.oracle_deform_backward.argtypes = [P, P, I, I, I, I, I, P, P, I, I, P, P, P, I, I,
+                                               P, P, P, P, P, P, I]
+        lib.oracle_deform_backward.restype = None
         _lib = lib
     return _lib
 
@@ -144,3 +153,47 @@ def backward(dout, N, Hf, Wf, K, E, img_h, img_w, grid: Grid, threads: int = 0):
                             grid.X, grid.Y, grid.Z, _ptr(grid.lo), _ptr(grid.cell),
                             _ptr(dF), _ptr(dB), threads)
     return dF, dB
+
+
+def deform_forward(features, K, E, img_h, img_w, anchors, offsets, weights, threads: int = 0):
+    """Deformable aggregation (SparseDriveV2 notes, "Deformable Aggregation"
+    steps 1-3).  features [B,N,C,Hf,Wf]; anchors [B,Q,3]; offsets [B,Q,Kp,3];
+    weights [B,Q,N,Kp].  Returns (out [B,Q,C] f64, bound [B,Q,C] f64)."""
+    F = _np(features, np.float64)
+    B, N, C, Hf, Wf = F.shape
+    A = _np(anchors, np.float32)
+    D = _np(offsets, np.float32)
+    W = _np(weights, np.float32)
+    Q, Kp = D.shape[1], D.shape[2]
+    assert A.shape == (B, Q, 3) and D.shape == (B, Q, Kp, 3) and W.shape == (B, Q, N, Kp)
+    Kc = _np(K, np.float32).reshape(B, N, 3, 3)
+    Ec = _np(E, np.float32).reshape(B, N, 4, 4)
+    out = np.zeros((B, Q, C), dtype=np.float64)
+    bound = np.zeros_like(out)
+    _load().oracle_deform_forward(_ptr(F), B, N, C, Hf, Wf, _ptr(Kc), _ptr(Ec), img_h, img_w,
+                                  _ptr(A), _ptr(D), _ptr(W), Q, Kp, _ptr(out), _ptr(bound), threads)
+    return out, bound
+
+
+def deform_backward(features, dout, K, E, img_h, img_w, anchors, offsets, weights, threads: int = 0):
+    """Gradients of the deformable aggregation for dout [B,Q,C]: returns a dict
+    with dF [B,N,C,Hf,Wf], dW [B,Q,N,Kp], dOff [B,Q,Kp,3] (f64) and their
+    bounds dF_bound, dW_bound, dOff_bound."""
+    F = _np(features, np.float64)
+    B, N, C, Hf, Wf = F.shape
+    G = _np(dout, np.float64)
+    A = _np(anchors, np.float32)
+    D = _np(offsets, np.float32)
+    W = _np(weights, np.float32)
+    Q, Kp = D.shape[1], D.shape[2]
+    assert G.shape == (B, Q, C) and W.shape == (B, Q, N, Kp)
+    Kc = _np(K, np.float32).reshape(B, N, 3, 3)
+    Ec = _np(E, np.float32).reshape(B, N, 4, 4)
+    r = {k: np.zeros(s, dtype=np.float64) for k, s in
+         [("dF", F.shape), ("dF_bound", F.shape), ("dW", W.shape), ("dW_bound", W.shape),
+          ("dOff", D.shape), ("dOff_bound", D.shape)]}
+    _load().oracle_deform_backward(_ptr(F), _ptr(G), B, N, C, Hf, Wf, _ptr(Kc), _ptr(Ec), img_h, img_w,
+                                   _ptr(A), _ptr(D), _ptr(W), Q, Kp,
+                                   _ptr(r["dF"]), _ptr(r["dF_bound"]), _ptr(r["dW"]), _ptr(r["dW_bound"]),
+                                   _ptr(r["dOff"]), _ptr(r["dOff_bound"]), threads)
+    return r

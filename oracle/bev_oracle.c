@@ -256,3 +256,192 @@ void oracle_backward(const double* dout, int B, int N, int C, int Hf, int Wf,
         }
     }
 }
+
+/* ------------------------------------------------------------------------
+ * Deformable aggregation (SparseDriveV2 notes, "Deformable Aggregation",
+ * steps 1-3): a query with 3-D anchor a and keypoint offsets d_k samples the
+ * cameras at its keypoints p_k = a + d_k (step 1), each projected as above
+ * and kept only where valid (step 2), and sums the bilinear samples with
+ * weights w_{n,k} (step 3):
+ *
+ *   out[b,q,c] = sum_n sum_k [valid(b,n,p_k)] w[b,q,n,k] * bilinear(F[b,n,c], fx, fy)
+ *
+ * Readings: the keypoint is a + d_k rounded to fp32 once per coordinate; the
+ * sampler phi of the notes is the same bilinear (align_corners=False, zero
+ * padding) as the dense path, the "small neighbourhood" being its 2x2 taps;
+ * no normalisation beyond the given weights; validity as in oracle_project.
+ * ---------------------------------------------------------------------- */
+
+static void keypoint(const float* anchors, const float* offsets, int b, int q, int k, int Q, int Kp,
+                     float p[3])
+{
+    const float* a = anchors + ((size_t)b * Q + q) * 3;
+    const float* d = offsets + (((size_t)b * Q + q) * Kp + k) * 3;
+    for (int r = 0; r < 3; ++r) p[r] = a[r] + d[r];
+}
+
+/* Forward.  F [B,N,C,Hf,Wf] fp64 (exact copies); anchors [B,Q,3], offsets
+ * [B,Q,Kp,3], weights [B,Q,N,Kp] fp32.  Writes out and bound [B,Q,C] fp64. */
+void oracle_deform_forward(const double* F, int B, int N, int C, int Hf, int Wf,
+                           const float* K, const float* E, int img_h, int img_w,
+                           const float* anchors, const float* offsets, const float* W, int Q, int Kp,
+                           double* out, double* bound, int threads)
+{
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic)
+#endif
+    for (long bq = 0; bq < (long)B * Q; ++bq) {
+        int b = (int)(bq / Q), q = (int)(bq % Q);
+        double* acc = out + (size_t)bq * C;
+        double* abs_acc = bound + (size_t)bq * C;
+        for (int c = 0; c < C; ++c) { acc[c] = 0.0; abs_acc[c] = 0.0; }
+        for (int n = 0; n < N; ++n) {
+            const float* Kn = K + ((size_t)b * N + n) * 9;
+            const float* En = E + ((size_t)b * N + n) * 16;
+            for (int k = 0; k < Kp; ++k) {
+                float p[3], u, v, fx, fy;
+                keypoint(anchors, offsets, b, q, k, Q, Kp, p);
+                if (!oracle_project(Kn, En, p[0], p[1], p[2], img_h, img_w, Hf, Wf, &u, &v, &fx, &fy))
+                    continue;
+                double w = W[(((size_t)b * Q + q) * N + n) * Kp + k];
+                int ys[4], xs[4];
+                float ws[4];
+                corners(fx, fy, ys, xs, ws);
+                for (int t = 0; t < 4; ++t) {
+                    if (ys[t] < 0 || ys[t] >= Hf || xs[t] < 0 || xs[t] >= Wf) continue;
+                    const double* Fp = F + (((size_t)b * N + n) * C * Hf + ys[t]) * Wf + xs[t];
+                    for (int c = 0; c < C; ++c) {
+                        double term = w * (double)ws[t] * Fp[(size_t)c * Hf * Wf];
+                        acc[c] += term;
+                        abs_acc[c] += fabs(term);
+                    }
+                }
+            }
+        }
+    }
+}
+
+/* Backward for dout [B,Q,C] fp64:
+ *   dF [B,N,C,Hf,Wf]  adjoint of the forward in F;
+ *   dW [B,Q,N,Kp]     sum_c dout * bilinear(F, fx, fy)  for valid (n, k), else 0;
+ *   dOff [B,Q,Kp,3]   derivative through the sampling position: with
+ *                     g = sum_c dout_c dphi_c/d(fx, fy) (the derivative of the
+ *                     zero-padded bilinear interpolant inside its cell),
+ *                     fx = u Wf/W_img - 0.5, u = uh / pc_z, pc = R p + t:
+ *                     dOff += w * R^T (g_x (Wf/W_img) du/dpc + g_y (Hf/H_img) dv/dpc),
+ *                     du/dpc = (K_00, K_01, K_02 - u) / pc_z, likewise v.
+ *                     The validity test and the corner choice are held fixed
+ *                     (no gradient flows through them), as for the dense path.
+ * Each output gets a bound (sum of absolute terms) of the same shape.  dF is
+ * split over (b, n), dW and dOff over (b, q). */
+void oracle_deform_backward(const double* F, const double* dout, int B, int N, int C, int Hf, int Wf,
+                            const float* K, const float* E, int img_h, int img_w,
+                            const float* anchors, const float* offsets, const float* W, int Q, int Kp,
+                            double* dF, double* dFb, double* dW, double* dWb, double* dOff, double* dOffb,
+                            int threads)
+{
+    memset(dF, 0, sizeof(double) * (size_t)B * N * C * Hf * Wf);
+    memset(dFb, 0, sizeof(double) * (size_t)B * N * C * Hf * Wf);
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic)
+#endif
+    for (long bn = 0; bn < (long)B * N; ++bn) {
+        int b = (int)(bn / N), n = (int)(bn % N);
+        const float* Kn = K + ((size_t)b * N + n) * 9;
+        const float* En = E + ((size_t)b * N + n) * 16;
+        double* dFn = dF + (size_t)bn * C * Hf * Wf;
+        double* dBn = dFb + (size_t)bn * C * Hf * Wf;
+        for (int q = 0; q < Q; ++q) {
+            const double* g = dout + ((size_t)b * Q + q) * C;
+            for (int k = 0; k < Kp; ++k) {
+                float p[3], u, v, fx, fy;
+                keypoint(anchors, offsets, b, q, k, Q, Kp, p);
+                if (!oracle_project(Kn, En, p[0], p[1], p[2], img_h, img_w, Hf, Wf, &u, &v, &fx, &fy))
+                    continue;
+                double w = W[(((size_t)b * Q + q) * N + n) * Kp + k];
+                int ys[4], xs[4];
+                float ws[4];
+                corners(fx, fy, ys, xs, ws);
+                for (int t = 0; t < 4; ++t) {
+                    if (ys[t] < 0 || ys[t] >= Hf || xs[t] < 0 || xs[t] >= Wf) continue;
+                    for (int c = 0; c < C; ++c) {
+                        double term = w * (double)ws[t] * g[c];
+                        size_t o = ((size_t)c * Hf + ys[t]) * Wf + xs[t];
+                        dFn[o] += term;
+                        dBn[o] += fabs(term);
+                    }
+                }
+            }
+        }
+    }
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic)
+#endif
+    for (long bq = 0; bq < (long)B * Q; ++bq) {
+        int b = (int)(bq / Q), q = (int)(bq % Q);
+        const double* g = dout + (size_t)bq * C;
+        double* dO = dOff + (size_t)bq * Kp * 3;
+        double* dOb = dOffb + (size_t)bq * Kp * 3;
+        for (int t = 0; t < Kp * 3; ++t) { dO[t] = 0.0; dOb[t] = 0.0; }
+        for (int n = 0; n < N; ++n) {
+            const float* Kn = K + ((size_t)b * N + n) * 9;
+            const float* En = E + ((size_t)b * N + n) * 16;
+            for (int k = 0; k < Kp; ++k) {
+                size_t wi = (((size_t)b * Q + q) * N + n) * Kp + k;
+                dW[wi] = 0.0;
+                dWb[wi] = 0.0;
+                float p[3], u, v, fx, fy;
+                keypoint(anchors, offsets, b, q, k, Q, Kp, p);
+                if (!oracle_project(Kn, En, p[0], p[1], p[2], img_h, img_w, Hf, Wf, &u, &v, &fx, &fy))
+                    continue;
+                double w = W[wi];
+                int ys[4], xs[4];
+                float ws[4];
+                corners(fx, fy, ys, xs, ws);
+                /* d(weight of corner t)/dfx and /dfy inside the cell */
+                double wx1 = (double)fx - floor((double)fx), wy1 = (double)fy - floor((double)fy);
+                double wx0 = 1.0 - wx1, wy0 = 1.0 - wy1;
+                double dwx[4] = {-wy0, wy0, -wy1, wy1};
+                double dwy[4] = {-wx0, -wx1, wx0, wx1};
+                double s = 0.0, sb = 0.0, gx = 0.0, gxb = 0.0, gy = 0.0, gyb = 0.0;
+                for (int t = 0; t < 4; ++t) {
+                    if (ys[t] < 0 || ys[t] >= Hf || xs[t] < 0 || xs[t] >= Wf) continue;
+                    const double* Fp = F + (((size_t)b * N + n) * C * Hf + ys[t]) * Wf + xs[t];
+                    for (int c = 0; c < C; ++c) {
+                        double fg = Fp[(size_t)c * Hf * Wf] * g[c];
+                        s += (double)ws[t] * fg;
+                        sb += fabs((double)ws[t] * fg);
+                        gx += dwx[t] * fg;
+                        gxb += fabs(dwx[t] * fg);
+                        gy += dwy[t] * fg;
+                        gyb += fabs(dwy[t] * fg);
+                    }
+                }
+                dW[wi] = s;
+                dWb[wi] = sb;
+                /* chain rule through the projection, in fp64 */
+                double pc[3];
+                for (int r = 0; r < 3; ++r)
+                    pc[r] = (double)En[4 * r] * p[0] + (double)En[4 * r + 1] * p[1] + (double)En[4 * r + 2] * p[2] +
+                            (double)En[4 * r + 3];
+                double uu = ((double)Kn[0] * pc[0] + (double)Kn[1] * pc[1] + (double)Kn[2] * pc[2]) / pc[2];
+                double vv = ((double)Kn[3] * pc[0] + (double)Kn[4] * pc[1] + (double)Kn[5] * pc[2]) / pc[2];
+                double sW = (double)((float)Wf / (float)img_w), sH = (double)((float)Hf / (float)img_h);
+                double du[3] = {Kn[0] / pc[2], Kn[1] / pc[2], (Kn[2] - uu) / pc[2]};
+                double dv[3] = {Kn[3] / pc[2], Kn[4] / pc[2], (Kn[5] - vv) / pc[2]};
+                for (int d = 0; d < 3; ++d) {
+                    double val = 0.0, vb = 0.0;
+                    for (int r = 0; r < 3; ++r) {
+                        double R = En[4 * r + d];
+                        val += R * (gx * sW * du[r] + gy * sH * dv[r]);
+                        vb += fabs(R) * (gxb * sW * fabs(du[r]) + gyb * sH * fabs(dv[r]));
+                    }
+                    dO[k * 3 + d] += w * val;
+                    dOb[k * 3 + d] += fabs(w) * vb;
+                }
+            }
+        }
+    }
+}

@@ -82,3 +82,61 @@ def tensorized_backward(dout, N, Hf, Wf, K, E, ranges, counts, img_h, img_w):
     out, _, amb = tensorized_forward(F, K, E, ranges, counts, img_h, img_w)
     (out * dout).sum().backward()
     return F.grad, amb
+
+
+# --------------------------------------------------------------------------
+# Deformable aggregation (SparseDriveV2 notes, "Deformable Aggregation"
+# steps 1-3), materialised: every (b, n, q, k) keypoint projected in float64,
+# the validity mask, a grid_sample of every keypoint in every camera, the
+# masked weighted sum.  Differentiable in the features, the weights and the
+# offsets (autograd through grid_sample's sampling grid).
+# --------------------------------------------------------------------------
+
+def deform_keypoints(anchors, offsets, offsets64=None):
+    """p = a + d, valued as the float32 sum; when ``offsets64`` (float64,
+    requiring grad) is given the result carries its gradient with slope 1."""
+    p32 = (torch.as_tensor(anchors, dtype=torch.float32)[:, :, None, :] +
+           torch.as_tensor(offsets, dtype=torch.float32)).to(torch.float64)
+    if offsets64 is None:
+        return p32
+    return p32 + (offsets64 - offsets64.detach())
+
+
+def deform_project(K, E, p, img_h, img_w):
+    """uv, depth, mask for every (b, n, q, k): float64, shapes [B,N,Q,Kp]."""
+    K = torch.as_tensor(K, dtype=torch.float64)
+    E = torch.as_tensor(E, dtype=torch.float64)
+    cam = torch.einsum("bnrk,bqtk->bnqtr", E[:, :, :3, :3], p) + E[:, :, None, None, :3, 3]
+    pix = torch.einsum("bnrk,bnqtk->bnqtr", K, cam)
+    depth = cam[..., 2]
+    safe = torch.where(depth.abs() > 1e-12, depth, torch.ones_like(depth))
+    u = pix[..., 0] / safe
+    v = pix[..., 1] / safe
+    mask = (depth > 0.1) & (u >= 0) & (u <= img_w) & (v >= 0) & (v <= img_h)
+    return u, v, depth, mask
+
+
+def tensorized_deform(features, K, E, img_h, img_w, anchors, offsets, weights, offsets64=None):
+    """Returns (out [B,Q,C], mask [B,N,Q,Kp], ambiguous [B,N,Q,Kp], fx, fy)."""
+    F = torch.as_tensor(features)
+    if F.dtype != torch.float64:
+        F = F.to(torch.float64)
+    B, N, C, Hf, Wf = F.shape
+    W = torch.as_tensor(weights)
+    if W.dtype != torch.float64:
+        W = W.to(torch.float64)
+    p = deform_keypoints(anchors, offsets, offsets64)                      # [B,Q,Kp,3]
+    Q, Kp = p.shape[1], p.shape[2]
+    u, v, depth, mask = deform_project(K, E, p, img_h, img_w)
+    gx = 2.0 * u / img_w - 1.0
+    gy = 2.0 * v / img_h - 1.0
+    grid = torch.stack([gx, gy], dim=-1)
+    grid = torch.where(mask[..., None], grid, torch.zeros_like(grid))
+    phi = Fn.grid_sample(F.reshape(B * N, C, Hf, Wf), grid.reshape(B * N, Q, Kp, 2), mode="bilinear",
+                         padding_mode="zeros", align_corners=False).reshape(B, N, C, Q, Kp)
+    wm = W.permute(0, 2, 1, 3) * mask.to(torch.float64)                    # [B,N,Q,Kp]
+    out = torch.einsum("bncqk,bnqk->bqc", phi, wm)
+    amb = ambiguous(u, v, depth, img_h, img_w)
+    fx = u * (Wf / img_w) - 0.5
+    fy = v * (Hf / img_h) - 0.5
+    return out, mask, amb, fx, fy

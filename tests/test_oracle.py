@@ -122,6 +122,7 @@ CASES = [
     ("random", 13, 3, 4, 6, 10, 48, 80, (-10, 10, -8, 8, -2, 4), (8, 7, 2)),
     ("random", 14, 2, 2, 5, 7, 40, 56, (-4, 4, -4, 4, -1, 3), (6, 8, 3)),
     ("random", 15, 3, 3, 9, 5, 72, 40, (-20, 20, -20, 20, -4, 4), (5, 5, 3)),
+    ("random", 16, 3, 3, 8, 11, 64, 176, (-12, 12, -12, 12, -2, 3), (6, 7, 3)),  # row / column strides differ
 ]
 
 
@@ -143,7 +144,7 @@ def test_oracle_matches_tensorized_forward(case):
     assert err.transpose(0, 2, 3, 1)[cell_ok].max() < 2e-3
 
 
-@pytest.mark.parametrize("case", CASES[:3], ids=[f"{c[0]}{c[1]}" for c in CASES[:3]])
+@pytest.mark.parametrize("case", CASES[:3] + CASES[5:], ids=[f"{c[0]}{c[1]}" for c in CASES[:3] + CASES[5:]])
 def test_oracle_backward_matches_autograd_of_tensorized(case):
     kind, seed, N, C, Hf, Wf, ih, iw, ranges, counts = case
     K, E = _rig(kind, seed, N, ih, iw)
