@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include "bev_deform.cuh"
 #include "bev_kernels.cuh"
 #include "bevsample.h"
 
@@ -326,4 +327,151 @@ BEV_API int bev_features_to_channels_last(const void* features, int dtype, int B
     if ((st = device_ptr(out, dev)) != BEV_OK) return st;
     return cuda_status(bev_launch_to_channels_last(features, BEV_NCHW, elem_size(dtype), B * N, C, Hf * Wf,
                                                    C, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------------------
+// Deformable aggregation
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kDeformMaxChunks = 128;  // 32 lanes x 4 chunks of 16 bytes
+
+bool deform_dims_ok(int B, int N, int C, int Hf, int Wf, int Q, int Kp) {
+    if (!dims_ok(B, N, C, Hf, Wf)) return false;
+    if (Q < 1 || Q > (1 << 26) || Kp < 1 || Kp > BEV_DEFORM_MAX_KEYPOINTS) return false;
+    return true;
+}
+
+// Channels-last fp32 gradient buffer of the backward: chunk channels per texel.
+size_t deform_grad_bytes(int dtype, int B, int N, int C, int Hf, int Wf) {
+    return (size_t)B * N * Hf * Wf * round_up(C, chan_per_chunk(dtype)) * sizeof(float);
+}
+
+size_t deform_ws(int dtype, int layout, int B, int N, int C, int Hf, int Wf, int for_backward) {
+    const size_t rep = forward_ws(dtype, layout, B, N, C, Hf, Wf);
+    if (!for_backward) return rep;
+    return align_up(rep) + align_up(deform_grad_bytes(dtype, B, N, C, Hf, Wf));
+}
+
+bev::GeoParams deform_geo(int Hf, int Wf, int img_h, int img_w) {
+    bev::GeoParams p;
+    memset(&p, 0, sizeof(p));
+    p.img_w = (float)img_w;
+    p.img_h = (float)img_h;
+    p.sW = (float)Wf / (float)img_w;
+    p.sH = (float)Hf / (float)img_h;
+    p.Hf = Hf;
+    p.Wf = Wf;
+    return p;
+}
+
+// Shared checks and set-up of both deformable calls: validates, repacks the
+// features to channels-last when needed and fills the launch arguments.
+int deform_prepare(const void* features, int dtype, int layout, int B, int N, int C, int Hf, int Wf,
+                   const float* K, const float* E, int img_h, int img_w, const float* anchors,
+                   const float* offsets, const float* weights, int Q, int Kp, void* workspace,
+                   size_t workspace_bytes, int for_backward, const void* const* extra, int n_extra,
+                   cudaStream_t s, bev::DeformArgs* a, int* V, int* dev_out) {
+    if (!features || !K || !E || !anchors || !offsets || !weights) return BEV_ERR_INVALID_ARG;
+    for (int k = 0; k < n_extra; ++k)
+        if (!extra[k]) return BEV_ERR_INVALID_ARG;
+    if (!deform_dims_ok(B, N, C, Hf, Wf, Q, Kp)) return BEV_ERR_INVALID_ARG;
+    if (img_h < 1 || img_w < 1 || img_h > BEV_MAX_DIM || img_w > BEV_MAX_DIM) return BEV_ERR_INVALID_ARG;
+    if (dtype != BEV_F32 && dtype != BEV_BF16) return BEV_ERR_UNSUPPORTED;
+    if (layout != BEV_NCHW && layout != BEV_NHWC) return BEV_ERR_UNSUPPORTED;
+    const int cpc = chan_per_chunk(dtype);
+    const int Qtot = round_up(C, cpc) / cpc;
+    if (Qtot > kDeformMaxChunks) return BEV_ERR_UNSUPPORTED;
+    const bool repack = needs_repack(dtype, layout, C);
+    const size_t ws_need = deform_ws(dtype, layout, B, N, C, Hf, Wf, for_backward);
+    if (ws_need > 0 && (!workspace || workspace_bytes < ws_need || ((uintptr_t)workspace % kAlign) != 0))
+        return BEV_ERR_WORKSPACE;
+    if (!repack && ((uintptr_t)features % 16) != 0) return BEV_ERR_INVALID_ARG;
+
+    int dev;
+    int st = current_device(&dev);
+    if (st != BEV_OK) return st;
+    const void* ptrs[6] = {features, K, E, anchors, offsets, weights};
+    for (int k = 0; k < 6; ++k)
+        if ((st = device_ptr(ptrs[k], dev)) != BEV_OK) return st;
+    for (int k = 0; k < n_extra; ++k)
+        if ((st = device_ptr(extra[k], dev)) != BEV_OK) return st;
+    if (ws_need > 0 && (st = device_ptr(workspace, dev)) != BEV_OK) return BEV_ERR_WORKSPACE;
+
+    const void* feat = features;
+    if (repack) {
+        st = cuda_status(bev_launch_to_channels_last(features, layout, elem_size(dtype), B * N, C, Hf * Wf,
+                                                     Qtot * cpc, workspace, s));
+        if (st != BEV_OK) return st;
+        feat = workspace;
+    }
+    memset(a, 0, sizeof(*a));
+    a->feat = feat;
+    a->K = K;
+    a->E = E;
+    a->anchors = anchors;
+    a->offsets = offsets;
+    a->weights = weights;
+    a->g = deform_geo(Hf, Wf, img_h, img_w);
+    a->B = B;
+    a->N = N;
+    a->C = C;
+    a->Q = Q;
+    a->Kp = Kp;
+    a->Qtot = Qtot;
+    a->chan_per_chunk = cpc;
+    *V = (Qtot + 31) / 32;
+    *dev_out = dev;
+    return BEV_OK;
+}
+
+}  // namespace
+
+BEV_API size_t bev_deform_workspace_size(int dtype, int layout, int B, int N, int C, int Hf, int Wf,
+                                         int for_backward) {
+    if (!dims_ok(B, N, C, Hf, Wf)) return (size_t)-1;
+    if ((dtype != BEV_F32 && dtype != BEV_BF16) || (layout != BEV_NCHW && layout != BEV_NHWC))
+        return (size_t)-1;
+    return deform_ws(dtype, layout, B, N, C, Hf, Wf, for_backward);
+}
+
+BEV_API int bev_deform_forward(const void* features, int dtype, int layout, int B, int N, int C, int Hf, int Wf,
+                               const float* intrinsics, const float* ego2cam, int img_h, int img_w,
+                               const float* anchors, const float* offsets, const float* weights, int Q, int Kp,
+                               float* out, void* workspace, size_t workspace_bytes, bev_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const void* extra[1] = {out};
+    bev::DeformArgs a;
+    int V, dev;
+    int st = deform_prepare(features, dtype, layout, B, N, C, Hf, Wf, intrinsics, ego2cam, img_h, img_w, anchors,
+                            offsets, weights, Q, Kp, workspace, workspace_bytes, 0, extra, 1, s, &a, &V, &dev);
+    if (st != BEV_OK) return st;
+    a.out = out;
+    a.vec_out = (C % a.chan_per_chunk == 0) && ((uintptr_t)out % 16 == 0);
+    return cuda_status(bev_launch_deform_forward(a, dtype == BEV_BF16, V, s));
+}
+
+BEV_API int bev_deform_backward(const void* features, int dtype, int layout, int B, int N, int C, int Hf, int Wf,
+                                const float* intrinsics, const float* ego2cam, int img_h, int img_w,
+                                const float* anchors, const float* offsets, const float* weights, int Q, int Kp,
+                                const float* dout, float* dfeatures, float* dweights, float* doffsets,
+                                void* workspace, size_t workspace_bytes, bev_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const void* extra[4] = {dout, dfeatures, dweights, doffsets};
+    bev::DeformArgs a;
+    int V, dev;
+    int st = deform_prepare(features, dtype, layout, B, N, C, Hf, Wf, intrinsics, ego2cam, img_h, img_w, anchors,
+                            offsets, weights, Q, Kp, workspace, workspace_bytes, 1, extra, 4, s, &a, &V, &dev);
+    if (st != BEV_OK) return st;
+    const size_t rep = align_up(forward_ws(dtype, layout, B, N, C, Hf, Wf));
+    float* grad = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + rep);
+    const size_t gbytes = deform_grad_bytes(dtype, B, N, C, Hf, Wf);
+    if ((st = cuda_status(cudaMemsetAsync(grad, 0, gbytes, s))) != BEV_OK) return st;
+    a.dout = dout;
+    a.dfeat = grad;
+    a.dweights = dweights;
+    a.doffsets = doffsets;
+    if ((st = cuda_status(bev_launch_deform_backward(a, dtype == BEV_BF16, V, s))) != BEV_OK) return st;
+    return cuda_status(bev_launch_to_nchw(grad, B * N, C, Hf * Wf, a.Qtot * a.chan_per_chunk, dfeatures, s));
 }

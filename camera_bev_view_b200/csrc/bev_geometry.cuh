@@ -37,10 +37,16 @@ __device__ __forceinline__ float cam_row(const float* e, float x, float y, float
     return __fadd_rn(t, e[3]);
 }
 
-// Project one voxel centre through one camera.  On success writes the
-// feature-map sampling position (fx, fy) and returns true.
-__device__ __forceinline__ bool project_voxel(const float* cam, float x, float y, float z,
-                                              const GeoParams& g, float& fx, float& fy) {
+// Image-plane quantities of one projection, for derivatives through it.
+struct ProjDetail {
+    float u, v, depth;
+};
+
+// Project one point (ego frame) through one camera.  On success writes the
+// feature-map sampling position (fx, fy) and returns true; `det` receives
+// u, v and the depth whenever the depth test passes.
+__device__ __forceinline__ bool project_point(const float* cam, float x, float y, float z, const GeoParams& g,
+                                              float& fx, float& fy, ProjDetail& det) {
     const float pcx = cam_row(cam + 0, x, y, z);
     const float pcy = cam_row(cam + 4, x, y, z);
     const float depth = cam_row(cam + 8, x, y, z);
@@ -52,10 +58,20 @@ __device__ __forceinline__ bool project_voxel(const float* cam, float x, float y
     vh = __fadd_rn(vh, __fmul_rn(k[5], depth));
     const float u = __fdiv_rn(uh, depth);
     const float v = __fdiv_rn(vh, depth);
+    det.u = u;
+    det.v = v;
+    det.depth = depth;
     if (!(u >= 0.0f && u <= g.img_w && v >= 0.0f && v <= g.img_h)) return false;
     fx = __fadd_rn(__fmul_rn(u, g.sW), -0.5f);
     fy = __fadd_rn(__fmul_rn(v, g.sH), -0.5f);
     return true;
+}
+
+// Project one voxel centre through one camera (see project_point).
+__device__ __forceinline__ bool project_voxel(const float* cam, float x, float y, float z,
+                                              const GeoParams& g, float& fx, float& fy) {
+    ProjDetail det;
+    return project_point(cam, x, y, z, g, fx, fy, det);
 }
 
 // Bilinear corners of (fx, fy): top-left texel and the four weights

@@ -13,6 +13,10 @@ The functions keep the C names:
     bev_sample_backward(dout, K, E, img_h, img_w, grid, N, Hf, Wf, ...) -> dfeatures
     bev_sample_backward_noalloc(dout, K, E, img_h, img_w, grid, N, Hf, Wf, out) -> dfeatures
     bev_features_to_channels_last(features, out=None) -> [B,N,Hf,Wf,C] copy
+    bev_deform_workspace_size(dtype, layout, B, N, C, Hf, Wf, for_backward) -> int
+    bev_deform_forward(features, K, E, img_h, img_w, anchors, offsets, weights, ...) -> [B,Q,C]
+    bev_deform_backward(features, K, E, img_h, img_w, anchors, offsets, weights, dout, ...)
+                                                     -> (dfeatures, dweights, doffsets)
     bev_status_string(status)                        -> str
 """
 from __future__ import annotations
@@ -81,6 +85,12 @@ def lib():
         L.bev_sample_backward_noalloc.restype = I
         L.bev_features_to_channels_last.argtypes = [P, I, I, I, I, I, I, P, P]
         L.bev_features_to_channels_last.restype = I
+        L.bev_deform_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+        L.bev_deform_workspace_size.restype = S
+        L.bev_deform_forward.argtypes = [P, I, I, I, I, I, I, I, P, P, I, I, P, P, P, I, I, P, P, S, P]
+        L.bev_deform_forward.restype = I
+        L.bev_deform_backward.argtypes = [P, I, I, I, I, I, I, I, P, P, I, I, P, P, P, I, I, P, P, P, P, P, S, P]
+        L.bev_deform_backward.restype = I
         L.bev_status_string.argtypes = [I]
         L.bev_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -201,3 +211,65 @@ def bev_sample_backward_noalloc(dout: torch.Tensor, K: torch.Tensor, E: torch.Te
     if st != 0:
         raise BevError(st, "bev_sample_backward_noalloc")
     return out
+
+
+def bev_deform_workspace_size(dtype: int, layout: int, B: int, N: int, C: int, Hf: int, Wf: int,
+                              for_backward: int) -> int:
+    v = lib().bev_deform_workspace_size(dtype, layout, B, N, C, Hf, Wf, for_backward)
+    if v == ctypes.c_size_t(-1).value:
+        raise BevError(-1, "bev_deform_workspace_size")
+    return int(v)
+
+
+def _feature_dims(features: torch.Tensor, layout: int):
+    if layout == NCHW:
+        B, N, C, Hf, Wf = features.shape
+    else:
+        B, N, Hf, Wf, C = features.shape
+    return B, N, C, Hf, Wf
+
+
+def bev_deform_forward(features: torch.Tensor, K: torch.Tensor, E: torch.Tensor, img_h: int, img_w: int,
+                       anchors: torch.Tensor, offsets: torch.Tensor, weights: torch.Tensor, layout: int = NCHW,
+                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """Deformable aggregation on device tensors: anchors [B,Q,3], offsets
+    [B,Q,Kp,3], weights [B,Q,N,Kp] (fp32).  Returns out [B,Q,C] fp32."""
+    B, N, C, Hf, Wf = _feature_dims(features, layout)
+    Q, Kp = offsets.shape[1], offsets.shape[2]
+    dev = features.device
+    dtype = _dtype_code(features)
+    if out is None:
+        out = torch.empty((B, Q, C), dtype=torch.float32, device=dev)
+    ws, ws_bytes = _workspace(bev_deform_workspace_size(dtype, layout, B, N, C, Hf, Wf, 0), dev, workspace)
+    st = lib().bev_deform_forward(
+        features.data_ptr(), dtype, layout, B, N, C, Hf, Wf, K.data_ptr(), E.data_ptr(), int(img_h), int(img_w),
+        anchors.data_ptr(), offsets.data_ptr(), weights.data_ptr(), Q, Kp, out.data_ptr(),
+        ws.data_ptr() if ws is not None else None, ws_bytes, _stream_ptr(stream))
+    if st != 0:
+        raise BevError(st, "bev_deform_forward")
+    return out
+
+
+def bev_deform_backward(features: torch.Tensor, K: torch.Tensor, E: torch.Tensor, img_h: int, img_w: int,
+                        anchors: torch.Tensor, offsets: torch.Tensor, weights: torch.Tensor, dout: torch.Tensor,
+                        layout: int = NCHW, out: tuple | None = None, workspace: torch.Tensor | None = None,
+                        stream=None):
+    """Gradients for dout [B,Q,C]: returns (dfeatures [B,N,C,Hf,Wf], dweights
+    [B,Q,N,Kp], doffsets [B,Q,Kp,3]), all fp32."""
+    B, N, C, Hf, Wf = _feature_dims(features, layout)
+    Q, Kp = offsets.shape[1], offsets.shape[2]
+    dev = features.device
+    dtype = _dtype_code(features)
+    if out is None:
+        out = (torch.empty((B, N, C, Hf, Wf), dtype=torch.float32, device=dev),
+               torch.empty((B, Q, N, Kp), dtype=torch.float32, device=dev),
+               torch.empty((B, Q, Kp, 3), dtype=torch.float32, device=dev))
+    dF, dW, dO = out
+    ws, ws_bytes = _workspace(bev_deform_workspace_size(dtype, layout, B, N, C, Hf, Wf, 1), dev, workspace)
+    st = lib().bev_deform_backward(
+        features.data_ptr(), dtype, layout, B, N, C, Hf, Wf, K.data_ptr(), E.data_ptr(), int(img_h), int(img_w),
+        anchors.data_ptr(), offsets.data_ptr(), weights.data_ptr(), Q, Kp, dout.data_ptr(), dF.data_ptr(),
+        dW.data_ptr(), dO.data_ptr(), ws.data_ptr() if ws is not None else None, ws_bytes, _stream_ptr(stream))
+    if st != 0:
+        raise BevError(st, "bev_deform_backward")
+    return dF, dW, dO

@@ -178,6 +178,62 @@ int bev_sample_backward_noalloc(const float* dout, int B, int N, int C, int Hf, 
 int bev_features_to_channels_last(const void* features, int dtype, int B, int N, int C, int Hf, int Wf,
                                   void* out, bev_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Deformable aggregation (SparseDriveV2 notes, "Deformable Aggregation",
+ * steps 1-3).  Each query q of batch item b has a 3-D anchor a and Kp
+ * keypoint offsets d_k; its keypoints p_k = a + d_k (fp32 sums, ego frame)
+ * are projected into every camera with the same geometry and validity test
+ * as bev_sample_forward, sampled bilinearly (align_corners=False, zero
+ * padding) where valid, and summed with per-(camera, keypoint) weights:
+ *   out[b, q, c] = sum_n sum_k [valid(b, n, p_k)] w[b, q, n, k] * bilinear(F[b, n, c], p_k)
+ * There is no normalisation beyond the given weights.
+ * ------------------------------------------------------------------------- */
+
+/* Keypoints per query accepted by the deformable-aggregation calls. */
+#define BEV_DEFORM_MAX_KEYPOINTS 64
+
+/* Device scratch (bytes, 256-byte aligned) that bev_deform_forward
+ * (for_backward = 0) or bev_deform_backward (for_backward = 1) needs; 0 when
+ * none.  (size_t)-1 for invalid arguments. */
+size_t bev_deform_workspace_size(int dtype, int layout, int B, int N, int C, int Hf, int Wf, int for_backward);
+
+/* Forward of the deformable aggregation.
+ *   features     as for bev_sample_forward; C <= 512 (fp32) or 1024 (bf16)
+ *   intrinsics, ego2cam, img_h, img_w   as for bev_sample_forward
+ *   anchors      [B,Q,3] fp32, ego frame
+ *   offsets      [B,Q,Kp,3] fp32
+ *   weights      [B,Q,N,Kp] fp32
+ *   Q, Kp        queries per batch item (>= 1), keypoints per query
+ *                (1..BEV_DEFORM_MAX_KEYPOINTS)
+ *   out          [B,Q,C] fp32, fully overwritten
+ *   workspace    at least bev_deform_workspace_size(dtype, layout, ..., 0) bytes
+ * Every output is computed by one warp in a fixed order, so results are
+ * reproducible bit for bit.  Returns BEV_OK, BEV_ERR_INVALID_ARG,
+ * BEV_ERR_UNSUPPORTED, BEV_ERR_WORKSPACE or BEV_ERR_CUDA. */
+int bev_deform_forward(const void* features, int dtype, int layout, int B, int N, int C, int Hf, int Wf,
+                       const float* intrinsics, const float* ego2cam, int img_h, int img_w,
+                       const float* anchors, const float* offsets, const float* weights, int Q, int Kp,
+                       float* out, void* workspace, size_t workspace_bytes, bev_stream_t stream);
+
+/* Backward of the deformable aggregation for dout [B,Q,C] fp32:
+ *   dfeatures  [B,N,C,Hf,Wf] fp32   adjoint in the features
+ *   dweights   [B,Q,N,Kp] fp32      the sample against dout for valid (n, k), else 0
+ *   doffsets   [B,Q,Kp,3] fp32      through the sampling position: the bilinear
+ *              derivative inside its cell, carried through u = uh / depth and
+ *              the extrinsic rotation; the validity test and the choice of cell
+ *              are held fixed (no gradient flows through them).  The anchor
+ *              gradient is the sum of a query's keypoint rows.
+ * All three are fully overwritten.  features as for bev_deform_forward (the
+ * backward reads them for dweights and doffsets); workspace at least
+ * bev_deform_workspace_size(.., 1) bytes.  dweights and doffsets are
+ * reproducible bit for bit; dfeatures is accumulated with atomics, so repeated
+ * calls may differ in the last bits. */
+int bev_deform_backward(const void* features, int dtype, int layout, int B, int N, int C, int Hf, int Wf,
+                        const float* intrinsics, const float* ego2cam, int img_h, int img_w,
+                        const float* anchors, const float* offsets, const float* weights, int Q, int Kp,
+                        const float* dout, float* dfeatures, float* dweights, float* doffsets,
+                        void* workspace, size_t workspace_bytes, bev_stream_t stream);
+
 /* Static, human-readable text for a status code. */
 const char* bev_status_string(int status);
 

@@ -431,12 +431,16 @@ void oracle_deform_backward(const double* F, const double* dout, int B, int N, i
                 double sW = (double)((float)Wf / (float)img_w), sH = (double)((float)Hf / (float)img_h);
                 double du[3] = {Kn[0] / pc[2], Kn[1] / pc[2], (Kn[2] - uu) / pc[2]};
                 double dv[3] = {Kn[3] / pc[2], Kn[4] / pc[2], (Kn[5] - vv) / pc[2]};
+                /* magnitudes for the bound: K_02 - u cancels near the principal
+                 * point, so its rounding scales with |K_02| + |u| */
+                double adu[3] = {fabs(du[0]), fabs(du[1]), (fabs(Kn[2]) + fabs(uu)) / fabs(pc[2])};
+                double adv[3] = {fabs(dv[0]), fabs(dv[1]), (fabs(Kn[5]) + fabs(vv)) / fabs(pc[2])};
                 for (int d = 0; d < 3; ++d) {
                     double val = 0.0, vb = 0.0;
                     for (int r = 0; r < 3; ++r) {
                         double R = En[4 * r + d];
                         val += R * (gx * sW * du[r] + gy * sH * dv[r]);
-                        vb += fabs(R) * (gxb * sW * fabs(du[r]) + gyb * sH * fabs(dv[r]));
+                        vb += fabs(R) * (gxb * sW * adu[r] + gyb * sH * adv[r]);
                     }
                     dO[k * 3 + d] += w * val;
                     dOb[k * 3 + d] += fabs(w) * vb;

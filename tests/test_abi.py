@@ -135,3 +135,69 @@ def test_valid_host_checks_then_cuda_error_without_device(L):
     # every host-side check passes; the first CUDA call reports that no device is usable
     assert _fwd(L) == -4
     assert _bwd(L) == -4
+
+
+# --------------------------------------------------------------------------
+# deformable aggregation
+# --------------------------------------------------------------------------
+
+def test_header_declares_the_deformable_calls():
+    names = declared_functions()
+    for n in ["bev_deform_workspace_size", "bev_deform_forward", "bev_deform_backward"]:
+        assert n in names
+
+
+def test_deform_workspace_sizes(L):
+    # fp32 NCHW: repack (B N Hf Wf C 4) for the forward; + gradient buffer for the backward
+    fwd = L.bev_deform_workspace_size(0, 0, 1, 6, 256, 64, 176, 0)
+    assert fwd == 6 * 64 * 176 * 256 * 4
+    bwd = L.bev_deform_workspace_size(0, 0, 1, 6, 256, 64, 176, 1)
+    assert bwd == fwd + 6 * 64 * 176 * 256 * 4
+    # NHWC with whole chunks is used in place: no repack
+    assert L.bev_deform_workspace_size(0, 1, 1, 6, 256, 64, 176, 0) == 0
+    # bf16: chunks of 8 channels, fp32 gradient buffer padded to them
+    assert L.bev_deform_workspace_size(1, 1, 2, 6, 12, 8, 22, 1) == ((2 * 6 * 8 * 22 * 16 * 2 + 255) // 256 * 256
+                                                                      + (2 * 6 * 8 * 22 * 16 * 4 + 255) // 256 * 256)
+    assert L.bev_deform_workspace_size(0, 0, 0, 6, 16, 8, 22, 0) == ctypes.c_size_t(-1).value
+    assert L.bev_deform_workspace_size(3, 0, 1, 6, 16, 8, 22, 0) == ctypes.c_size_t(-1).value
+
+
+def _dfwd(L, **kw):
+    a = dict(features=FAKE, dtype=0, layout=0, B=1, N=6, C=256, Hf=64, Wf=176, K=FAKE, E=FAKE, img_h=512,
+             img_w=1408, A=FAKE, D=FAKE, W=FAKE, Q=900, Kp=13, out=FAKE, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.bev_deform_forward(a["features"], a["dtype"], a["layout"], a["B"], a["N"], a["C"], a["Hf"], a["Wf"],
+                                a["K"], a["E"], a["img_h"], a["img_w"], a["A"], a["D"], a["W"], a["Q"], a["Kp"],
+                                a["out"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def _dbwd(L, **kw):
+    a = dict(features=FAKE, dtype=0, layout=0, B=1, N=6, C=256, Hf=64, Wf=176, K=FAKE, E=FAKE, img_h=512,
+             img_w=1408, A=FAKE, D=FAKE, W=FAKE, Q=900, Kp=13, dout=FAKE, dF=FAKE, dW=FAKE, dO=FAKE,
+             ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.bev_deform_backward(a["features"], a["dtype"], a["layout"], a["B"], a["N"], a["C"], a["Hf"],
+                                 a["Wf"], a["K"], a["E"], a["img_h"], a["img_w"], a["A"], a["D"], a["W"], a["Q"],
+                                 a["Kp"], a["dout"], a["dF"], a["dW"], a["dO"], a["ws"], a["ws_bytes"],
+                                 a["stream"])
+
+
+def test_deform_argument_errors(L):
+    common = [(dict(features=None), -1), (dict(K=None), -1), (dict(A=None), -1), (dict(D=None), -1),
+              (dict(W=None), -1), (dict(Q=0), -1), (dict(Kp=0), -1), (dict(Kp=65), -1), (dict(N=33), -1),
+              (dict(img_h=0), -1), (dict(dtype=2), -2), (dict(layout=7), -2),
+              (dict(C=513), -2),                                  # beyond 4 chunks per lane (fp32)
+              (dict(ws=None), -3), (dict(ws_bytes=64), -3), (dict(ws=FAKE + 8), -3)]
+    for kw, want in common + [(dict(out=None), -1)]:
+        assert _dfwd(L, **kw) == want, kw
+    for kw, want in common + [(dict(dout=None), -1), (dict(dF=None), -1), (dict(dW=None), -1),
+                              (dict(dO=None), -1)]:
+        assert _dbwd(L, **kw) == want, kw
+    # bf16 takes up to 1024 channels
+    assert _dfwd(L, dtype=1, C=1024) != -2 and _dfwd(L, dtype=1, C=1032) == -2
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_deform_valid_host_checks_then_cuda_error_without_device(L):
+    assert _dfwd(L) == -4
+    assert _dbwd(L) == -4
