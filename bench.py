@@ -21,6 +21,11 @@ used on the data path ("scaling": "weak").
 --impl reference times the CPU oracle (oracle/, plain C loop nest in fp64) on
 the host cores, on a band of BEV rows per step, and prints the same JSON line
 with "impl": "reference".
+
+--op deform measures the deformable aggregation instead (SparseDriveV2 notes,
+"Deformable Aggregation"): one step = forward + backward (feature, weight and
+keypoint-offset gradients) over the queries of the ``deform`` workload (900
+queries x 13 keypoints, 6 cameras, C256, 64x176 maps), timed the same way.
 """
 from __future__ import annotations
 
@@ -53,7 +58,11 @@ def parse_args():
     ap.add_argument("--workload", default="nuscenes")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    return ap.parse_args()
+    ap.add_argument("--op", choices=["vt", "deform"], default="vt")
+    args = ap.parse_args()
+    if args.op == "deform" and args.workload == "nuscenes":
+        args.workload = "deform"
+    return args
 
 
 def dist_env():
@@ -79,6 +88,8 @@ def hbm_peak():
 KERNEL_SOURCES = {
     "sample_forward_kernel": ["bev_forward.cu", "bev_warp.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
     "sample_backward_kernel": ["bev_backward.cu", "bev_warp.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
+    "deform_forward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
+    "deform_backward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
 }
 
 
@@ -322,6 +333,37 @@ def run_ours(args):
         per = {name: [ev[k][s].elapsed_time(ev[k][s + 1]) for k in range(args.steps)]
                for s, name in enumerate(names)}
     stage_ms = {name: sum(v) / len(v) for name, v in per.items()}
+
+    # forward with a hot L2 (no flush), and as one CUDA graph of 100
+    # back-to-back launches (launch overhead amortised), per launch
+    with torch.cuda.stream(stream):
+        hot = []
+        for k in range(60):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graphs["forward"].replay()
+            e1.record(stream)
+            e1.synchronize()
+            if k >= 10:
+                hot.append(e0.elapsed_time(e1))
+        g100 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g100, stream=stream):
+            for _ in range(100):
+                stages["forward"]()
+        g100.replay()
+        reps = []
+        for k in range(8):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g100.replay()
+            e1.record(stream)
+            e1.synchronize()
+            if k >= 2:
+                reps.append(e0.elapsed_time(e1) / 100)
+        g100.reset()
+    fwd_hot_ms = statistics.median(hot)
+    fwd_b2b_ms = statistics.median(reps)
     ms = max_over_ranks(sum(stage_ms.values()), world, dev)
     elems = B * C * X * Y
     value = whole_job_rate(elems, world, ms)
@@ -382,7 +424,11 @@ def run_ours(args):
                    "timing": "CUDA events around CUDA-graph replays of each stage, launching stream"},
         "stages_ms": stage_ms,
         "forward_only": {"elements_per_s": elems / (stage_ms["forward"] * 1e-3), "GB_per_s": fwd_gbs,
-                         "frac_of_hbm_peak": fwd_gbs / peak},
+                         "frac_of_hbm_peak": fwd_gbs / peak,
+                         "hot_l2_us": 1e3 * fwd_hot_ms,
+                         "graph_of_100_us_per_launch": 1e3 * fwd_b2b_ms,
+                         "note": "L2 flushed before each timed step; hot_l2_us: no flush; graph_of_100: 100 "
+                                 "back-to-back launches in one CUDA graph after one flush, per launch"},
         "roofline": roofline,
         "e2e": {"value": whole_job_rate(elems, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -402,9 +448,164 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+DEFORM_METRIC = "deformable aggregation output elements/s (B·Q·C) and achieved HBM GB/s vs roofline, 1×B200"
+
+
+def deform_oracle_step(w, threads):
+    """One oracle forward + backward of the deformable aggregation over all
+    queries of the workload (same seeded inputs); returns seconds."""
+    import oracle
+    from camera_bev_view_b200 import inputs as I
+    F = I.make_features(w)
+    K, E = I.make_rigs(w)
+    A, D, W = I.make_queries(w)
+    g = I.make_query_dout(w)
+    t0 = time.perf_counter()
+    oracle.deform_forward(F, K, E, w.img_h, w.img_w, A, D, W, threads=threads)
+    oracle.deform_backward(F, g, K, E, w.img_h, w.img_w, A, D, W, threads=threads)
+    return time.perf_counter() - t0
+
+
+def deform_cpu_baseline(w, seconds):
+    """The oracle as it stands on the host cores, whole steps until `seconds`."""
+    threads = cpu_cores()
+    spent, steps = 0.0, 0
+    while steps == 0 or spent < seconds:
+        spent += deform_oracle_step(w, threads)
+        steps += 1
+    return {"value": w.out_elems * steps / spent, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{steps} whole forward+backward step(s) of the {w.name} workload ({spent:.1f} s, "
+                      f"OpenMP over queries / (batch, camera))"}
+
+
+def run_deform(args):
+    import torch
+
+    from camera_bev_view_b200 import inputs as I
+    from camera_bev_view_b200 import ops
+
+    rank, world, local = dist_env()
+    w = I.DEFORM_WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        threads = cpu_cores()
+        for _ in range(args.warmup):
+            deform_oracle_step(w, threads)
+        times = [deform_oracle_step(w, threads) for _ in range(args.steps)]
+        value = w.out_elems * len(times) / sum(times)
+        line = {"impl": "reference", "metric": DEFORM_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded queries, N(0,1) features, 6-camera rig)",
+                "config": {"workload": w.name},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                 "sample": "all queries, forward + backward, per step"},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    F_h = I.make_features(w, shard=rank)
+    K_h, E_h = I.make_rigs(w, shard=rank)
+    A_h, D_h, W_h = I.make_queries(w, shard=rank)
+    g_h = I.make_query_dout(w, shard=rank)
+    F, K, E, A, D, W, g = (t.to(dev) for t in (F_h, K_h, E_h, A_h, D_h, W_h, g_h))
+    B, N, C, Hf, Wf = F.shape
+    Fcl = F.permute(0, 1, 3, 4, 2).contiguous()
+    esize = F.element_size()
+    dt = ops.BF16 if esize == 2 else ops.F32
+    out = torch.empty((B, w.Q, C), device=dev)
+    grads = (torch.empty((B, N, C, Hf, Wf), device=dev), torch.empty((B, w.Q, N, w.Kp), device=dev),
+             torch.empty((B, w.Q, w.Kp, 3), device=dev))
+    ws = torch.empty(max(256, ops.bev_deform_workspace_size(dt, ops.NHWC, B, N, C, Hf, Wf, 1)),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stages = {
+        "forward": lambda: ops.bev_deform_forward(Fcl, K, E, w.img_h, w.img_w, A, D, W, layout=ops.NHWC, out=out,
+                                                  workspace=ws),
+        "backward": lambda: ops.bev_deform_backward(Fcl, K, E, w.img_h, w.img_w, A, D, W, g, layout=ops.NHWC,
+                                                    out=grads, workspace=ws),
+    }
+    # texels some valid keypoint samples: the support of the feature gradient
+    # for dout = 1 (weights are >= 0, so nothing cancels); measured once,
+    # outside the timed region, to count the feature bytes a launch must read
+    ones = torch.ones_like(g)
+    dF1, _, _ = ops.bev_deform_backward(Fcl, K, E, w.img_h, w.img_w, A, D, W, ones, layout=ops.NHWC)
+    touched = int(torch.count_nonzero(dF1[:, :, 0]).item())
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for f in stages.values():
+            f()
+        stream.synchronize()
+        for name, f in stages.items():
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                f()
+            graphs[name] = gr
+        for _ in range(args.warmup):
+            flush.zero_()
+            for gr in graphs.values():
+                gr.replay()
+        stream.synchronize()
+        names = list(stages)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local) as clocks:
+            for k in range(args.steps):
+                flush.zero_()
+                ev[k][0].record(stream)
+                for si, name in enumerate(names):
+                    graphs[name].replay()
+                    ev[k][si + 1].record(stream)
+            torch.cuda.synchronize(dev)
+        per = {name: [ev[k][si].elapsed_time(ev[k][si + 1]) for k in range(args.steps)]
+               for si, name in enumerate(names)}
+    for gr in graphs.values():
+        gr.reset()
+    stage_ms = {name: sum(v) / len(v) for name, v in per.items()}
+    ms = sum(stage_ms.values())
+    elems = w.out_elems
+    peak, peak_src = hbm_peak()
+    q_in = B * w.Q * (3 + w.Kp * 3 + N * w.Kp) * 4
+    fwd_bytes = touched * C * esize + q_in + elems * 4
+    bwd_bytes = touched * C * esize + q_in + elems * 4 + B * N * C * Hf * Wf * 4 + B * w.Q * w.Kp * (N + 3) * 4
+    dom = "forward" if stage_ms["forward"] >= stage_ms["backward"] else "backward"
+    dom_bytes = fwd_bytes if dom == "forward" else bwd_bytes
+    kname = "deform_forward_kernel" if dom == "forward" else "deform_backward_kernel"
+    achieved = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
+    line = {
+        "metric": DEFORM_METRIC, "value": elems / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if esize == 4 else "bf16",
+        "data": "synthetic (seeded queries, N(0,1) features, 6-camera rig)",
+        "config": {"workload": f"{w.name}: B{B} N{N} C{C} {Hf}x{Wf} (img {w.img_h}x{w.img_w}) Q{w.Q} K{w.Kp}",
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "timing": "CUDA events around CUDA-graph replays of each stage, launching stream"},
+        "stages_ms": stage_ms,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(kname, w.name), "kernel": kname, "stage": dom,
+                     "algorithmic_bytes_per_launch": dom_bytes, "touched_texels": touched,
+                     "note": "texels some valid keypoint samples, read once, + query inputs + outputs "
+                             "(backward: + dF written and dweights/doffsets)",
+                     "peak_source": peak_src},
+        "gpu_launches": args.steps * 4,
+        "clocks": clocks.summary(),
+    }
+    if args.cpu_seconds > 0:
+        line["cpu_baseline"] = deform_cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    if args.op == "deform":
+        run_deform(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -448,7 +448,6 @@ BEV_API int bev_deform_forward(const void* features, int dtype, int layout, int 
                             offsets, weights, Q, Kp, workspace, workspace_bytes, 0, extra, 1, s, &a, &V, &dev);
     if (st != BEV_OK) return st;
     a.out = out;
-    a.vec_out = (C % a.chan_per_chunk == 0) && ((uintptr_t)out % 16 == 0);
     return cuda_status(bev_launch_deform_forward(a, dtype == BEV_BF16, V, s));
 }
 

@@ -8,12 +8,15 @@
 // The geometry is the pinned fp32 projection of the dense path
 // (bev_geometry.cuh), so validity and corners match the oracle bit for bit.
 //
-// One warp per query.  Its lanes first take one (camera, keypoint) pair each
-// -- keypoint, projection, weight -- 32 pairs per pass; the valid pairs of a
-// pass are then visited in turn, each broadcast to the warp, whose lanes
-// read the four bilinear corners of their channel chunks (16-byte loads from
-// the channels-last features, V chunks per lane) and accumulate in fp32.
-// Up to two pairs are in flight per step.
+// One CTA per query; its kDeformWarps warps split the query's (camera,
+// keypoint) pairs, warp w taking every kDeformWarps-th pair from w.  A warp's
+// lanes first take one pair each -- keypoint, projection, weight -- 32 pairs
+// per pass; the valid pairs of a pass are then visited in turn, each
+// broadcast to the warp, whose lanes read the four bilinear corners of their
+// channel chunks (16-byte loads from the channels-last features, V chunks
+// per lane) and accumulate in fp32, up to two pairs in flight per step.  The
+// warps' partial sums meet in shared memory and are added in warp order, so
+// the result does not depend on timing.
 //
 // Backward, per valid pair: the lane-local dot products of the four corners
 // with dout are reduced over the warp into the weight gradient (the sample
@@ -21,8 +24,8 @@
 // carries the latter through the projection to the keypoint offset,
 //   d/dp = w R^T (g_x (Wf/W_img) du/dpc + g_y (Hf/H_img) dv/dpc),
 //   du/dpc = (K00, K01, K02 - u) / depth, dv/dpc likewise,
-// adding into a per-warp shared-memory accumulator in pair order
-// (deterministic).  The feature gradient is reduced into an fp32
+// adding into a per-warp shared-memory accumulator in pair order; the warps'
+// accumulators are added in warp order at the end (deterministic).  The feature gradient is reduced into an fp32
 // channels-last buffer with 16-byte vector reductions.
 #include "bev_deform.cuh"
 
@@ -126,12 +129,10 @@ __global__ void __launch_bounds__(kDeformWarps * 32) deform_forward_kernel(const
     constexpr int NF = DChunk<BF16>::kFloats;
     extern __shared__ __align__(16) float dsmem[];
     float* cams = dsmem;
-    const int b = blockIdx.y;
+    const int q = blockIdx.x, b = blockIdx.y;
     stage_cams(a, b, cams);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = blockIdx.x * kDeformWarps + warp;
-    if (q >= a.Q) return;
     const GeoParams& g = a.g;
     const float* A = a.anchors + ((size_t)b * a.Q + q) * 3;
     const float ax = A[0], ay = A[1], az = A[2];
@@ -151,8 +152,8 @@ __global__ void __launch_bounds__(kDeformWarps * 32) deform_forward_kernel(const
     // registers allow: 8 x 16-byte loads per lane in flight)
     constexpr int PP = V <= 2 ? 2 : 1;
     const int pairs = a.N * a.Kp;
-    for (int p0 = 0; p0 < pairs; p0 += 32) {
-        const Pair my = project_pair(a, cams, b, q, p0 + lane, ax, ay, az);
+    for (int p0 = warp; p0 < pairs; p0 += 32 * kDeformWarps) {
+        const Pair my = project_pair(a, cams, b, q, p0 + kDeformWarps * lane, ax, ay, az);
         unsigned m = __ballot_sync(0xffffffffu, my.ok);
         while (m) {
             int src[PP];
@@ -199,20 +200,25 @@ __global__ void __launch_bounds__(kDeformWarps * 32) deform_forward_kernel(const
         }
     }
 
-    float* o = a.out + ((size_t)b * a.Q + q) * a.C;
+    // the warps' partial sums, added in warp order
+    const int cpad = (a.C > a.Kp * 3 ? a.C : a.Kp * 3) + 3 & ~3;
+    float* part = dsmem + (a.N * kCamFloats + 3) / 4 * 4 + warp * cpad;
 #pragma unroll
     for (int v = 0; v < V; ++v) {
         const int c0 = (lane + 32 * v) * NF;
         if (!lane_ok[v]) continue;
-        if (a.vec_out) {
 #pragma unroll
-            for (int e = 0; e < NF; e += 4)
-                *reinterpret_cast<float4*>(o + c0 + e) = make_float4(acc[v][e], acc[v][e + 1], acc[v][e + 2], acc[v][e + 3]);
-        } else {
+        for (int e = 0; e < NF; ++e)
+            if (c0 + e < a.C) part[c0 + e] = acc[v][e];
+    }
+    __syncthreads();
+    const float* part0 = dsmem + (a.N * kCamFloats + 3) / 4 * 4;
+    float* o = a.out + ((size_t)b * a.Q + q) * a.C;
+    for (int c = threadIdx.x; c < a.C; c += kDeformWarps * 32) {
+        float s = part0[c];
 #pragma unroll
-            for (int e = 0; e < NF; ++e)
-                if (c0 + e < a.C) o[c0 + e] = acc[v][e];
-        }
+        for (int ww = 1; ww < kDeformWarps; ++ww) s = __fadd_rn(s, part0[ww * cpad + c]);
+        o[c] = s;
     }
 }
 
@@ -221,15 +227,14 @@ __global__ void __launch_bounds__(kDeformWarps * 32) deform_backward_kernel(cons
     constexpr int NF = DChunk<BF16>::kFloats;
     extern __shared__ __align__(16) float dsmem[];
     float* cams = dsmem;
-    const int b = blockIdx.y;
+    const int q = blockIdx.x, b = blockIdx.y;
     stage_cams(a, b, cams);
-    __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = blockIdx.x * kDeformWarps + warp;
-    if (q >= a.Q) return;
-    float* doff = dsmem + a.N * kCamFloats + warp * kDeformMaxKeypoints * 3;
+    const int cpad = (a.C > a.Kp * 3 ? a.C : a.Kp * 3) + 3 & ~3;
+    float* doff0 = dsmem + (a.N * kCamFloats + 3) / 4 * 4;
+    float* doff = doff0 + warp * cpad;
     for (int t = lane; t < a.Kp * 3; t += 32) doff[t] = 0.0f;
-    __syncwarp();
+    __syncthreads();
     const GeoParams& g = a.g;
     const float* A = a.anchors + ((size_t)b * a.Q + q) * 3;
     const float ax = A[0], ay = A[1], az = A[2];
@@ -252,9 +257,10 @@ __global__ void __launch_bounds__(kDeformWarps * 32) deform_backward_kernel(cons
     float* dW = a.dweights + ((size_t)b * a.Q + q) * a.N * a.Kp;
 
     const int pairs = a.N * a.Kp;
-    for (int p0 = 0; p0 < pairs; p0 += 32) {
-        const Pair my = project_pair(a, cams, b, q, p0 + lane, ax, ay, az);
-        if (p0 + lane < pairs && !my.ok) dW[p0 + lane] = 0.0f;  // no sample, no gradient
+    for (int p0 = warp; p0 < pairs; p0 += 32 * kDeformWarps) {
+        const int pr = p0 + kDeformWarps * lane;
+        const Pair my = project_pair(a, cams, b, q, pr, ax, ay, az);
+        if (pr < pairs && !my.ok) dW[pr] = 0.0f;  // no sample, no gradient
         unsigned m = __ballot_sync(0xffffffffu, my.ok);
         while (m) {
             const int src = __ffs(m) - 1;
@@ -271,18 +277,20 @@ __global__ void __launch_bounds__(kDeformWarps * 32) deform_backward_kernel(cons
             const uint4* Fn = featb + (size_t)n * texels * a.Qtot;
             float* Gn = gradb + (size_t)n * texels * tstride;
             // lane-local dot products of each corner with dout
+            uint4 dv[4][V];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int v = 0; v < V; ++v)
+                    dv[t][v] = (in[t] && lane_ok[v]) ? __ldg(Fn + (size_t)tex[t] * a.Qtot + 32 * v) : make_uint4(0, 0, 0, 0);
             float dot[4];
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-                uint4 dv[V];
-#pragma unroll
-                for (int v = 0; v < V; ++v)
-                    dv[v] = (in[t] && lane_ok[v]) ? __ldg(Fn + (size_t)tex[t] * a.Qtot + 32 * v) : make_uint4(0, 0, 0, 0);
                 float s = 0.0f;
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     float f[NF];
-                    DChunk<BF16>::unpack(dv[v], f);
+                    DChunk<BF16>::unpack(dv[t][v], f);
 #pragma unroll
                     for (int e = 0; e < NF; ++e) s = __fmaf_rn(f[e], dg[v][e], s);
                 }
@@ -313,35 +321,41 @@ __global__ void __launch_bounds__(kDeformWarps * 32) deform_backward_kernel(cons
             gx = warp_sum(gx);
             gy = warp_sum(gy);
             if (lane == src) {
-                dW[p0 + lane] = s;
+                dW[pr] = s;
                 const float* cam = cams + n * kCamFloats;
                 const float rd = 1.0f / my.det.depth;
                 const float du[3] = {cam[12] * rd, cam[13] * rd, (cam[14] - my.det.u) * rd};
-                const float dv[3] = {cam[15] * rd, cam[16] * rd, (cam[17] - my.det.v) * rd};
+                const float dv3[3] = {cam[15] * rd, cam[16] * rd, (cam[17] - my.det.v) * rd};
                 const float ax_ = gx * g.sW, ay_ = gy * g.sH;
 #pragma unroll
                 for (int dd = 0; dd < 3; ++dd) {
                     float val = 0.0f;
 #pragma unroll
-                    for (int r = 0; r < 3; ++r) val += cam[4 * r + dd] * (ax_ * du[r] + ay_ * dv[r]);
+                    for (int r = 0; r < 3; ++r) val += cam[4 * r + dd] * (ax_ * du[r] + ay_ * dv3[r]);
                     doff[my.k * 3 + dd] += w * val;
                 }
             }
             __syncwarp();
         }
     }
+    __syncthreads();
     float* dO = a.doffsets + ((size_t)b * a.Q + q) * a.Kp * 3;
-    for (int t = lane; t < a.Kp * 3; t += 32) dO[t] = doff[t];
+    for (int t = threadIdx.x; t < a.Kp * 3; t += kDeformWarps * 32) {
+        float s = doff0[t];
+#pragma unroll
+        for (int ww = 1; ww < kDeformWarps; ++ww) s = __fadd_rn(s, doff0[ww * cpad + t]);
+        dO[t] = s;
+    }
 }
 
 namespace {
 
 template <typename Kernel>
 cudaError_t launch(Kernel k, const DeformArgs& a, cudaStream_t st) {
-    const size_t smem = deform_smem_bytes(a.N);
+    const size_t smem = deform_smem_bytes(a.N, a.C, a.Kp);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid((a.Q + kDeformWarps - 1) / kDeformWarps, a.B);
+    const dim3 grid(a.Q, a.B);
     k<<<grid, kDeformWarps * 32, smem, st>>>(a);
     return cudaGetLastError();
 }

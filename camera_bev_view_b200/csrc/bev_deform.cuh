@@ -11,8 +11,8 @@ namespace bev {
 // Keypoints per query the kernels accept (per-warp shared-memory accumulator
 // of the offset gradient).
 constexpr int kDeformMaxKeypoints = 64;
-// Queries per CTA: one warp each.
-constexpr int kDeformWarps = 8;
+// One CTA per query; its warps split the query's (camera, keypoint) pairs.
+constexpr int kDeformWarps = 4;
 
 struct DeformArgs {
     const void* feat;       // channels-last [B*N][Hf*Wf][Qtot chunks of 16 bytes]
@@ -30,11 +30,14 @@ struct DeformArgs {
     int B, N, C, Q, Kp;
     int Qtot;               // 16-byte feature chunks per texel
     int chan_per_chunk;     // 4 (fp32) or 8 (bf16)
-    int vec_out;            // forward: C % chan_per_chunk == 0 and out 16-byte aligned
 };
 
-inline size_t deform_smem_bytes(int N) {
-    return sizeof(float) * ((size_t)N * kCamFloats + (size_t)kDeformWarps * kDeformMaxKeypoints * 3);
+// Shared memory of one CTA: calibrations, then per warp either the partial
+// sums of the forward (C floats) or the offset-gradient accumulator of the
+// backward (Kp x 3 floats).
+inline size_t deform_smem_bytes(int N, int C, int Kp) {
+    const size_t per_warp = (size_t)((C > Kp * 3 ? C : Kp * 3) + 3) & ~(size_t)3;
+    return sizeof(float) * (((size_t)N * kCamFloats + 3) / 4 * 4 + (size_t)kDeformWarps * per_warp);
 }
 
 }  // namespace bev

@@ -6,6 +6,10 @@
 //   NCHW case is a 32x32 shared-memory tiled transpose (coalesced on both
 //   sides); the unaligned-NHWC case is a straight strided copy.
 // to_nchw: the fp32 channels-last gradient buffer [BN][HW][Cp] -> [BN][C][HW].
+//   When HW is a multiple of 4 and the output is 16-byte aligned, each thread
+//   moves a 4 texel x 4 channel block with 16-byte loads and 16-byte stores
+//   (a register transpose; whole 32-byte sectors on both sides); otherwise a
+//   32x32 shared-memory tiled transpose.
 #include <stdint.h>
 
 #include "bev_kernels.cuh"
@@ -63,6 +67,31 @@ __global__ void __launch_bounds__(256) nhwc_to_nchw_kernel(const float* __restri
     }
 }
 
+// 4x4 register-blocked transpose: block (16 x 16 threads) covers 64 texels x
+// 64 channels; thread (tx, ty) reads texels 4 ty .. 4 ty + 3 at channels
+// 4 tx .. 4 tx + 3 and writes them back as four channel rows.  HW % 4 == 0,
+// Cp % 4 == 0, dst 16-byte aligned.
+__global__ void __launch_bounds__(256) nhwc_to_nchw_v4_kernel(const float* __restrict__ src, int C, int HW,
+                                                              int Cp, float* __restrict__ dst) {
+    const size_t bn = blockIdx.z;
+    const int p = blockIdx.x * 64 + 4 * threadIdx.y;
+    const int c = blockIdx.y * 64 + 4 * threadIdx.x;
+    if (p >= HW || c >= C) return;
+    const float* s = src + (bn * HW + p) * (size_t)Cp + c;
+    float4 r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) r[j] = __ldg(reinterpret_cast<const float4*>(s + (size_t)j * Cp));
+    float* d = dst + (bn * C + c) * (size_t)HW + p;
+    const float col[4][4] = {{r[0].x, r[1].x, r[2].x, r[3].x},
+                             {r[0].y, r[1].y, r[2].y, r[3].y},
+                             {r[0].z, r[1].z, r[2].z, r[3].z},
+                             {r[0].w, r[1].w, r[2].w, r[3].w}};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (c + i < C)
+            *reinterpret_cast<float4*>(d + (size_t)i * HW) = make_float4(col[i][0], col[i][1], col[i][2], col[i][3]);
+}
+
 }  // namespace bev
 
 cudaError_t bev_launch_to_channels_last(const void* src, int layout, int esize, int BN, int C, int HW,
@@ -92,6 +121,11 @@ cudaError_t bev_launch_to_channels_last(const void* src, int layout, int esize, 
 
 cudaError_t bev_launch_to_nchw(const float* src, int BN, int C, int HW, int Cp, float* dst,
                                cudaStream_t stream) {
+    if (HW % 4 == 0 && Cp % 4 == 0 && ((uintptr_t)src % 16) == 0 && ((uintptr_t)dst % 16) == 0) {
+        const dim3 grid((HW + 63) / 64, (C + 63) / 64, BN);
+        bev::nhwc_to_nchw_v4_kernel<<<grid, dim3(16, 16), 0, stream>>>(src, C, HW, Cp, dst);
+        return cudaGetLastError();
+    }
     const dim3 grid((HW + bev::kT - 1) / bev::kT, (C + bev::kT - 1) / bev::kT, BN);
     const dim3 block(bev::kT, 8);
     bev::nhwc_to_nchw_kernel<<<grid, block, 0, stream>>>(src, C, HW, Cp, dst);

@@ -207,8 +207,9 @@ size_t bev_deform_workspace_size(int dtype, int layout, int B, int N, int C, int
  *                (1..BEV_DEFORM_MAX_KEYPOINTS)
  *   out          [B,Q,C] fp32, fully overwritten
  *   workspace    at least bev_deform_workspace_size(dtype, layout, ..., 0) bytes
- * Every output is computed by one warp in a fixed order, so results are
- * reproducible bit for bit.  Returns BEV_OK, BEV_ERR_INVALID_ARG,
+ * Each query is one CTA whose warps split its (camera, keypoint) pairs and
+ * add their partial sums in a fixed order, so results are reproducible bit
+ * for bit.  Returns BEV_OK, BEV_ERR_INVALID_ARG,
  * BEV_ERR_UNSUPPORTED, BEV_ERR_WORKSPACE or BEV_ERR_CUDA. */
 int bev_deform_forward(const void* features, int dtype, int layout, int B, int N, int C, int Hf, int Wf,
                        const float* intrinsics, const float* ego2cam, int img_h, int img_w,
