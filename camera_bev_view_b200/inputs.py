@@ -23,6 +23,18 @@ the tens, over six surround cameras):
   deform       B1 N6 C256 64x176 (img 512x1408) Q900 K13  fp32
   deform_bf16  B4 N6 C256 64x176 (img 512x1408) Q900 K13  bf16
 
+Lift-splat pooling workloads (LSS tutorial, "Lift" and "Splat": 41 depth
+bins over [4, 45) m at 1 m, 64-d context, 8x22 features per camera from
+128x352 images, 6 cameras, a 200x200 BEV at 0.5 m; z is one pillar, taken
+as [-10, 10] m):
+
+  lss_tiny  B1 N6 C8  D8  8x22  (img 128x352)  40x40 over +-20 m   fp32
+  lss       B1 N6 C64 D41 8x22  (img 128x352)  200x200 over +-50 m fp32
+  lss_b4    B4 N6 C64 D41 16x44 (img 256x704)  200x200 over +-50 m fp32
+
+Depth distributions are a softmax over the bins of N(0, 1) * 2 logits;
+context features and the upstream gradient are N(0, 1).
+
 Anchors are uniform over x, y in [-50, 50] m and z in [-2, 2] m; keypoint
 offsets uniform in [-2, 2] m per axis; weights uniform in [0, 1) / (N K);
 the upstream gradient is N(0, 1).
@@ -125,6 +137,68 @@ DEFORM_WORKLOADS = {
     "deform": DeformWorkload("deform", 11, 1, 6, 256, 64, 176, 512, 1408, 900, 13, "f32"),
     "deform_bf16": DeformWorkload("deform_bf16", 12, 4, 6, 256, 64, 176, 512, 1408, 900, 13, "bf16"),
 }
+
+
+@dataclasses.dataclass(frozen=True)
+class LssWorkload:
+    name: str
+    index: int            # seed family
+    B: int
+    N: int
+    C: int
+    D: int                # depth bins
+    Hf: int
+    Wf: int
+    img_h: int
+    img_w: int
+    X: int
+    Y: int
+    xr: tuple
+    yr: tuple
+    zr: tuple
+    dbound: tuple         # (dmin, dmax, dstep)
+    dtype: str = "f32"
+
+    @property
+    def ranges(self):
+        return (self.xr[0], self.xr[1], self.yr[0], self.yr[1], self.zr[0], self.zr[1])
+
+    @property
+    def res_xy(self):
+        return ((self.xr[1] - self.xr[0]) / self.X, (self.yr[1] - self.yr[0]) / self.Y)
+
+    @property
+    def out_elems(self):
+        return self.B * self.C * self.X * self.Y
+
+    def scaled(self, **kw):
+        return dataclasses.replace(self, **kw)
+
+
+LSS_WORKLOADS = {
+    "lss_tiny": LssWorkload("lss_tiny", 20, 1, 6, 8, 8, 8, 22, 128, 352, 40, 40, (-20.0, 20.0), (-20.0, 20.0),
+                            (-10.0, 10.0), (4.0, 12.0, 1.0)),
+    "lss": LssWorkload("lss", 21, 1, 6, 64, 41, 8, 22, 128, 352, 200, 200, (-50.0, 50.0), (-50.0, 50.0),
+                       (-10.0, 10.0), (4.0, 45.0, 1.0)),
+    "lss_b4": LssWorkload("lss_b4", 22, 4, 6, 64, 41, 16, 44, 256, 704, 200, 200, (-50.0, 50.0), (-50.0, 50.0),
+                          (-10.0, 10.0), (4.0, 45.0, 1.0)),
+}
+
+
+def make_lss_inputs(w: LssWorkload, shard: int = 0):
+    """(depth [B,N,D,Hf,Wf], feat [B,N,C,Hf,Wf]) float32 torch (CPU): depth is a
+    softmax over the bins of N(0,1) * 2 logits; feat is N(0,1)."""
+    g = torch.Generator().manual_seed(7000 + w.index + 100003 * shard)
+    logits = 2.0 * torch.randn((w.B, w.N, w.D, w.Hf, w.Wf), generator=g, dtype=torch.float32)
+    depth = torch.softmax(logits, dim=2)
+    feat = torch.randn((w.B, w.N, w.C, w.Hf, w.Wf), generator=g, dtype=torch.float32)
+    return depth.contiguous(), feat
+
+
+def make_lss_dout(w: LssWorkload, shard: int = 0) -> torch.Tensor:
+    """Upstream gradient [B,C,X,Y] float32, i.i.d. N(0,1)."""
+    g = torch.Generator().manual_seed(8000 + w.index + 100003 * shard)
+    return torch.randn((w.B, w.C, w.X, w.Y), generator=g, dtype=torch.float32)
 
 
 def make_queries(w: DeformWorkload, shard: int = 0):

@@ -9,7 +9,9 @@ loop nest (FlashBEV reading notes, "Method" items 1 and 4): per height bin the
 mean over valid cameras of the bilinear samples, summed over height.  See the
 header comment of ``bev_oracle.c`` for every reading it takes.
 
-Also the deformable aggregation of the SparseDriveV2 notes ("Deformable
+Also the lift-splat BEV pooling of the LSS tutorial ("Lift", "Splat"):
+``lss_forward`` / ``lss_backward`` (pins in ``tests/test_oracle_lss.py``), and
+the deformable aggregation of the SparseDriveV2 notes ("Deformable
 Aggregation", steps 1-3): ``deform_forward`` / ``deform_backward`` (pins in
 ``tests/test_oracle_deform.py``).
 
@@ -65,6 +67,13 @@ def _load():
         lib.oracle_deform_backward.argtypes = [P, P, I, I, I, I, I, P, P, I, I, P, P, P, I, I,
                                                P, P, P, P, P, P, I]
         lib.oracle_deform_backward.restype = None
+        lib.oracle_lss_cell.argtypes = [P, P, I, I, I, I, I, I, I, F, F, I, I, P, F, P, P]
+        lib.oracle_lss_cell.restype = I
+        lib.oracle_lss_forward.argtypes = [P, P, I, I, I, I, I, I, P, P, I, I, F, F, I, I, P, F, P, P, P, P]
+        lib.oracle_lss_forward.restype = None
+        lib.oracle_lss_backward.argtypes = [P, P, P, I, I, I, I, I, I, P, P, I, I, F, F, I, I, P, F, P,
+                                            P, P, P, P]
+        lib.oracle_lss_backward.restype = None
         _lib = lib
     return _lib
 
@@ -196,4 +205,66 @@ def deform_backward(features, dout, K, E, img_h, img_w, anchors, offsets, weight
                                    _ptr(A), _ptr(D), _ptr(W), Q, Kp,
                                    _ptr(r["dF"]), _ptr(r["dF_bound"]), _ptr(r["dW"]), _ptr(r["dW_bound"]),
                                    _ptr(r["dOff"]), _ptr(r["dOff_bound"]), threads)
+    return r
+
+
+class LssGrid:
+    """BEV pillars of the lift-splat pooling: counts X, Y from x/y ranges and
+    cell sizes (oracle's own), one z slab [zmin, zmax), depth bins."""
+
+    def __init__(self, ranges, res_xy, dbound):
+        g = Grid((ranges[0], ranges[1], ranges[2], ranges[3], ranges[4], ranges[5]),
+                 (res_xy[0], res_xy[1], ranges[5] - ranges[4]))
+        self.X, self.Y = g.X, g.Y
+        self.lo = g.lo
+        self.zmax = np.float32(ranges[5])
+        self.cell = np.ascontiguousarray(g.cell[:2])
+        self.dmin, self.dmax, self.dstep = (np.float32(v) for v in dbound)
+        self.D = int(round((float(dbound[1]) - float(dbound[0])) / float(dbound[2])))
+
+
+def lss_cell(K, E, h, w, k, img_h, img_w, Hf, Wf, grid: LssGrid):
+    """(cell index i*Y + j or -1, ego point) of one frustum point."""
+    K = _np(K, np.float32).reshape(9)
+    E = _np(E, np.float32).reshape(16)
+    p = np.zeros(3, dtype=np.float32)
+    c = _load().oracle_lss_cell(_ptr(K), _ptr(E), h, w, k, img_h, img_w, Hf, Wf, float(grid.dmin), float(grid.dstep),
+                                grid.X, grid.Y, _ptr(grid.lo), float(grid.zmax), _ptr(grid.cell), _ptr(p))
+    return int(c), p
+
+
+def lss_forward(depth, feat, K, E, img_h, img_w, grid: LssGrid):
+    """Lift-splat pooling.  depth [B,N,D,Hf,Wf], feat [B,N,C,Hf,Wf].  Returns
+    (out [B,C,X,Y] f64, bound [B,C,X,Y] f64, count [B,X,Y] int32)."""
+    A = _np(depth, np.float64)
+    Fe = _np(feat, np.float64)
+    B, N, D, Hf, Wf = A.shape
+    C = Fe.shape[2]
+    assert Fe.shape == (B, N, C, Hf, Wf) and D == grid.D
+    Kc = _np(K, np.float32).reshape(B, N, 3, 3)
+    Ec = _np(E, np.float32).reshape(B, N, 4, 4)
+    out = np.zeros((B, C, grid.X, grid.Y), dtype=np.float64)
+    bound = np.zeros_like(out)
+    count = np.zeros((B, grid.X, grid.Y), dtype=np.int32)
+    _load().oracle_lss_forward(_ptr(A), _ptr(Fe), B, N, D, C, Hf, Wf, _ptr(Kc), _ptr(Ec), img_h, img_w,
+                               float(grid.dmin), float(grid.dstep), grid.X, grid.Y, _ptr(grid.lo), float(grid.zmax),
+                               _ptr(grid.cell), _ptr(out), _ptr(bound), _ptr(count))
+    return out, bound, count
+
+
+def lss_backward(depth, feat, dout, K, E, img_h, img_w, grid: LssGrid):
+    """Returns dict ddepth, ddepth_bound [B,N,D,Hf,Wf], dfeat, dfeat_bound [B,N,C,Hf,Wf] (f64)."""
+    A = _np(depth, np.float64)
+    Fe = _np(feat, np.float64)
+    G = _np(dout, np.float64)
+    B, N, D, Hf, Wf = A.shape
+    C = Fe.shape[2]
+    Kc = _np(K, np.float32).reshape(B, N, 3, 3)
+    Ec = _np(E, np.float32).reshape(B, N, 4, 4)
+    r = {k: np.zeros(s, dtype=np.float64) for k, s in
+         [("ddepth", A.shape), ("ddepth_bound", A.shape), ("dfeat", Fe.shape), ("dfeat_bound", Fe.shape)]}
+    _load().oracle_lss_backward(_ptr(A), _ptr(Fe), _ptr(G), B, N, D, C, Hf, Wf, _ptr(Kc), _ptr(Ec), img_h, img_w,
+                                float(grid.dmin), float(grid.dstep), grid.X, grid.Y, _ptr(grid.lo), float(grid.zmax),
+                                _ptr(grid.cell), _ptr(r["ddepth"]), _ptr(r["ddepth_bound"]), _ptr(r["dfeat"]),
+                                _ptr(r["dfeat_bound"]))
     return r

@@ -449,3 +449,126 @@ void oracle_deform_backward(const double* F, const double* dout, int B, int N, i
         }
     }
 }
+
+/* ------------------------------------------------------------------------
+ * Lift-splat BEV pooling (LSS tutorial, "Lift" and "Splat" sections): every
+ * feature pixel (h, w) of camera n spreads D depth bins along its ray; the
+ * point of bin k carries depth[b,n,k,h,w] * feat[b,n,:,h,w] (the outer
+ * product of the depth distribution and the context vector), is placed in
+ * the ego frame with the camera's calibration, and is summed into the BEV
+ * pillar (i, j) it falls in; z is not binned (one pillar per cell), and
+ * points outside [xmin,xmax) x [ymin,ymax) x [zmin,zmax) are dropped:
+ *
+ *   out[b, c, i, j] = sum over (n, k, h, w) with cell (i, j) of depth[b,n,k,h,w] feat[b,n,c,h,w]
+ *
+ * Readings: the pixel of feature texel (h, w) is its centre in image pixels,
+ * u = (w + 0.5) W_img / Wf, v = (h + 0.5) H_img / Hf (the inverse of the
+ * sampling convention above); bin k sits at depth dmin + k * dstep (the bin's
+ * lower edge, as the tutorial lists depths 4, 5, ..., 44 for [4, 45) at 1 m);
+ * the camera point is depth * K^-1 [u v 1]^T with K upper triangular; E maps
+ * ego to camera with a rotation R, so ego = R^T (pc - t).  The fp32 order:
+ *   yn = (v - cy) / fy;  xn = ((u - cx) - s * yn) / fx;  pc = (xn d, yn d, d)
+ *   q = pc - t;  x = (R00 q0 + R10 q1) + R20 q2  (likewise y, z)
+ *   i = floor((x - xmin) / dx), j = floor((y - ymin) / dy)
+ * ---------------------------------------------------------------------- */
+
+/* Cell of one frustum point, or -1 when it falls outside the grid. */
+int oracle_lss_cell(const float* K, const float* E, int h, int w, int k, int img_h, int img_w, int Hf, int Wf,
+                    float dmin, float dstep, int X, int Y, const float lo[3], float zmax, const float cell[2],
+                    float p_out[3])
+{
+    float sWi = (float)img_w / (float)Wf, sHi = (float)img_h / (float)Hf;
+    float u = ((float)w + 0.5f) * sWi;
+    float v = ((float)h + 0.5f) * sHi;
+    float d = (float)k * dstep;
+    d = dmin + d;
+    float yn = (v - K[5]) / K[4];
+    float t = K[1] * yn;
+    float xn = ((u - K[2]) - t) / K[0];
+    float pc[3] = {xn * d, yn * d, d};
+    float q[3];
+    for (int r = 0; r < 3; ++r) q[r] = pc[r] - E[4 * r + 3];
+    float p[3];
+    for (int a = 0; a < 3; ++a) {
+        float s0 = E[a] * q[0];
+        float s1 = E[4 + a] * q[1];
+        float s2 = E[8 + a] * q[2];
+        float acc = s0 + s1;
+        p[a] = acc + s2;
+    }
+    if (p_out) { p_out[0] = p[0]; p_out[1] = p[1]; p_out[2] = p[2]; }
+    if (!(p[2] >= lo[2] && p[2] < zmax)) return -1;
+    float fi = floorf((p[0] - lo[0]) / cell[0]);
+    float fj = floorf((p[1] - lo[1]) / cell[1]);
+    if (!(fi >= 0.0f && fi < (float)X && fj >= 0.0f && fj < (float)Y)) return -1;
+    return (int)fi * Y + (int)fj;
+}
+
+/* Forward.  depth [B,N,D,Hf,Wf], feat [B,N,C,Hf,Wf] fp64 (exact copies of the
+ * inputs); K [B,N,3,3], E [B,N,4,4]; grid lo = (xmin, ymin, zmin), zmax,
+ * cell = (dx, dy).  Writes out and bound [B,C,X,Y] fp64 and count [B,X,Y]
+ * (points per pillar). */
+void oracle_lss_forward(const double* depth, const double* feat, int B, int N, int D, int C, int Hf, int Wf,
+                        const float* K, const float* E, int img_h, int img_w, float dmin, float dstep,
+                        int X, int Y, const float lo[3], float zmax, const float cell[2],
+                        double* out, double* bound, int32_t* count)
+{
+    memset(out, 0, sizeof(double) * (size_t)B * C * X * Y);
+    memset(bound, 0, sizeof(double) * (size_t)B * C * X * Y);
+    memset(count, 0, sizeof(int32_t) * (size_t)B * X * Y);
+    for (int b = 0; b < B; ++b)
+        for (int n = 0; n < N; ++n) {
+            const float* Kn = K + ((size_t)b * N + n) * 9;
+            const float* En = E + ((size_t)b * N + n) * 16;
+            for (int h = 0; h < Hf; ++h)
+                for (int w = 0; w < Wf; ++w)
+                    for (int k = 0; k < D; ++k) {
+                        int cl = oracle_lss_cell(Kn, En, h, w, k, img_h, img_w, Hf, Wf, dmin, dstep, X, Y, lo, zmax,
+                                                 cell, NULL);
+                        if (cl < 0) continue;
+                        ++count[(size_t)b * X * Y + cl];
+                        double a = depth[((((size_t)b * N + n) * D + k) * Hf + h) * Wf + w];
+                        for (int c = 0; c < C; ++c) {
+                            double term = a * feat[((((size_t)b * N + n) * C + c) * Hf + h) * Wf + w];
+                            size_t o = ((size_t)b * C + c) * X * Y + cl;
+                            out[o] += term;
+                            bound[o] += fabs(term);
+                        }
+                    }
+        }
+}
+
+/* Backward for dout [B,C,X,Y] fp64: ddepth [B,N,D,Hf,Wf] = sum_c dout[cell] feat,
+ * dfeat [B,N,C,Hf,Wf] = sum_k depth dout[cell_k]; bounds of the same shapes. */
+void oracle_lss_backward(const double* depth, const double* feat, const double* dout, int B, int N, int D, int C,
+                         int Hf, int Wf, const float* K, const float* E, int img_h, int img_w, float dmin,
+                         float dstep, int X, int Y, const float lo[3], float zmax, const float cell[2],
+                         double* ddepth, double* ddb, double* dfeat, double* dfb)
+{
+    memset(ddepth, 0, sizeof(double) * (size_t)B * N * D * Hf * Wf);
+    memset(ddb, 0, sizeof(double) * (size_t)B * N * D * Hf * Wf);
+    memset(dfeat, 0, sizeof(double) * (size_t)B * N * C * Hf * Wf);
+    memset(dfb, 0, sizeof(double) * (size_t)B * N * C * Hf * Wf);
+    for (int b = 0; b < B; ++b)
+        for (int n = 0; n < N; ++n) {
+            const float* Kn = K + ((size_t)b * N + n) * 9;
+            const float* En = E + ((size_t)b * N + n) * 16;
+            for (int h = 0; h < Hf; ++h)
+                for (int w = 0; w < Wf; ++w)
+                    for (int k = 0; k < D; ++k) {
+                        int cl = oracle_lss_cell(Kn, En, h, w, k, img_h, img_w, Hf, Wf, dmin, dstep, X, Y, lo, zmax,
+                                                 cell, NULL);
+                        if (cl < 0) continue;
+                        size_t di = ((((size_t)b * N + n) * D + k) * Hf + h) * Wf + w;
+                        double a = depth[di];
+                        for (int c = 0; c < C; ++c) {
+                            size_t fi = ((((size_t)b * N + n) * C + c) * Hf + h) * Wf + w;
+                            double g = dout[((size_t)b * C + c) * X * Y + cl];
+                            ddepth[di] += g * feat[fi];
+                            ddb[di] += fabs(g * feat[fi]);
+                            dfeat[fi] += a * g;
+                            dfb[fi] += fabs(a * g);
+                        }
+                    }
+        }
+}

@@ -140,3 +140,61 @@ def tensorized_deform(features, K, E, img_h, img_w, anchors, offsets, weights, o
     fx = u * (Wf / img_w) - 0.5
     fy = v * (Hf / img_h) - 0.5
     return out, mask, amb, fx, fy
+
+
+# --------------------------------------------------------------------------
+# Lift-splat BEV pooling (LSS tutorial, "Lift" and "Splat"), materialised:
+# every frustum point (b, n, k, h, w) in float64 -- pixel centre, depth of
+# bin k, K^-1 by torch.linalg.inv, E^-1 by torch.linalg.inv -- its pillar by
+# floor, the outer product depth x feat as an explicit [.., D, C] tensor, and
+# a float64 index_add into the BEV grid.
+# --------------------------------------------------------------------------
+
+def lss_points(K, E, Hf, Wf, img_h, img_w, dbound):
+    """Ego points [B,N,D,Hf,Wf,3] of every frustum point, float64."""
+    K = torch.as_tensor(K, dtype=torch.float64)
+    E = torch.as_tensor(E, dtype=torch.float64)
+    dmin, dmax, dstep = (float(v) for v in dbound)
+    D = int(round((dmax - dmin) / dstep))
+    ds = dmin + dstep * torch.arange(D, dtype=torch.float64)
+    us = (torch.arange(Wf, dtype=torch.float64) + 0.5) * (img_w / Wf)
+    vs = (torch.arange(Hf, dtype=torch.float64) + 0.5) * (img_h / Hf)
+    v, u = torch.meshgrid(vs, us, indexing="ij")
+    pix = torch.stack([u, v, torch.ones_like(u)], dim=-1)                      # [Hf,Wf,3]
+    rays = torch.einsum("bnrk,hwk->bnhwr", torch.linalg.inv(K), pix)           # camera frame, depth 1
+    pc = ds[None, None, :, None, None, None] * rays[:, :, None]                # [B,N,D,Hf,Wf,3]
+    Einv = torch.linalg.inv(E)
+    return torch.einsum("bnrk,bndhwk->bndhwr", Einv[:, :, :3, :3], pc) + Einv[:, :, None, None, None, :3, 3]
+
+
+def tensorized_lss(depth, feat, K, E, img_h, img_w, ranges, counts_xy, dbound, margin=1e-4):
+    """Returns (out [B,C,X,Y], count [B,X,Y], ambiguous [B,N,D,Hf,Wf]) in float64;
+    ``ambiguous`` marks points within ``margin`` (relative to the cell) of a
+    cell edge or of the z slab's bounds."""
+    A = torch.as_tensor(depth)
+    A = A if A.dtype == torch.float64 else A.to(torch.float64)
+    Fe = torch.as_tensor(feat)
+    Fe = Fe if Fe.dtype == torch.float64 else Fe.to(torch.float64)
+    B, N, D, Hf, Wf = A.shape
+    C = Fe.shape[2]
+    X, Y = counts_xy
+    xmin, xmax, ymin, ymax, zmin, zmax = (float(r) for r in ranges)
+    dx, dy = (xmax - xmin) / X, (ymax - ymin) / Y
+    P = lss_points(K, E, Hf, Wf, img_h, img_w, dbound)
+    fi = (P[..., 0] - xmin) / dx
+    fj = (P[..., 1] - ymin) / dy
+    i, j = torch.floor(fi), torch.floor(fj)
+    inside = (i >= 0) & (i < X) & (j >= 0) & (j < Y) & (P[..., 2] >= zmin) & (P[..., 2] < zmax)
+    amb = (((fi - torch.round(fi)).abs() < margin) | ((fj - torch.round(fj)).abs() < margin) |
+           ((P[..., 2] - zmin).abs() < margin) | ((P[..., 2] - zmax).abs() < margin))
+    pts = A[:, :, :, None] * Fe[:, :, None]                                    # [B,N,D,C,Hf,Wf] outer product
+    cellid = torch.where(inside, (i * Y + j).long(), torch.zeros_like(i).long())
+    out = torch.zeros((B, C, X * Y), dtype=torch.float64)
+    count = torch.zeros((B, X * Y), dtype=torch.float64)
+    for b in range(B):
+        m = inside[b].reshape(-1)
+        idx = cellid[b].reshape(-1)[m]
+        vals = pts[b].permute(0, 1, 3, 4, 2).reshape(-1, C)[m]                 # [points, C]
+        out[b].index_add_(1, idx, vals.t())
+        count[b].index_add_(0, idx, torch.ones_like(idx, dtype=torch.float64))
+    return out.reshape(B, C, X, Y), count.reshape(B, X, Y), amb
