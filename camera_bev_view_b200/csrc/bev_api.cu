@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include "bev_deform.cuh"
+#include "bev_lss.cuh"
 #include "bev_kernels.cuh"
 #include "bevsample.h"
 
@@ -473,4 +474,116 @@ BEV_API int bev_deform_backward(const void* features, int dtype, int layout, int
     a.doffsets = doffsets;
     if ((st = cuda_status(bev_launch_deform_backward(a, dtype == BEV_BF16, V, s))) != BEV_OK) return st;
     return cuda_status(bev_launch_to_nchw(grad, B * N, C, Hf * Wf, a.Qtot * a.chan_per_chunk, dfeatures, s));
+}
+
+// ---------------------------------------------------------------------------
+// Lift-splat BEV pooling
+// ---------------------------------------------------------------------------
+
+namespace {
+
+bool lss_dims_ok(int B, int N, int D, int C, int Hf, int Wf, int X, int Y) {
+    if (!dims_ok(B, N, C, Hf, Wf)) return false;
+    if (D < 1 || D > 4096 || X < 1 || Y < 1 || X > BEV_MAX_DIM || Y > BEV_MAX_DIM) return false;
+    return true;
+}
+
+size_t lss_ws(int B, int C, int X, int Y, int for_backward) {
+    const size_t cells = (size_t)B * X * Y * C;
+    if (for_backward) return align_up(cells * sizeof(float));
+    return align_up(2 * sizeof(unsigned)) + align_up(cells * sizeof(unsigned long long));
+}
+
+int lss_prepare(const float* depth, const float* feat, int B, int N, int D, int C, int Hf, int Wf, const float* K,
+                const float* E, int img_h, int img_w, float dmin, float dstep, const bev_grid_t* grid,
+                void* workspace, size_t workspace_bytes, int for_backward, const void* const* extra, int n_extra,
+                bev::LssArgs* a) {
+    if (!depth || !feat || !K || !E || !grid) return BEV_ERR_INVALID_ARG;
+    for (int k = 0; k < n_extra; ++k)
+        if (!extra[k]) return BEV_ERR_INVALID_ARG;
+    if (!grid_ok(grid)) return BEV_ERR_INVALID_ARG;
+    if (!lss_dims_ok(B, N, D, C, Hf, Wf, grid->X, grid->Y)) return BEV_ERR_INVALID_ARG;
+    if (img_h < 1 || img_w < 1 || img_h > BEV_MAX_DIM || img_w > BEV_MAX_DIM) return BEV_ERR_INVALID_ARG;
+    if (!isfinite(dmin) || !isfinite(dstep) || !(dstep > 0.0f)) return BEV_ERR_INVALID_ARG;
+    if (C > bev::kLssMaxChannels) return BEV_ERR_UNSUPPORTED;
+    const size_t ws_need = lss_ws(B, C, grid->X, grid->Y, for_backward);
+    if (!workspace || workspace_bytes < ws_need || ((uintptr_t)workspace % kAlign) != 0) return BEV_ERR_WORKSPACE;
+    int dev;
+    int st = current_device(&dev);
+    if (st != BEV_OK) return st;
+    const void* ptrs[4] = {depth, feat, K, E};
+    for (int k = 0; k < 4; ++k)
+        if ((st = device_ptr(ptrs[k], dev)) != BEV_OK) return st;
+    for (int k = 0; k < n_extra; ++k)
+        if ((st = device_ptr(extra[k], dev)) != BEV_OK) return st;
+    if ((st = device_ptr(workspace, dev)) != BEV_OK) return BEV_ERR_WORKSPACE;
+    memset(a, 0, sizeof(*a));
+    a->depth = depth;
+    a->feat = feat;
+    a->K = K;
+    a->E = E;
+    a->B = B;
+    a->N = N;
+    a->D = D;
+    a->C = C;
+    a->Hf = Hf;
+    a->Wf = Wf;
+    a->X = grid->X;
+    a->Y = grid->Y;
+    a->sWi = (float)img_w / (float)Wf;
+    a->sHi = (float)img_h / (float)Hf;
+    a->dmin = dmin;
+    a->dstep = dstep;
+    a->xmin = grid->xmin;
+    a->ymin = grid->ymin;
+    a->zmin = grid->zmin;
+    a->zmax = grid->zmax;
+    a->dx = grid->dx;
+    a->dy = grid->dy;
+    a->points_per_batch = (long long)N * D * Hf * Wf;
+    return BEV_OK;
+}
+
+}  // namespace
+
+BEV_API size_t bev_lss_workspace_size(int B, int N, int C, int D, int Hf, int Wf, int X, int Y, int for_backward) {
+    if (!lss_dims_ok(B, N, D, C, Hf, Wf, X, Y)) return (size_t)-1;
+    return lss_ws(B, C, X, Y, for_backward);
+}
+
+BEV_API int bev_lss_forward(const float* depth, const float* feat, int B, int N, int D, int C, int Hf, int Wf,
+                            const float* intrinsics, const float* ego2cam, int img_h, int img_w, float dmin,
+                            float dstep, const bev_grid_t* grid, float* out, void* workspace,
+                            size_t workspace_bytes, bev_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const void* extra[1] = {out};
+    bev::LssArgs a;
+    int st = lss_prepare(depth, feat, B, N, D, C, Hf, Wf, intrinsics, ego2cam, img_h, img_w, dmin, dstep, grid,
+                         workspace, workspace_bytes, 0, extra, 1, &a);
+    if (st != BEV_OK) return st;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    a.maxabs = reinterpret_cast<unsigned*>(ws);
+    a.acc = reinterpret_cast<unsigned long long*>(ws + align_up(2 * sizeof(unsigned)));
+    a.out = out;
+    if ((st = cuda_status(cudaMemsetAsync(workspace, 0, lss_ws(B, C, a.X, a.Y, 0), s))) != BEV_OK) return st;
+    return cuda_status(bev_launch_lss_forward(a, s));
+}
+
+BEV_API int bev_lss_backward(const float* depth, const float* feat, const float* dout, int B, int N, int D, int C,
+                             int Hf, int Wf, const float* intrinsics, const float* ego2cam, int img_h, int img_w,
+                             float dmin, float dstep, const bev_grid_t* grid, float* ddepth, float* dfeat,
+                             void* workspace, size_t workspace_bytes, bev_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const void* extra[3] = {dout, ddepth, dfeat};
+    bev::LssArgs a;
+    int st = lss_prepare(depth, feat, B, N, D, C, Hf, Wf, intrinsics, ego2cam, img_h, img_w, dmin, dstep, grid,
+                         workspace, workspace_bytes, 1, extra, 3, &a);
+    if (st != BEV_OK) return st;
+    float* dcl = static_cast<float*>(workspace);
+    st = cuda_status(bev_launch_to_channels_last(dout, BEV_NCHW, 4, B, C, a.X * a.Y, C, dcl, s));
+    if (st != BEV_OK) return st;
+    a.dout_cl = dcl;
+    a.ddepth = ddepth;
+    a.dfeat = dfeat;
+    return cuda_status(bev_launch_lss_backward(a, s));
 }

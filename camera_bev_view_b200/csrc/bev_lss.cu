@@ -1,0 +1,291 @@
+// bev_lss.cu -- lift-splat BEV pooling, forward and backward (sm_100a).
+//
+// LSS tutorial, "Lift" and "Splat": every feature pixel (h, w) of camera n
+// spreads D depth bins along its ray; the point of bin k carries
+// depth[b,n,k,h,w] * feat[b,n,:,h,w] (the outer product), is placed in the
+// ego frame and summed into the BEV pillar it falls in:
+//   out[b, c, i, j] = sum over (n, k, h, w) in pillar (i, j) of depth * feat[c]
+// The tutorial makes the variable-length sum per pillar deterministic by
+// sorting the points by pillar and differencing a prefix sum.  Here every
+// term is instead converted to a 64-bit fixed-point integer (2^-s units, s
+// chosen per call from max|depth| max|feat| and the number of points per
+// batch item, so no pillar sum can overflow) and added with integer
+// reductions in L2: integer addition is exact and associative, so the sums
+// do not depend on the order in which the points arrive, and one pass over
+// the points suffices.  Bins of one pixel that land in the same pillar are
+// merged in registers first.  A final transpose converts the channels-last
+// integer sums to the fp32 [B,C,X,Y] output.
+//
+// Backward (a gather, deterministic): dout is made channels-last; each
+// pixel's bins read the dout vector of their pillar:
+//   ddepth[b,n,k,h,w] = dout[pillar] . feat[b,n,:,h,w]
+//   dfeat[b,n,c,h,w]  = sum_k depth[b,n,k,h,w] dout[pillar_k, c]
+// Four warps per pixel split its bins; their dfeat partials are added in warp
+// order.
+//
+// The frustum geometry follows one fixed fp32 order (separate roundings, IEEE
+// divides), the same as the oracle's, so pillar assignments are reproducible
+// bit for bit:
+//   u = (w + 0.5) (W_img / Wf);  v = (h + 0.5) (H_img / Hf);  d = dmin + k dstep
+//   yn = (v - cy) / fy;  xn = ((u - cx) - s yn) / fx;  pc = (xn d, yn d, d)
+//   q = pc - t;  x = (R00 q0 + R10 q1) + R20 q2 (likewise y, z)
+//   i = floor((x - xmin) / dx), j = floor((y - ymin) / dy), zmin <= z < zmax
+#include <stdint.h>
+
+#include "bev_lss.cuh"
+
+namespace bev {
+
+namespace {
+
+// Pillar (i * Y + j) of frustum point (h, w, k) of one camera, or -1.
+__device__ __forceinline__ int lss_cell(const LssArgs& a, const float* K, const float* E, int h, int w, int k) {
+    const float u = __fmul_rn(__fadd_rn((float)w, 0.5f), a.sWi);
+    const float v = __fmul_rn(__fadd_rn((float)h, 0.5f), a.sHi);
+    const float d = __fadd_rn(a.dmin, __fmul_rn((float)k, a.dstep));
+    const float yn = __fdiv_rn(__fsub_rn(v, K[5]), K[4]);
+    const float t = __fmul_rn(K[1], yn);
+    const float xn = __fdiv_rn(__fsub_rn(__fsub_rn(u, K[2]), t), K[0]);
+    const float pc[3] = {__fmul_rn(xn, d), __fmul_rn(yn, d), d};
+    float q[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) q[r] = __fsub_rn(pc[r], E[4 * r + 3]);
+    float p[3];
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+        p[c] = __fadd_rn(__fadd_rn(__fmul_rn(E[c], q[0]), __fmul_rn(E[4 + c], q[1])), __fmul_rn(E[8 + c], q[2]));
+    if (!(p[2] >= a.zmin && p[2] < a.zmax)) return -1;
+    const float fi = floorf(__fdiv_rn(__fsub_rn(p[0], a.xmin), a.dx));
+    const float fj = floorf(__fdiv_rn(__fsub_rn(p[1], a.ymin), a.dy));
+    if (!(fi >= 0.0f && fi < (float)a.X && fj >= 0.0f && fj < (float)a.Y)) return -1;
+    return (int)fi * a.Y + (int)fj;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Fraction bits s of the fixed point: |sum| <= points * max|depth| max|feat|
+// must stay below 2^62.
+__device__ __forceinline__ int lss_frac_bits(const LssArgs& a) {
+    const float m = __fmul_rn(__uint_as_float(a.maxabs[0]), __uint_as_float(a.maxabs[1]));
+    if (!(m > 0.0f)) return 0;
+    int e_m, e_p;
+    frexpf(m, &e_m);                       // m < 2^e_m
+    frexp((double)a.points_per_batch, &e_p);  // points < 2^e_p
+    return 62 - e_m - e_p;
+}
+
+}  // namespace
+
+// max |depth| and max |feat| (non-negative floats compare like their bits)
+__global__ void __launch_bounds__(256) lss_maxabs_kernel(const float* __restrict__ depth, size_t nd,
+                                                         const float* __restrict__ feat, size_t nf,
+                                                         unsigned* __restrict__ maxabs) {
+    unsigned md = 0, mf = 0;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nd; i += stride)
+        md = max(md, __float_as_uint(fabsf(depth[i])));
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nf; i += stride)
+        mf = max(mf, __float_as_uint(fabsf(feat[i])));
+    md = __reduce_max_sync(0xffffffffu, md);
+    mf = __reduce_max_sync(0xffffffffu, mf);
+    if ((threadIdx.x & 31) == 0) {
+        atomicMax(maxabs, md);
+        atomicMax(maxabs + 1, mf);
+    }
+}
+
+// One warp per pixel (b, n, h, w); lanes take channels c = lane + 32 v.
+template <int V>
+__global__ void __launch_bounds__(256) lss_forward_kernel(const LssArgs a) {
+    const int lane = threadIdx.x & 31;
+    const long long pix = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const long long npix = (long long)a.B * a.N * a.Hf * a.Wf;
+    if (pix >= npix) return;
+    const int w = (int)(pix % a.Wf);
+    const int h = (int)((pix / a.Wf) % a.Hf);
+    const long long bn = pix / ((long long)a.Hf * a.Wf);
+    const int b = (int)(bn / a.N);
+    const float* K = a.K + bn * 9;
+    const float* E = a.E + bn * 16;
+    const size_t hw = (size_t)a.Hf * a.Wf;
+    const size_t poff = (size_t)h * a.Wf + w;
+    const int s = lss_frac_bits(a);
+    float f[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        const int c = lane + 32 * v;
+        f[v] = c < a.C ? a.feat[((size_t)bn * a.C + c) * hw + poff] : 0.0f;
+    }
+    unsigned long long* acc = a.acc + (size_t)b * a.X * a.Y * a.C;
+    long long run[V];
+    int run_cell = -1;
+    for (int k0 = 0; k0 < a.D; k0 += 32) {
+        const int k = k0 + lane;
+        int cell = -1;
+        float al = 0.0f;
+        if (k < a.D) {
+            cell = lss_cell(a, K, E, h, w, k);
+            al = a.depth[((size_t)bn * a.D + k) * hw + poff];
+        }
+        const int kn = min(32, a.D - k0);
+        for (int kk = 0; kk < kn; ++kk) {
+            const int ck = __shfl_sync(0xffffffffu, cell, kk);
+            const float ak = __shfl_sync(0xffffffffu, al, kk);
+            if (ck < 0) continue;
+            if (ck != run_cell) {
+                if (run_cell >= 0) {
+#pragma unroll
+                    for (int v = 0; v < V; ++v)
+                        if (lane + 32 * v < a.C)
+                            atomicAdd(acc + (size_t)run_cell * a.C + lane + 32 * v, (unsigned long long)run[v]);
+                }
+                run_cell = ck;
+#pragma unroll
+                for (int v = 0; v < V; ++v) run[v] = 0;
+            }
+#pragma unroll
+            for (int v = 0; v < V; ++v) run[v] += __float2ll_rn(ldexpf(__fmul_rn(ak, f[v]), s));
+        }
+    }
+    if (run_cell >= 0) {
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+            if (lane + 32 * v < a.C)
+                atomicAdd(acc + (size_t)run_cell * a.C + lane + 32 * v, (unsigned long long)run[v]);
+    }
+}
+
+// Fixed-point channels-last sums [B][X*Y][C] -> fp32 out [B][C][X*Y], 32x32
+// tiles through shared memory.
+__global__ void __launch_bounds__(256) lss_convert_kernel(const LssArgs a) {
+    __shared__ float tile[32][33];
+    const int b = blockIdx.z;
+    const int p0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+    const int XY = a.X * a.Y;
+    const int s = lss_frac_bits(a);
+    const unsigned long long* acc = a.acc + (size_t)b * XY * a.C;
+    for (int r = threadIdx.y; r < 32; r += 8) {
+        const int p = p0 + r, c = c0 + threadIdx.x;
+        float v = 0.0f;
+        if (p < XY && c < a.C) v = (float)ldexp((double)(long long)acc[(size_t)p * a.C + c], -s);
+        tile[r][threadIdx.x] = v;
+    }
+    __syncthreads();
+    for (int r = threadIdx.y; r < 32; r += 8) {
+        const int c = c0 + r, p = p0 + threadIdx.x;
+        if (c < a.C && p < XY) a.out[((size_t)b * a.C + c) * XY + p] = tile[threadIdx.x][r];
+    }
+}
+
+// Backward: one CTA of kLssWarps warps per pixel; warp w takes bins
+// k = w, w + kLssWarps, ...; dout is channels-last [B][X*Y][C].
+template <int V>
+__global__ void __launch_bounds__(kLssWarps * 32) lss_backward_kernel(const LssArgs a) {
+    __shared__ float part[kLssWarps][kLssMaxChannels];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long pix = blockIdx.x;
+    const int w = (int)(pix % a.Wf);
+    const int h = (int)((pix / a.Wf) % a.Hf);
+    const long long bn = pix / ((long long)a.Hf * a.Wf);
+    const int b = (int)(bn / a.N);
+    const float* K = a.K + bn * 9;
+    const float* E = a.E + bn * 16;
+    const size_t hw = (size_t)a.Hf * a.Wf;
+    const size_t poff = (size_t)h * a.Wf + w;
+    const float* G = a.dout_cl + (size_t)b * a.X * a.Y * a.C;
+    float f[V], df[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        const int c = lane + 32 * v;
+        f[v] = c < a.C ? a.feat[((size_t)bn * a.C + c) * hw + poff] : 0.0f;
+        df[v] = 0.0f;
+    }
+    for (int k0 = warp; k0 < a.D; k0 += 32 * kLssWarps) {
+        const int k = k0 + kLssWarps * lane;
+        int cell = -1;
+        float al = 0.0f;
+        if (k < a.D) {
+            cell = lss_cell(a, K, E, h, w, k);
+            al = a.depth[((size_t)bn * a.D + k) * hw + poff];
+        }
+        float dd = 0.0f;  // this lane's bin's ddepth
+        for (int kk = 0; kk < 32 && k0 + kLssWarps * kk < a.D; ++kk) {
+            const int ck = __shfl_sync(0xffffffffu, cell, kk);
+            const float ak = __shfl_sync(0xffffffffu, al, kk);
+            if (ck < 0) continue;
+            float g[V];
+            float dot = 0.0f;
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const int c = lane + 32 * v;
+                g[v] = c < a.C ? G[(size_t)ck * a.C + c] : 0.0f;
+                dot = __fmaf_rn(g[v], f[v], dot);
+                df[v] = __fmaf_rn(ak, g[v], df[v]);
+            }
+            dot = warp_sum(dot);
+            if (lane == kk) dd = dot;
+        }
+        if (k < a.D) a.ddepth[((size_t)bn * a.D + k) * hw + poff] = dd;
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+        if (lane + 32 * v < a.C) part[warp][lane + 32 * v] = df[v];
+    __syncthreads();
+    for (int c = threadIdx.x; c < a.C; c += kLssWarps * 32) {
+        float s = part[0][c];
+#pragma unroll
+        for (int ww = 1; ww < kLssWarps; ++ww) s = __fadd_rn(s, part[ww][c]);
+        a.dfeat[((size_t)bn * a.C + c) * hw + poff] = s;
+    }
+}
+
+}  // namespace bev
+
+cudaError_t bev_launch_lss_forward(const bev::LssArgs& a, cudaStream_t st) {
+    using namespace bev;
+    const size_t nd = (size_t)a.B * a.N * a.D * a.Hf * a.Wf, nf = (size_t)a.B * a.N * a.C * a.Hf * a.Wf;
+    const size_t mx = (nd > nf ? nd : nf);
+    const int mblocks = (int)((mx + 255) / 256 < 148 * 8 ? (mx + 255) / 256 : 148 * 8);
+    lss_maxabs_kernel<<<mblocks, 256, 0, st>>>(a.depth, nd, a.feat, nf, a.maxabs);
+    const long long npix = (long long)a.B * a.N * a.Hf * a.Wf;
+    const unsigned blocks = (unsigned)((npix + 7) / 8);
+    const int V = (a.C + 31) / 32;
+    switch (V) {
+        case 1: lss_forward_kernel<1><<<blocks, 256, 0, st>>>(a); break;
+        case 2: lss_forward_kernel<2><<<blocks, 256, 0, st>>>(a); break;
+        case 3: lss_forward_kernel<3><<<blocks, 256, 0, st>>>(a); break;
+        case 4: lss_forward_kernel<4><<<blocks, 256, 0, st>>>(a); break;
+        case 5: lss_forward_kernel<5><<<blocks, 256, 0, st>>>(a); break;
+        case 6: lss_forward_kernel<6><<<blocks, 256, 0, st>>>(a); break;
+        case 7: lss_forward_kernel<7><<<blocks, 256, 0, st>>>(a); break;
+        case 8: lss_forward_kernel<8><<<blocks, 256, 0, st>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    const int XY = a.X * a.Y;
+    const dim3 grid((XY + 31) / 32, (a.C + 31) / 32, a.B);
+    lss_convert_kernel<<<grid, dim3(32, 8), 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t bev_launch_lss_backward(const bev::LssArgs& a, cudaStream_t st) {
+    using namespace bev;
+    const long long npix = (long long)a.B * a.N * a.Hf * a.Wf;
+    const int V = (a.C + 31) / 32;
+    const dim3 grid((unsigned)npix);
+    switch (V) {
+        case 1: lss_backward_kernel<1><<<grid, kLssWarps * 32, 0, st>>>(a); break;
+        case 2: lss_backward_kernel<2><<<grid, kLssWarps * 32, 0, st>>>(a); break;
+        case 3: lss_backward_kernel<3><<<grid, kLssWarps * 32, 0, st>>>(a); break;
+        case 4: lss_backward_kernel<4><<<grid, kLssWarps * 32, 0, st>>>(a); break;
+        case 5: lss_backward_kernel<5><<<grid, kLssWarps * 32, 0, st>>>(a); break;
+        case 6: lss_backward_kernel<6><<<grid, kLssWarps * 32, 0, st>>>(a); break;
+        case 7: lss_backward_kernel<7><<<grid, kLssWarps * 32, 0, st>>>(a); break;
+        case 8: lss_backward_kernel<8><<<grid, kLssWarps * 32, 0, st>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}

@@ -17,6 +17,9 @@ The functions keep the C names:
     bev_deform_forward(features, K, E, img_h, img_w, anchors, offsets, weights, ...) -> [B,Q,C]
     bev_deform_backward(features, K, E, img_h, img_w, anchors, offsets, weights, dout, ...)
                                                      -> (dfeatures, dweights, doffsets)
+    bev_lss_workspace_size(B, N, C, D, Hf, Wf, X, Y, for_backward) -> int
+    bev_lss_forward(depth, feat, K, E, img_h, img_w, dmin, dstep, grid, ...) -> [B,C,X,Y]
+    bev_lss_backward(depth, feat, dout, K, E, img_h, img_w, dmin, dstep, grid, ...) -> (ddepth, dfeat)
     bev_status_string(status)                        -> str
 """
 from __future__ import annotations
@@ -91,6 +94,14 @@ def lib():
         L.bev_deform_forward.restype = I
         L.bev_deform_backward.argtypes = [P, I, I, I, I, I, I, I, P, P, I, I, P, P, P, I, I, P, P, P, P, P, S, P]
         L.bev_deform_backward.restype = I
+        Fl = ctypes.c_float
+        L.bev_lss_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I]
+        L.bev_lss_workspace_size.restype = S
+        L.bev_lss_forward.argtypes = [P, P, I, I, I, I, I, I, P, P, I, I, Fl, Fl, ctypes.POINTER(BevGrid), P, P, S, P]
+        L.bev_lss_forward.restype = I
+        L.bev_lss_backward.argtypes = [P, P, P, I, I, I, I, I, I, P, P, I, I, Fl, Fl, ctypes.POINTER(BevGrid),
+                                       P, P, P, S, P]
+        L.bev_lss_backward.restype = I
         L.bev_status_string.argtypes = [I]
         L.bev_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -273,3 +284,50 @@ def bev_deform_backward(features: torch.Tensor, K: torch.Tensor, E: torch.Tensor
     if st != 0:
         raise BevError(st, "bev_deform_backward")
     return dF, dW, dO
+
+
+def bev_lss_workspace_size(B: int, N: int, C: int, D: int, Hf: int, Wf: int, X: int, Y: int,
+                           for_backward: int) -> int:
+    v = lib().bev_lss_workspace_size(B, N, C, D, Hf, Wf, X, Y, for_backward)
+    if v == ctypes.c_size_t(-1).value:
+        raise BevError(-1, "bev_lss_workspace_size")
+    return int(v)
+
+
+def bev_lss_forward(depth: torch.Tensor, feat: torch.Tensor, K: torch.Tensor, E: torch.Tensor, img_h: int,
+                    img_w: int, dmin: float, dstep: float, grid: BevGrid, out: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Lift-splat pooling: depth [B,N,D,Hf,Wf], feat [B,N,C,Hf,Wf] fp32 ->
+    out [B,C,X,Y] fp32."""
+    B, N, D, Hf, Wf = depth.shape
+    C = feat.shape[2]
+    dev = depth.device
+    if out is None:
+        out = torch.empty((B, C, grid.X, grid.Y), dtype=torch.float32, device=dev)
+    ws, ws_bytes = _workspace(bev_lss_workspace_size(B, N, C, D, Hf, Wf, grid.X, grid.Y, 0), dev, workspace)
+    st = lib().bev_lss_forward(depth.data_ptr(), feat.data_ptr(), B, N, D, C, Hf, Wf, K.data_ptr(), E.data_ptr(),
+                               int(img_h), int(img_w), float(dmin), float(dstep), ctypes.byref(grid), out.data_ptr(),
+                               ws.data_ptr() if ws is not None else None, ws_bytes, _stream_ptr(stream))
+    if st != 0:
+        raise BevError(st, "bev_lss_forward")
+    return out
+
+
+def bev_lss_backward(depth: torch.Tensor, feat: torch.Tensor, dout: torch.Tensor, K: torch.Tensor, E: torch.Tensor,
+                     img_h: int, img_w: int, dmin: float, dstep: float, grid: BevGrid, out: tuple | None = None,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """Gradients for dout [B,C,X,Y]: (ddepth [B,N,D,Hf,Wf], dfeat [B,N,C,Hf,Wf])."""
+    B, N, D, Hf, Wf = depth.shape
+    C = feat.shape[2]
+    dev = depth.device
+    if out is None:
+        out = (torch.empty_like(depth, dtype=torch.float32), torch.empty_like(feat, dtype=torch.float32))
+    dd, df = out
+    ws, ws_bytes = _workspace(bev_lss_workspace_size(B, N, C, D, Hf, Wf, grid.X, grid.Y, 1), dev, workspace)
+    st = lib().bev_lss_backward(depth.data_ptr(), feat.data_ptr(), dout.data_ptr(), B, N, D, C, Hf, Wf,
+                                K.data_ptr(), E.data_ptr(), int(img_h), int(img_w), float(dmin), float(dstep),
+                                ctypes.byref(grid), dd.data_ptr(), df.data_ptr(),
+                                ws.data_ptr() if ws is not None else None, ws_bytes, _stream_ptr(stream))
+    if st != 0:
+        raise BevError(st, "bev_lss_backward")
+    return dd, df

@@ -235,6 +235,56 @@ int bev_deform_backward(const void* features, int dtype, int layout, int B, int 
                         const float* dout, float* dfeatures, float* dweights, float* doffsets,
                         void* workspace, size_t workspace_bytes, bev_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Lift-splat BEV pooling (LSS tutorial, "Lift" and "Splat").  Every feature
+ * pixel (h, w) of camera n spreads D depth bins along its ray; bin k sits at
+ * depth dmin + k * dstep, at the pixel centre u = (w + 0.5) W_img / Wf,
+ * v = (h + 0.5) H_img / Hf.  Its point, depth * K^-1 [u v 1]^T in the camera
+ * frame, is placed in the ego frame as R^T (pc - t) (E = [R | t] maps ego to
+ * camera, R a rotation; K upper triangular) and carries
+ * depth[b,n,k,h,w] * feat[b,n,:,h,w].  Points are summed into the BEV pillar
+ * (i, j) = (floor((x - xmin) / dx), floor((y - ymin) / dy)); z is not binned
+ * and points outside [xmin, xmax) x [ymin, ymax) x [zmin, zmax) are dropped:
+ *   out[b, c, i, j] = sum over points in pillar (i, j) of depth * feat[c]
+ * grid: from bev_grid_spec; X, Y, xmin, ymin, zmin, zmax, dx, dy are used, Z
+ * is ignored.  The fp32 order of the geometry is fixed (separate roundings,
+ * IEEE divides):
+ *   yn = (v - K12) / K11;  xn = ((u - K02) - K01 yn) / K00;  pc = (xn d, yn d, d)
+ *   q = pc - t;  x = (R00 q0 + R10 q1) + R20 q2  (likewise y, z)
+ * ------------------------------------------------------------------------- */
+
+/* Device scratch (bytes, 256-byte aligned) of bev_lss_forward (for_backward
+ * = 0) or bev_lss_backward (1); (size_t)-1 for invalid arguments. */
+size_t bev_lss_workspace_size(int B, int N, int C, int D, int Hf, int Wf, int X, int Y, int for_backward);
+
+/* Forward of the lift-splat pooling.
+ *   depth      [B,N,D,Hf,Wf] fp32 (for instance a softmax over the bins)
+ *   feat       [B,N,C,Hf,Wf] fp32, C <= 256
+ *   intrinsics [B,N,3,3], ego2cam [B,N,4,4] fp32; img_h, img_w the image size
+ *   dmin, dstep  depth of bin 0 and the bin spacing (> 0)
+ *   out        [B,C,X,Y] fp32, fully overwritten
+ * Each term depth * feat is rounded to a 64-bit fixed point with s fraction
+ * bits, s = 62 - e(max|depth| max|feat|) - e(N D Hf Wf) (e(v): the smallest e
+ * with v < 2^e), and the pillar sums are exact integer sums, so results are
+ * reproducible bit for bit whatever the order of the points; the absolute
+ * error of a pillar is at most (its points) * 2^-(s+1) plus the final
+ * rounding to fp32.  Returns BEV_OK, BEV_ERR_INVALID_ARG, BEV_ERR_UNSUPPORTED,
+ * BEV_ERR_WORKSPACE or BEV_ERR_CUDA. */
+int bev_lss_forward(const float* depth, const float* feat, int B, int N, int D, int C, int Hf, int Wf,
+                    const float* intrinsics, const float* ego2cam, int img_h, int img_w, float dmin, float dstep,
+                    const bev_grid_t* grid, float* out, void* workspace, size_t workspace_bytes,
+                    bev_stream_t stream);
+
+/* Backward of the lift-splat pooling for dout [B,C,X,Y] fp32:
+ *   ddepth [B,N,D,Hf,Wf] = dout[pillar of the point] . feat (0 for dropped points)
+ *   dfeat  [B,N,C,Hf,Wf] = sum_k depth * dout[pillar of bin k]
+ * Both fully overwritten; a gather in a fixed order, so reproducible bit for
+ * bit.  Other arguments as for bev_lss_forward. */
+int bev_lss_backward(const float* depth, const float* feat, const float* dout, int B, int N, int D, int C,
+                     int Hf, int Wf, const float* intrinsics, const float* ego2cam, int img_h, int img_w,
+                     float dmin, float dstep, const bev_grid_t* grid, float* ddepth, float* dfeat,
+                     void* workspace, size_t workspace_bytes, bev_stream_t stream);
+
 /* Static, human-readable text for a status code. */
 const char* bev_status_string(int status);
 

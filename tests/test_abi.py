@@ -201,3 +201,58 @@ def test_deform_argument_errors(L):
 def test_deform_valid_host_checks_then_cuda_error_without_device(L):
     assert _dfwd(L) == -4
     assert _dbwd(L) == -4
+
+
+# --------------------------------------------------------------------------
+# lift-splat pooling
+# --------------------------------------------------------------------------
+
+def test_header_declares_the_lss_calls():
+    names = declared_functions()
+    for n in ["bev_lss_workspace_size", "bev_lss_forward", "bev_lss_backward"]:
+        assert n in names
+
+
+def test_lss_workspace_sizes(L):
+    assert L.bev_lss_workspace_size(1, 6, 64, 41, 8, 22, 200, 200, 0) == 256 + 200 * 200 * 64 * 8
+    assert L.bev_lss_workspace_size(1, 6, 64, 41, 8, 22, 200, 200, 1) == 200 * 200 * 64 * 4
+    assert L.bev_lss_workspace_size(1, 6, 64, 0, 8, 22, 200, 200, 0) == ctypes.c_size_t(-1).value
+    assert L.bev_lss_workspace_size(1, 6, 64, 41, 8, 22, 0, 200, 0) == ctypes.c_size_t(-1).value
+
+
+def _lfwd(L, **kw):
+    g = ops.bev_grid_spec((-50, 50, -50, 50, -10, 10), (0.5, 0.5, 20.0))
+    a = dict(depth=FAKE, feat=FAKE, B=1, N=6, D=41, C=64, Hf=8, Wf=22, K=FAKE, E=FAKE, img_h=128, img_w=352,
+             dmin=4.0, dstep=1.0, grid=ctypes.byref(g), out=FAKE, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.bev_lss_forward(a["depth"], a["feat"], a["B"], a["N"], a["D"], a["C"], a["Hf"], a["Wf"], a["K"],
+                             a["E"], a["img_h"], a["img_w"], a["dmin"], a["dstep"], a["grid"], a["out"], a["ws"],
+                             a["ws_bytes"], a["stream"])
+
+
+def _lbwd(L, **kw):
+    g = ops.bev_grid_spec((-50, 50, -50, 50, -10, 10), (0.5, 0.5, 20.0))
+    a = dict(depth=FAKE, feat=FAKE, dout=FAKE, B=1, N=6, D=41, C=64, Hf=8, Wf=22, K=FAKE, E=FAKE, img_h=128,
+             img_w=352, dmin=4.0, dstep=1.0, grid=ctypes.byref(g), dd=FAKE, df=FAKE, ws=FAKE, ws_bytes=1 << 30,
+             stream=None)
+    a.update(kw)
+    return L.bev_lss_backward(a["depth"], a["feat"], a["dout"], a["B"], a["N"], a["D"], a["C"], a["Hf"], a["Wf"],
+                              a["K"], a["E"], a["img_h"], a["img_w"], a["dmin"], a["dstep"], a["grid"], a["dd"],
+                              a["df"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_lss_argument_errors(L):
+    common = [(dict(depth=None), -1), (dict(feat=None), -1), (dict(K=None), -1), (dict(grid=None), -1),
+              (dict(D=0), -1), (dict(N=40), -1), (dict(img_w=0), -1), (dict(dstep=0.0), -1),
+              (dict(dstep=float("nan")), -1), (dict(dmin=float("inf")), -1), (dict(C=257), -2),
+              (dict(ws=None), -3), (dict(ws_bytes=64), -3), (dict(ws=FAKE + 8), -3)]
+    for kw, want in common + [(dict(out=None), -1)]:
+        assert _lfwd(L, **kw) == want, kw
+    for kw, want in common + [(dict(dout=None), -1), (dict(dd=None), -1), (dict(df=None), -1)]:
+        assert _lbwd(L, **kw) == want, kw
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_lss_valid_host_checks_then_cuda_error_without_device(L):
+    assert _lfwd(L) == -4
+    assert _lbwd(L) == -4
