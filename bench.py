@@ -22,6 +22,10 @@ used on the data path ("scaling": "weak").
 the host cores, on a band of BEV rows per step, and prints the same JSON line
 with "impl": "reference".
 
+--op lss measures the lift-splat BEV pooling (LSS tutorial, "Lift" and
+"Splat"): one step = forward + backward (depth and feature gradients) of the
+``lss`` workload (6 cameras, 8x22 features, 41 depth bins, C64, 200x200).
+
 --op deform measures the deformable aggregation instead (SparseDriveV2 notes,
 "Deformable Aggregation"): one step = forward + backward (feature, weight and
 keypoint-offset gradients) over the queries of the ``deform`` workload (900
@@ -58,10 +62,12 @@ def parse_args():
     ap.add_argument("--workload", default="nuscenes")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--op", choices=["vt", "deform"], default="vt")
+    ap.add_argument("--op", choices=["vt", "deform", "lss"], default="vt")
     args = ap.parse_args()
     if args.op == "deform" and args.workload == "nuscenes":
         args.workload = "deform"
+    if args.op == "lss" and args.workload == "nuscenes":
+        args.workload = "lss"
     return args
 
 
@@ -90,6 +96,8 @@ KERNEL_SOURCES = {
     "sample_backward_kernel": ["bev_backward.cu", "bev_warp.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
     "deform_forward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
     "deform_backward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
+    "lss_forward_kernel": ["bev_lss.cu", "bev_lss.cuh"],
+    "lss_backward_kernel": ["bev_lss.cu", "bev_lss.cuh"],
 }
 
 
@@ -601,9 +609,147 @@ def run_deform(args):
     print(json.dumps(line), flush=True)
 
 
+LSS_METRIC = "lift-splat BEV pooling output elements/s (B·C·X·Y) and achieved HBM GB/s vs roofline, 1×B200"
+
+
+def lss_oracle_step(w):
+    """One oracle forward + backward of the lift-splat pooling over the whole
+    workload (same seeded inputs); returns seconds.  Single-threaded."""
+    import oracle
+    from camera_bev_view_b200 import inputs as I
+    depth, feat = I.make_lss_inputs(w)
+    K, E = I.make_rigs(w)
+    dout = I.make_lss_dout(w)
+    g = oracle.LssGrid(w.ranges, w.res_xy, w.dbound)
+    t0 = time.perf_counter()
+    oracle.lss_forward(depth, feat, K, E, w.img_h, w.img_w, g)
+    oracle.lss_backward(depth, feat, dout, K, E, w.img_h, w.img_w, g)
+    return time.perf_counter() - t0
+
+
+def run_lss(args):
+    import torch
+
+    from camera_bev_view_b200 import inputs as I
+    from camera_bev_view_b200 import ops
+
+    rank, world, local = dist_env()
+    w = I.LSS_WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        for _ in range(args.warmup):
+            lss_oracle_step(w)
+        times = [lss_oracle_step(w) for _ in range(args.steps)]
+        value = w.out_elems * len(times) / sum(times)
+        line = {"impl": "reference", "metric": LSS_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (softmax depth, N(0,1) features, 6-camera rig)", "config": {"workload": w.name},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                 "sample": "the whole workload, forward + backward, per step"},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    depth_h, feat_h = I.make_lss_inputs(w, shard=rank)
+    K_h, E_h = I.make_rigs(w, shard=rank)
+    dout_h = I.make_lss_dout(w, shard=rank)
+    depth, feat, K, E, dout = (t.to(dev) for t in (depth_h, feat_h, K_h, E_h, dout_h))
+    B, N, D, Hf, Wf = depth.shape
+    C = feat.shape[2]
+    g = ops.bev_grid_spec(w.ranges, w.res_xy + (w.zr[1] - w.zr[0],))
+    dmin, _, dstep = w.dbound
+    out = torch.empty((B, C, w.X, w.Y), device=dev)
+    grads = (torch.empty_like(depth), torch.empty_like(feat))
+    ws = torch.empty(max(ops.bev_lss_workspace_size(B, N, C, D, Hf, Wf, w.X, w.Y, 0),
+                         ops.bev_lss_workspace_size(B, N, C, D, Hf, Wf, w.X, w.Y, 1)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stages = {
+        "forward": lambda: ops.bev_lss_forward(depth, feat, K, E, w.img_h, w.img_w, dmin, dstep, g, out=out,
+                                               workspace=ws),
+        "backward": lambda: ops.bev_lss_backward(depth, feat, dout, K, E, w.img_h, w.img_w, dmin, dstep, g,
+                                                 out=grads, workspace=ws),
+    }
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for f in stages.values():
+            f()
+        stream.synchronize()
+        for name, f in stages.items():
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                f()
+            graphs[name] = gr
+        for _ in range(args.warmup):
+            flush.zero_()
+            for gr in graphs.values():
+                gr.replay()
+        stream.synchronize()
+        names = list(stages)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local) as clocks:
+            for k in range(args.steps):
+                flush.zero_()
+                ev[k][0].record(stream)
+                for si, name in enumerate(names):
+                    graphs[name].replay()
+                    ev[k][si + 1].record(stream)
+            torch.cuda.synchronize(dev)
+        per = {name: [ev[k][si].elapsed_time(ev[k][si + 1]) for k in range(args.steps)]
+               for si, name in enumerate(names)}
+    for gr in graphs.values():
+        gr.reset()
+    stage_ms = {name: sum(v) / len(v) for name, v in per.items()}
+    ms = sum(stage_ms.values())
+    elems = w.out_elems
+    peak, peak_src = hbm_peak()
+    inputs_bytes = (depth.numel() + feat.numel()) * 4
+    fwd_bytes = inputs_bytes + elems * 4
+    bwd_bytes = inputs_bytes + elems * 4 + (depth.numel() + feat.numel()) * 4
+    dom = "forward" if stage_ms["forward"] >= stage_ms["backward"] else "backward"
+    dom_bytes = fwd_bytes if dom == "forward" else bwd_bytes
+    kname = "lss_forward_kernel" if dom == "forward" else "lss_backward_kernel"
+    achieved = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
+    line = {
+        "metric": LSS_METRIC, "value": elems / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (softmax depth, N(0,1) features, 6-camera rig)",
+        "config": {"workload": f"{w.name}: B{B} N{N} D{D} C{C} {Hf}x{Wf} (img {w.img_h}x{w.img_w}) -> {w.X}x{w.Y}",
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "timing": "CUDA events around CUDA-graph replays of each stage, launching stream"},
+        "stages_ms": stage_ms,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(kname, w.name), "kernel": kname, "stage": dom,
+                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "note": "depth and features read once + output written once (backward: + dout read, "
+                             "ddepth and dfeat written); timed over the whole call",
+                     "peak_source": peak_src},
+        "gpu_launches": args.steps * 6,
+        "clocks": clocks.summary(),
+    }
+    if args.cpu_seconds > 0:
+        spent, steps = 0.0, 0
+        while steps == 0 or spent < args.cpu_seconds:
+            spent += lss_oracle_step(w)
+            steps += 1
+        line["cpu_baseline"] = {"value": elems * steps / spent, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": f"{steps} whole forward+backward step(s) of the {w.name} workload "
+                                          f"({spent:.1f} s, single-threaded)"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
-    if args.op == "deform":
+    if args.op == "lss":
+        run_lss(args)
+    elif args.op == "deform":
         run_deform(args)
     elif args.impl == "reference":
         run_reference(args)

@@ -3,8 +3,10 @@
 // to_channels_last: features [BN][C][HW] (or [BN][HW][C]) -> [BN][HW][Cp] with
 //   zero padding channels, so that one texel's channel vector is contiguous
 //   and 16-byte aligned for the gather kernels.  Pure HBM-bound copies: the
-//   NCHW case is a 32x32 shared-memory tiled transpose (coalesced on both
-//   sides); the unaligned-NHWC case is a straight strided copy.
+//   NCHW case moves 4x4 blocks with 16-byte loads and stores for 4-byte
+//   elements when the shapes allow it, else a 32x32 shared-memory tiled
+//   transpose (coalesced on both sides); the unaligned-NHWC case is a straight
+//   strided copy.
 // to_nchw: the fp32 channels-last gradient buffer [BN][HW][Cp] -> [BN][C][HW].
 //   When HW is a multiple of 4 and the output is 16-byte aligned, each thread
 //   moves a 4 texel x 4 channel block with 16-byte loads and 16-byte stores
@@ -67,6 +69,29 @@ __global__ void __launch_bounds__(256) nhwc_to_nchw_kernel(const float* __restri
     }
 }
 
+// 4x4 register-blocked NCHW -> channels-last copy for 4-byte elements: block
+// (16 x 16 threads) covers 64 channels x 64 texels; thread (tx, ty) reads
+// channels 4 ty .. 4 ty + 3 at texels 4 tx .. 4 tx + 3 and writes them as four
+// texel rows; padding channels (C <= c < Cp) are written as 0.  HW % 4 == 0,
+// Cp % 4 == 0, both pointers 16-byte aligned.
+__global__ void __launch_bounds__(256) nchw_to_nhwc_v4_kernel(const float* __restrict__ src, int C, int HW,
+                                                              int Cp, float* __restrict__ dst) {
+    const size_t bn = blockIdx.z;
+    const int c = blockIdx.y * 64 + 4 * threadIdx.y;
+    const int p = blockIdx.x * 64 + 4 * threadIdx.x;
+    if (p >= HW || c >= Cp) return;
+    float4 r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r[i] = c + i < C ? __ldg(reinterpret_cast<const float4*>(src + (bn * C + c + i) * (size_t)HW + p))
+                         : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float* d = dst + (bn * HW + p) * (size_t)Cp + c;
+    *reinterpret_cast<float4*>(d) = make_float4(r[0].x, r[1].x, r[2].x, r[3].x);
+    *reinterpret_cast<float4*>(d + Cp) = make_float4(r[0].y, r[1].y, r[2].y, r[3].y);
+    *reinterpret_cast<float4*>(d + 2 * (size_t)Cp) = make_float4(r[0].z, r[1].z, r[2].z, r[3].z);
+    *reinterpret_cast<float4*>(d + 3 * (size_t)Cp) = make_float4(r[0].w, r[1].w, r[2].w, r[3].w);
+}
+
 // 4x4 register-blocked transpose: block (16 x 16 threads) covers 64 texels x
 // 64 channels; thread (tx, ty) reads texels 4 ty .. 4 ty + 3 at channels
 // 4 tx .. 4 tx + 3 and writes them back as four channel rows.  HW % 4 == 0,
@@ -96,7 +121,11 @@ __global__ void __launch_bounds__(256) nhwc_to_nchw_v4_kernel(const float* __res
 
 cudaError_t bev_launch_to_channels_last(const void* src, int layout, int esize, int BN, int C, int HW,
                                         int Cp, void* dst, cudaStream_t stream) {
-    if (layout == 0) {  // NCHW
+    if (layout == 0 && esize == 4 && HW % 4 == 0 && Cp % 4 == 0 && ((uintptr_t)src % 16) == 0 &&
+        ((uintptr_t)dst % 16) == 0) {
+        const dim3 grid((HW + 63) / 64, (Cp + 63) / 64, BN);
+        bev::nchw_to_nhwc_v4_kernel<<<grid, dim3(16, 16), 0, stream>>>((const float*)src, C, HW, Cp, (float*)dst);
+    } else if (layout == 0) {  // NCHW
         const dim3 grid((HW + bev::kT - 1) / bev::kT, (Cp + bev::kT - 1) / bev::kT, BN);
         const dim3 block(bev::kT, 8);
         if (esize == 4)

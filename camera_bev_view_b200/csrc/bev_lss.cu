@@ -85,16 +85,56 @@ __global__ void __launch_bounds__(256) lss_maxabs_kernel(const float* __restrict
                                                          const float* __restrict__ feat, size_t nf,
                                                          unsigned* __restrict__ maxabs) {
     unsigned md = 0, mf = 0;
+    const size_t tid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
     const size_t stride = (size_t)gridDim.x * blockDim.x;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nd; i += stride)
-        md = max(md, __float_as_uint(fabsf(depth[i])));
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nf; i += stride)
-        mf = max(mf, __float_as_uint(fabsf(feat[i])));
+    auto absmax = [&](const float* p, size_t n) -> unsigned {
+        unsigned m = 0;
+        // 16-byte loads, four in flight per thread, when the array allows
+        if (((uintptr_t)p & 15) == 0) {
+            const float4* p4 = reinterpret_cast<const float4*>(p);
+            const size_t n4 = n / 4;
+            size_t i = tid;
+            for (; i + 3 * stride < n4; i += 4 * stride) {
+                float4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) v[u] = __ldg(p4 + i + u * stride);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    m = max(m, max(max(__float_as_uint(fabsf(v[u].x)), __float_as_uint(fabsf(v[u].y))),
+                                   max(__float_as_uint(fabsf(v[u].z)), __float_as_uint(fabsf(v[u].w)))));
+            }
+            for (; i < n4; i += stride) {
+                const float4 v = __ldg(p4 + i);
+                m = max(m, max(max(__float_as_uint(fabsf(v.x)), __float_as_uint(fabsf(v.y))),
+                               max(__float_as_uint(fabsf(v.z)), __float_as_uint(fabsf(v.w)))));
+            }
+            for (size_t j = 4 * n4 + tid; j < n; j += stride) m = max(m, __float_as_uint(fabsf(p[j])));
+        } else {
+            for (size_t j = tid; j < n; j += stride) m = max(m, __float_as_uint(fabsf(p[j])));
+        }
+        return m;
+    };
+    md = absmax(depth, nd);
+    mf = absmax(feat, nf);
     md = __reduce_max_sync(0xffffffffu, md);
     mf = __reduce_max_sync(0xffffffffu, mf);
+    // one pair of atomics per CTA: the global maxima live at two addresses,
+    // so per-warp atomics would queue up behind each other in L2
+    __shared__ unsigned sd[8], sf[8];
     if ((threadIdx.x & 31) == 0) {
-        atomicMax(maxabs, md);
-        atomicMax(maxabs + 1, mf);
+        sd[threadIdx.x >> 5] = md;
+        sf[threadIdx.x >> 5] = mf;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        md = threadIdx.x < 8 ? sd[threadIdx.x] : 0u;
+        mf = threadIdx.x < 8 ? sf[threadIdx.x] : 0u;
+        md = __reduce_max_sync(0xffffffffu, md);
+        mf = __reduce_max_sync(0xffffffffu, mf);
+        if (threadIdx.x == 0) {
+            atomicMax(maxabs, md);
+            atomicMax(maxabs + 1, mf);
+        }
     }
 }
 
@@ -213,21 +253,35 @@ __global__ void __launch_bounds__(kLssWarps * 32) lss_backward_kernel(const LssA
             al = a.depth[((size_t)bn * a.D + k) * hw + poff];
         }
         float dd = 0.0f;  // this lane's bin's ddepth
-        for (int kk = 0; kk < 32 && k0 + kLssWarps * kk < a.D; ++kk) {
-            const int ck = __shfl_sync(0xffffffffu, cell, kk);
-            const float ak = __shfl_sync(0xffffffffu, al, kk);
-            if (ck < 0) continue;
-            float g[V];
-            float dot = 0.0f;
+        const int kn = min(32, (a.D - k0 + kLssWarps - 1) / kLssWarps);
+        // four bins per step: their dout vectors are loaded before any is used
+        for (int kb = 0; kb < kn; kb += 4) {
+            int ck[4];
+            float ak[4], g[4][V];
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int c = lane + 32 * v;
-                g[v] = c < a.C ? G[(size_t)ck * a.C + c] : 0.0f;
-                dot = __fmaf_rn(g[v], f[v], dot);
-                df[v] = __fmaf_rn(ak, g[v], df[v]);
+            for (int u = 0; u < 4; ++u) {
+                const int kk = kb + u;
+                ck[u] = __shfl_sync(0xffffffffu, cell, kk & 31);
+                ak[u] = __shfl_sync(0xffffffffu, al, kk & 31);
+                if (kk >= kn) ck[u] = -1;
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    const int c = lane + 32 * v;
+                    g[u][v] = (ck[u] >= 0 && c < a.C) ? G[(size_t)ck[u] * a.C + c] : 0.0f;
+                }
             }
-            dot = warp_sum(dot);
-            if (lane == kk) dd = dot;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (ck[u] < 0) continue;
+                float dot = 0.0f;
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    dot = __fmaf_rn(g[u][v], f[v], dot);
+                    df[v] = __fmaf_rn(ak[u], g[u][v], df[v]);
+                }
+                dot = warp_sum(dot);
+                if (lane == kb + u) dd = dot;
+            }
         }
         if (k < a.D) a.ddepth[((size_t)bn * a.D + k) * hw + poff] = dd;
     }
@@ -249,7 +303,7 @@ cudaError_t bev_launch_lss_forward(const bev::LssArgs& a, cudaStream_t st) {
     using namespace bev;
     const size_t nd = (size_t)a.B * a.N * a.D * a.Hf * a.Wf, nf = (size_t)a.B * a.N * a.C * a.Hf * a.Wf;
     const size_t mx = (nd > nf ? nd : nf);
-    const int mblocks = (int)((mx + 255) / 256 < 148 * 8 ? (mx + 255) / 256 : 148 * 8);
+    const int mblocks = (int)((mx / 4 + 255) / 256 < 148 * 4 ? (mx / 4 + 255) / 256 + 1 : 148 * 4);
     lss_maxabs_kernel<<<mblocks, 256, 0, st>>>(a.depth, nd, a.feat, nf, a.maxabs);
     const long long npix = (long long)a.B * a.N * a.Hf * a.Wf;
     const unsigned blocks = (unsigned)((npix + 7) / 8);
