@@ -38,14 +38,26 @@ namespace bev {
 
 namespace {
 
-// Pillar (i * Y + j) of frustum point (h, w, k) of one camera, or -1.
-__device__ __forceinline__ int lss_cell(const LssArgs& a, const float* K, const float* E, int h, int w, int k) {
+// Ray of feature pixel (h, w) through one camera: (xn, yn) with the camera
+// point of depth d at (xn d, yn d, d).
+struct Ray {
+    float xn, yn;
+};
+
+__device__ __forceinline__ Ray lss_ray(const LssArgs& a, const float* K, int h, int w) {
     const float u = __fmul_rn(__fadd_rn((float)w, 0.5f), a.sWi);
     const float v = __fmul_rn(__fadd_rn((float)h, 0.5f), a.sHi);
+    Ray r;
+    r.yn = __fdiv_rn(__fsub_rn(v, K[5]), K[4]);
+    const float t = __fmul_rn(K[1], r.yn);
+    r.xn = __fdiv_rn(__fsub_rn(__fsub_rn(u, K[2]), t), K[0]);
+    return r;
+}
+
+// Pillar (i * Y + j) of bin k of a pixel's ray, or -1.
+__device__ __forceinline__ int lss_cell(const LssArgs& a, const Ray& ray, const float* E, int k) {
     const float d = __fadd_rn(a.dmin, __fmul_rn((float)k, a.dstep));
-    const float yn = __fdiv_rn(__fsub_rn(v, K[5]), K[4]);
-    const float t = __fmul_rn(K[1], yn);
-    const float xn = __fdiv_rn(__fsub_rn(__fsub_rn(u, K[2]), t), K[0]);
+    const float xn = ray.xn, yn = ray.yn;
     const float pc[3] = {__fmul_rn(xn, d), __fmul_rn(yn, d), d};
     float q[3];
 #pragma unroll
@@ -68,15 +80,19 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Fraction bits s of the fixed point: |sum| <= points * max|depth| max|feat|
-// must stay below 2^62.
+// must stay below 2^62.  Clamped to [-126, 127] so that 2^s is an fp32
+// number (a smaller s only costs resolution).
 __device__ __forceinline__ int lss_frac_bits(const LssArgs& a) {
     const float m = __fmul_rn(__uint_as_float(a.maxabs[0]), __uint_as_float(a.maxabs[1]));
     if (!(m > 0.0f)) return 0;
     int e_m, e_p;
     frexpf(m, &e_m);                       // m < 2^e_m
     frexp((double)a.points_per_batch, &e_p);  // points < 2^e_p
-    return 62 - e_m - e_p;
+    return max(-126, min(127, 62 - e_m - e_p));
 }
+
+// 2^s as fp32, s in [-126, 127], built from its exponent bits (exact).
+__device__ __forceinline__ float pow2f(int s) { return __int_as_float((s + 127) << 23); }
 
 }  // namespace
 
@@ -153,7 +169,8 @@ __global__ void __launch_bounds__(256) lss_forward_kernel(const LssArgs a) {
     const float* E = a.E + bn * 16;
     const size_t hw = (size_t)a.Hf * a.Wf;
     const size_t poff = (size_t)h * a.Wf + w;
-    const int s = lss_frac_bits(a);
+    const float scale = pow2f(lss_frac_bits(a));
+    const Ray ray = lss_ray(a, K, h, w);
     float f[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) {
@@ -168,7 +185,7 @@ __global__ void __launch_bounds__(256) lss_forward_kernel(const LssArgs a) {
         int cell = -1;
         float al = 0.0f;
         if (k < a.D) {
-            cell = lss_cell(a, K, E, h, w, k);
+            cell = lss_cell(a, ray, E, k);
             al = a.depth[((size_t)bn * a.D + k) * hw + poff];
         }
         const int kn = min(32, a.D - k0);
@@ -188,7 +205,7 @@ __global__ void __launch_bounds__(256) lss_forward_kernel(const LssArgs a) {
                 for (int v = 0; v < V; ++v) run[v] = 0;
             }
 #pragma unroll
-            for (int v = 0; v < V; ++v) run[v] += __float2ll_rn(ldexpf(__fmul_rn(ak, f[v]), s));
+            for (int v = 0; v < V; ++v) run[v] += __float2ll_rn(__fmul_rn(__fmul_rn(ak, f[v]), scale));
         }
     }
     if (run_cell >= 0) {
@@ -237,6 +254,7 @@ __global__ void __launch_bounds__(kLssWarps * 32) lss_backward_kernel(const LssA
     const size_t hw = (size_t)a.Hf * a.Wf;
     const size_t poff = (size_t)h * a.Wf + w;
     const float* G = a.dout_cl + (size_t)b * a.X * a.Y * a.C;
+    const Ray ray = lss_ray(a, K, h, w);
     float f[V], df[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) {
@@ -249,7 +267,7 @@ __global__ void __launch_bounds__(kLssWarps * 32) lss_backward_kernel(const LssA
         int cell = -1;
         float al = 0.0f;
         if (k < a.D) {
-            cell = lss_cell(a, K, E, h, w, k);
+            cell = lss_cell(a, ray, E, k);
             al = a.depth[((size_t)bn * a.D + k) * hw + poff];
         }
         float dd = 0.0f;  // this lane's bin's ddepth

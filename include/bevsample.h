@@ -265,7 +265,8 @@ size_t bev_lss_workspace_size(int B, int N, int C, int D, int Hf, int Wf, int X,
  *   out        [B,C,X,Y] fp32, fully overwritten
  * Each term depth * feat is rounded to a 64-bit fixed point with s fraction
  * bits, s = 62 - e(max|depth| max|feat|) - e(N D Hf Wf) (e(v): the smallest e
- * with v < 2^e), and the pillar sums are exact integer sums, so results are
+ * with v < 2^e) clamped to [-126, 127] (max|depth| max|feat| must be finite in
+ * fp32), and the pillar sums are exact integer sums, so results are
  * reproducible bit for bit whatever the order of the points; the absolute
  * error of a pillar is at most (its points) * 2^-(s+1) plus the final
  * rounding to fp32.  Returns BEV_OK, BEV_ERR_INVALID_ARG, BEV_ERR_UNSUPPORTED,
