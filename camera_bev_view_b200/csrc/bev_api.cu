@@ -263,6 +263,18 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
     a.tile_j = bev::kTileJ;
     a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
     a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
+    // Few tiles (under two waves of resident CTAs): the launch would end on a
+    // short wave of the heaviest, near-rig tiles, so split every tile's
+    // cameras over two CTAs that add into the zeroed output.
+    int sms;
+    if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
+    const long long ctas = (long long)a.tiles_i * a.tiles_j * B * slices;
+    a.cam_split = ctas < 2LL * sms * bev::kCtasPerSm;
+    if (a.cam_split) {
+        if ((st = cuda_status(cudaMemsetAsync(out, 0, (size_t)B * C * grid->X * grid->Y * sizeof(float), s))) !=
+            BEV_OK)
+            return st;
+    }
     return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, V, slices, s));
 }
 

@@ -17,6 +17,11 @@
 
 namespace bev {
 
+__device__ __forceinline__ void red_add_f32x4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 // Channel chunks of 16 bytes: 4 fp32 or 8 bf16 channels, accumulated in fp32
 // pairs with the packed fp32x2 FMA of sm_100 (each half is an IEEE fma.rn).
 template <bool BF16>
@@ -156,6 +161,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
     setup_tile(a, s, b, ti0, tj0);
     const int nA = s.act[32];
+    // camera split: half h of the tile gathers the active cameras aa with
+    // aa % 2 == h (both halves count over all of them); a tile seen by one
+    // camera is left to half 0
+    const int half = a.cam_split ? (int)(blockIdx.x & 1) : 0;
+    const int cstep = a.cam_split ? 2 : 1;
+    if (half == 1 && nA < 2) return;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / L, ql = lane - sub * L;
@@ -164,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
     const uint4* feat = reinterpret_cast<const uint4*>(a.feat) + chunk0 + ql + (size_t)b * a.N * texels * a.Qtot;
     const int i = ti0 + warp;
     const float x = voxel_centre(g.xmin, i, g.dx);
-    const bool write_count = a.count != nullptr && blockIdx.z == 0;
+    const bool write_count = a.count != nullptr && blockIdx.z == 0 && half == 0;
     const int zn = min(kZPerLaneMax, (g.Z + L - 1) / L);  // bins per lane per chunk
 
     float2 acc[CG][V][P];
@@ -200,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
                 if (write_count && t < zn && in_grid && z < g.Z)
                     a.count[(((size_t)b * g.X + i) * g.Y + j) * g.Z + z] = (uint8_t)cnt[t];
             }
-            for (int aa = 0; aa < nA; ++aa) {
+            for (int aa = half; aa < nA; aa += cstep) {
                 const Items it = aa == 0 ? keep0
                                : aa == 1 ? keep1
                                          : project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
@@ -242,21 +253,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
         }
     }
     __syncwarp();
+    // With a camera split the two halves of a tile add their partial sums
+    // into the zeroed output: two additions onto 0 give the same bits in
+    // either order.
     if (i < g.X) {
         if ((g.Y & 3) == 0) {  // rows of 8 cells start 16-byte aligned: two float4 per channel
             for (int t = lane; t < c_real * 2; t += 32) {
                 const int c = t >> 1, jc = (t & 1) * 4;
                 if (tj0 + jc < g.Y) {
                     const float* sp = stage + c * kStageStride + jc;
-                    *reinterpret_cast<float4*>(a.out + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0 + jc) =
-                        make_float4(sp[0], sp[1], sp[2], sp[3]);
+                    float* op = a.out + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0 + jc;
+                    if (a.cam_split)
+                        red_add_f32x4(op, sp[0], sp[1], sp[2], sp[3]);
+                    else
+                        *reinterpret_cast<float4*>(op) = make_float4(sp[0], sp[1], sp[2], sp[3]);
                 }
             }
         } else {
             for (int t = lane; t < c_real * kCellsPerWarp; t += 32) {
                 const int c = t >> 3, jc = t & 7;
-                if (tj0 + jc < g.Y)
-                    a.out[(((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0 + jc] = stage[c * kStageStride + jc];
+                if (tj0 + jc < g.Y) {
+                    float* op = a.out + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0 + jc;
+                    if (a.cam_split)
+                        atomicAdd(op, stage[c * kStageStride + jc]);
+                    else
+                        *op = stage[c * kStageStride + jc];
+                }
             }
         }
     }
@@ -313,7 +335,7 @@ static cudaError_t launch_fwd_bf16(const SampleArgs& a, int V, dim3 grid, size_t
 
 cudaError_t bev_launch_forward(const bev::SampleArgs& a, bool bf16, int V, int slices,
                                cudaStream_t stream) {
-    const dim3 grid(a.tiles_i * a.tiles_j, a.B, slices);
+    const dim3 grid(a.tiles_i * a.tiles_j * (a.cam_split ? 2 : 1), a.B, slices);
     const size_t smem = bev::sample_smem_bytes(a.N);
     return bf16 ? bev::launch_fwd_bf16(a, V, grid, smem, stream)
                 : bev::launch_fwd_f32(a, V, grid, smem, stream);

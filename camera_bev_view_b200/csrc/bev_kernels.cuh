@@ -57,6 +57,7 @@ struct SampleArgs {
     int L;                  // lanes per cell (4, 8, 16 or 32)
     int tile_j;             // cells per tile row: kTileJ (forward) or a multiple of 32 / L (backward)
     int tiles_i, tiles_j;   // tiles along X and Y
+    int cam_split;          // forward: two CTAs per tile, each gathering every other camera
 };
 
 // Bytes of dynamic shared memory of one CTA (see carve_smem).

@@ -43,7 +43,8 @@ __device__ __forceinline__ CtaSmem carve_smem(unsigned char* smem, int N) {
     return s;
 }
 
-// Tile of this CTA.  Tiles are issued in rings of increasing Chebyshev
+// Tile of this CTA (with a camera split, CTAs 2t and 2t + 1 share tile t).
+// Tiles are issued in rings of increasing Chebyshev
 // distance from the centre tile of the grid: for rigs mounted near the grid
 // centre the nearest voxels see the most texels, so the heaviest tiles start
 // first and the light outer ring fills the tail of the launch.  Any order
@@ -62,7 +63,7 @@ __device__ inline void tile_origin(const SampleArgs& a, int* slot, int& ti0, int
         };
         // ring r of rank k: the smallest r with area(r) > k (binary search)
         int lo = 0, hi = max(max(ci, Ti - 1 - ci), max(cj, Tj - 1 - cj));
-        const int rank = blockIdx.x;
+        const int rank = a.cam_split ? blockIdx.x >> 1 : blockIdx.x;
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
             if (area(mid) > rank) hi = mid; else lo = mid + 1;
