@@ -35,16 +35,39 @@ __device__ __forceinline__ void scatter_texel(float* p, const float (&d)[V][4], 
             red_add_v4(p + v * L * 4, w * d[v][0], w * d[v][1], w * d[v][2], w * d[v][3]);
 }
 
+// Merged path: walk the cell's patch two rows by two columns per step, as
+// the forward does; the trip counts are the warp's largest patch and other
+// cells are predicated off past their own.  Texels with weight 0 get no
+// reduction.
 template <int L, int V>
 __device__ __forceinline__ void scatter_patch(const float (&d)[V][4], const float* pf, const Patch& pt, float* Gn,
                                               int Wf, int tstride, int ql, int nchunks) {
     const int h = pt.h, w = pt.w;
-    const float* pw = pf + pt.off;
-    float* grow = Gn + ((size_t)pt.y0 * Wf + pt.x0) * tstride;
-    for (int r = 0; r < h; ++r, grow += (size_t)Wf * tstride, pw += w) {
-        for (int cc = 0; cc < w; ++cc) {
-            const float wt = pw[cc];
-            if (wt != 0.0f) scatter_texel<L, V>(grow + (size_t)cc * tstride, d, wt, ql, nchunks);
+    const int hmax = __reduce_max_sync(0xffffffffu, h);
+    const int wmax = __reduce_max_sync(0xffffffffu, w);
+    const size_t rstride = (size_t)Wf * tstride;
+    bool lane_ok[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) lane_ok[v] = ql + v * L < nchunks;
+    for (int c0 = 0; c0 < wmax; c0 += 2) {
+        const bool c0in = c0 < w, c1in = c0 + 1 < w;
+        const float* pw = pf + pt.off + c0;
+        float* rp = Gn + ((size_t)pt.y0 * Wf + pt.x0 + c0) * tstride;
+        for (int r0 = 0; r0 < hmax; r0 += 2, pw += 2 * w, rp += 2 * rstride) {
+            const bool r0in = r0 < h, r1in = r0 + 1 < h;
+            const bool in[4] = {r0in && c0in, r0in && c1in, r1in && c0in, r1in && c1in};
+            const float wt[4] = {in[0] ? pw[0] : 0.0f, in[1] ? pw[1] : 0.0f, in[2] ? pw[w] : 0.0f,
+                                 in[3] ? pw[w + 1] : 0.0f};
+            float* pp[4] = {rp, rp + tstride, rp + rstride, rp + rstride + tstride};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (wt[u] == 0.0f) continue;
+#pragma unroll
+                for (int v = 0; v < V; ++v)
+                    if (lane_ok[v])
+                        red_add_v4(pp[u] + v * L * 4, wt[u] * d[v][0], wt[u] * d[v][1], wt[u] * d[v][2],
+                                   wt[u] * d[v][3]);
+            }
         }
     }
 }
