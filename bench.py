@@ -63,6 +63,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--op", choices=["vt", "deform", "lss"], default="vt")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the hot-L2 and back-to-back forward timings (for launch-list profiling)")
     args = ap.parse_args()
     if args.op == "deform" and args.workload == "nuscenes":
         args.workload = "deform"
@@ -344,34 +346,36 @@ def run_ours(args):
 
     # forward with a hot L2 (no flush), and as one CUDA graph of 100
     # back-to-back launches (launch overhead amortised), per launch
-    with torch.cuda.stream(stream):
-        hot = []
-        for k in range(60):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            graphs["forward"].replay()
-            e1.record(stream)
-            e1.synchronize()
-            if k >= 10:
-                hot.append(e0.elapsed_time(e1))
-        g100 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g100, stream=stream):
-            for _ in range(100):
-                stages["forward"]()
-        g100.replay()
-        reps = []
-        for k in range(8):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+    fwd_hot_ms = fwd_b2b_ms = float("nan")
+    if not args.no_extras:
+        with torch.cuda.stream(stream):
+            hot = []
+            for k in range(60):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graphs["forward"].replay()
+                e1.record(stream)
+                e1.synchronize()
+                if k >= 10:
+                    hot.append(e0.elapsed_time(e1))
+            g100 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g100, stream=stream):
+                for _ in range(100):
+                    stages["forward"]()
             g100.replay()
-            e1.record(stream)
-            e1.synchronize()
-            if k >= 2:
-                reps.append(e0.elapsed_time(e1) / 100)
-        g100.reset()
-    fwd_hot_ms = statistics.median(hot)
-    fwd_b2b_ms = statistics.median(reps)
+            reps = []
+            for k in range(8):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g100.replay()
+                e1.record(stream)
+                e1.synchronize()
+                if k >= 2:
+                    reps.append(e0.elapsed_time(e1) / 100)
+            g100.reset()
+        fwd_hot_ms = statistics.median(hot)
+        fwd_b2b_ms = statistics.median(reps)
     ms = max_over_ranks(sum(stage_ms.values()), world, dev)
     elems = B * C * X * Y
     value = whole_job_rate(elems, world, ms)
