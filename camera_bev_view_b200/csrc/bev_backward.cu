@@ -75,12 +75,12 @@ __device__ __forceinline__ void scatter_patch(const float (&d)[V][4], const floa
 // Fallback for cells whose patches did not fit: each valid bin's four
 // corners, broadcast from the lane that projected it.  Called by the whole
 // warp.
-template <int L, int V>
-__device__ __forceinline__ void scatter_direct(const float (&d)[V][4], const Items& it,
-                                               const float (&rc)[kZPerLaneMax], int zn, bool mine, int sub,
+template <int L, int V, int ZN>
+__device__ __forceinline__ void scatter_direct(const float (&d)[V][4], const Items<ZN>& it,
+                                               const float (&rc)[ZN], int zn, bool mine, int sub,
                                                float* Gn, int Hf, int Wf, int tstride, int ql, int nchunks) {
 #pragma unroll
-    for (int t = 0; t < kZPerLaneMax; ++t) {
+    for (int t = 0; t < ZN; ++t) {
         if (t >= zn) break;
         for (int zz = 0; zz < L; ++zz) {
             const int src = sub * L + zz;
@@ -127,7 +127,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(c
     const int tstride = a.Qtot * 4;  // floats per texel in the gradient buffer
     float* grad = a.dfeat + (size_t)(chunk0 + ql) * 4 + (size_t)b * a.N * texels * tstride;
     const float x = voxel_centre(g.xmin, i, g.dx);
-    const int zn = min(kZPerLaneMax, (g.Z + L - 1) / L);
+    constexpr int ZN = kZPerLaneBwd;
+    const int zn = min(ZN, (g.Z + L - 1) / L);
     const size_t cstride = (size_t)g.X * g.Y;
 
     // G cells at a time along the warp's row of tile_j cells
@@ -149,30 +150,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(c
         for (int z0 = 0; z0 < g.Z; z0 += L * zn) {
             // valid cameras per bin of this lane, over all active cameras; the
             // projections of the first two cameras are kept for the merge pass
-            int cnt[kZPerLaneMax] = {0, 0, 0, 0};
-            Items keep0, keep1;
+            int cnt[ZN] = {};
+            Items<ZN> keep0, keep1;
             for (int aa = 0; aa < nA; ++aa) {
-                const Items it = project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
+                const Items<ZN> it = project_items<L, ZN>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
                 if (aa == 0) keep0 = it;
                 if (aa == 1) keep1 = it;
 #pragma unroll
-                for (int t = 0; t < kZPerLaneMax; ++t) cnt[t] += (it.ok >> t) & 1u;
+                for (int t = 0; t < ZN; ++t) cnt[t] += (it.ok >> t) & 1u;
             }
-            float rc[kZPerLaneMax];
+            float rc[ZN];
 #pragma unroll
-            for (int t = 0; t < kZPerLaneMax; ++t) rc[t] = cnt[t] > 0 ? __frcp_rn((float)cnt[t]) : 0.0f;
+            for (int t = 0; t < ZN; ++t) rc[t] = cnt[t] > 0 ? __frcp_rn((float)cnt[t]) : 0.0f;
             for (int aa = 0; aa < nA; ++aa) {
-                const Items it = aa == 0 ? keep0
-                               : aa == 1 ? keep1
-                                         : project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
+                const Items<ZN> it = aa == 0 ? keep0
+                                   : aa == 1 ? keep1
+                                             : project_items<L, ZN>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
                 float* Gn = grad + (size_t)s.act[aa] * texels * tstride;
                 // always merged: a merged texel costs one reduction per chunk
                 // instead of one per bin that touches it
-                Patch pt = patch_box<L>(it, zn, g.Hf, g.Wf);
-                merge_patches<L>(pt, it, rc, zn, sub, ql, g.Hf, g.Wf, region);
+                Patch pt = patch_box<L, ZN>(it, zn, g.Hf, g.Wf);
+                merge_patches<L, ZN>(pt, it, rc, zn, sub, ql, g.Hf, g.Wf, region);
                 scatter_patch<L, V>(d, reinterpret_cast<const float*>(region), pt, Gn, g.Wf, tstride, ql, nchunks);
                 if (__any_sync(0xffffffffu, pt.overflow))
-                    scatter_direct<L, V>(d, it, rc, zn, pt.overflow, sub, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
+                    scatter_direct<L, V, ZN>(d, it, rc, zn, pt.overflow, sub, Gn, g.Hf, g.Wf, tstride, ql, nchunks);
                 __syncwarp();  // the region is rebuilt for the next camera
             }
         }

@@ -105,8 +105,8 @@ __device__ __forceinline__ void gather_patch(Acc<BF16, V>& acc, const float* pf,
 // corners and accumulate.  Branch-free: corners outside the map, invalid bins
 // and cells with mine == false carry weight 0 and their loads are predicated
 // off.  Called by the whole warp.
-template <bool BF16, int L, int V>
-__device__ __forceinline__ void gather_bins(Acc<BF16, V>& acc, const Items& it, const float (&rc)[kZPerLaneMax],
+template <bool BF16, int L, int V, int ZN>
+__device__ __forceinline__ void gather_bins(Acc<BF16, V>& acc, const Items<ZN>& it, const float (&rc)[ZN],
                                             int zn, bool mine, int sub, const uint4* Fn, int Hf, int Wf, int Qtot,
                                             int ql, int nchunks) {
     bool lane_ok[V];
@@ -114,7 +114,7 @@ __device__ __forceinline__ void gather_bins(Acc<BF16, V>& acc, const Items& it, 
     for (int v = 0; v < V; ++v) lane_ok[v] = ql + v * L < nchunks;
     const ptrdiff_t rs = (ptrdiff_t)Wf * Qtot;
 #pragma unroll
-    for (int t = 0; t < kZPerLaneMax; ++t) {
+    for (int t = 0; t < ZN; ++t) {
         if (t >= zn) break;
         const float rct = (mine && (it.ok >> t & 1u)) ? rc[t] : 0.0f;
 #pragma unroll 2
@@ -176,7 +176,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
     const int i = ti0 + warp;
     const float x = voxel_centre(g.xmin, i, g.dx);
     const bool write_count = a.count != nullptr && blockIdx.z == 0 && half == 0;
-    const int zn = min(kZPerLaneMax, (g.Z + L - 1) / L);  // bins per lane per chunk
+    constexpr int ZN = kZPerLaneFwd;
+    const int zn = min(ZN, (g.Z + L - 1) / L);  // bins per lane per chunk
 
     float2 acc[CG][V][P];
 #pragma unroll
@@ -194,39 +195,39 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(co
         for (int z0 = 0; z0 < g.Z; z0 += L * zn) {
             // valid cameras per bin of this lane, over all active cameras; the
             // projections of the first two cameras are kept for the merge pass
-            int cnt[kZPerLaneMax] = {0, 0, 0, 0};
-            Items keep0, keep1;
+            int cnt[ZN] = {};
+            Items<ZN> keep0, keep1;
             for (int aa = 0; aa < nA; ++aa) {
-                const Items it = project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
+                const Items<ZN> it = project_items<L, ZN>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
                 if (aa == 0) keep0 = it;
                 if (aa == 1) keep1 = it;
 #pragma unroll
-                for (int t = 0; t < kZPerLaneMax; ++t) cnt[t] += (it.ok >> t) & 1u;
+                for (int t = 0; t < ZN; ++t) cnt[t] += (it.ok >> t) & 1u;
             }
-            float rc[kZPerLaneMax];
+            float rc[ZN];
 #pragma unroll
-            for (int t = 0; t < kZPerLaneMax; ++t) {
+            for (int t = 0; t < ZN; ++t) {
                 rc[t] = cnt[t] > 0 ? __frcp_rn((float)cnt[t]) : 0.0f;
                 const int z = z0 + ql + L * t;
                 if (write_count && t < zn && in_grid && z < g.Z)
                     a.count[(((size_t)b * g.X + i) * g.Y + j) * g.Z + z] = (uint8_t)cnt[t];
             }
             for (int aa = half; aa < nA; aa += cstep) {
-                const Items it = aa == 0 ? keep0
-                               : aa == 1 ? keep1
-                                         : project_items<L>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
+                const Items<ZN> it = aa == 0 ? keep0
+                                   : aa == 1 ? keep1
+                                             : project_items<L, ZN>(s.cams + s.act[aa] * kCamFloats, x, y, in_grid, z0, zn, ql, g);
                 const uint4* Fn = feat + (size_t)s.act[aa] * texels * a.Qtot;
-                Patch pt = patch_box<L>(it, zn, g.Hf, g.Wf);
+                Patch pt = patch_box<L, ZN>(it, zn, g.Hf, g.Wf);
                 if (merge_pays<L>(pt, zn, kMergeStepsFwd)) {
-                    merge_patches<L>(pt, it, rc, zn, sub, ql, g.Hf, g.Wf, region);
+                    merge_patches<L, ZN>(pt, it, rc, zn, sub, ql, g.Hf, g.Wf, region);
                     gather_patch<BF16, L, V>(acc[q], reinterpret_cast<const float*>(region), pt, Fn, g.Wf, a.Qtot,
                                              ql, nchunks);
                     if (__any_sync(0xffffffffu, pt.overflow))
-                        gather_bins<BF16, L, V>(acc[q], it, rc, zn, pt.overflow, sub, Fn, g.Hf, g.Wf, a.Qtot, ql,
+                        gather_bins<BF16, L, V, ZN>(acc[q], it, rc, zn, pt.overflow, sub, Fn, g.Hf, g.Wf, a.Qtot, ql,
                                                 nchunks);
                     __syncwarp();  // the region is rebuilt for the next camera
                 } else {
-                    gather_bins<BF16, L, V>(acc[q], it, rc, zn, true, sub, Fn, g.Hf, g.Wf, a.Qtot, ql, nchunks);
+                    gather_bins<BF16, L, V, ZN>(acc[q], it, rc, zn, true, sub, Fn, g.Hf, g.Wf, a.Qtot, ql, nchunks);
                 }
             }
         }

@@ -19,8 +19,14 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCellsPerWarp = kTile / kWarps;
 static_assert(kCellsPerWarp == kTileJ && kWarps == kTileI, "one warp per tile row");
-// Height bins a lane projects per chunk (chunk = lanes per cell * this).
-constexpr int kZPerLaneMax = 4;
+// Height bins a lane projects per chunk (chunk = lanes per cell * this).  The
+// projections of a chunk stay in registers (two of them cached per cell
+// group), so the forward, whose accumulators already fill the register file,
+// takes two; the backward, which holds dout instead, takes four.  Taller
+// grids take more chunks.
+constexpr int kZPerLaneFwd = 2;
+constexpr int kZPerLaneBwd = 4;
+constexpr int kZPerLaneMax = kZPerLaneBwd;
 // Merged-weight entries of one warp for one (camera, height chunk): the
 // patches of the cells the warp works on at once.  Each entry is an exact
 // fixed-point sum split over two 32-bit words (see merge_patches).

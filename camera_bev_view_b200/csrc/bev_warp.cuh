@@ -187,21 +187,23 @@ constexpr float kTwoM20 = 9.5367431640625e-07f;
 constexpr float kTwo40 = 1099511627776.0f;
 constexpr float kTwoM40 = 9.094947017729282379150390625e-13f;
 
-// One cell group's projections for one camera in one height chunk.
+// One cell group's projections for one camera in one height chunk: ZN bins
+// per lane.
+template <int ZN>
 struct Items {
-    float fx[kZPerLaneMax], fy[kZPerLaneMax];
+    float fx[ZN], fy[ZN];
     unsigned ok;  // bit t: item t is a valid voxel
 };
 
 // Project this lane's bins z = z0 + ql + L t (t < zn) of voxel column (x, y)
 // through one camera.
-template <int L>
-__device__ __forceinline__ Items project_items(const float* cam, float x, float y, bool in_grid, int z0,
+template <int L, int ZN>
+__device__ __forceinline__ Items<ZN> project_items(const float* cam, float x, float y, bool in_grid, int z0,
                                                int zn, int ql, const GeoParams& g) {
-    Items it;
+    Items<ZN> it;
     it.ok = 0;
 #pragma unroll
-    for (int t = 0; t < kZPerLaneMax; ++t) {
+    for (int t = 0; t < ZN; ++t) {
         it.fx[t] = 0.0f;
         it.fy[t] = 0.0f;
         const int z = z0 + ql + L * t;
@@ -228,13 +230,13 @@ struct Patch {
 // Box of texels the valid voxels of this lane's cell touch through one
 // camera (uniform over the cell's lanes); h == 0 when the cell has no valid
 // voxel.  `off` and `overflow` are set by merge_patches.
-template <int L>
-__device__ __forceinline__ Patch patch_box(const Items& it, int zn, int Hf, int Wf) {
+template <int L, int ZN>
+__device__ __forceinline__ Patch patch_box(const Items<ZN>& it, int zn, int Hf, int Wf) {
     // lo = (ylo, xlo), hi = (yhi + 1, xhi + 1) as 16-bit fields (dimensions
     // are below 2^15); an empty cell keeps lo = (0xffff, 0xffff), hi = 0
     unsigned lo = 0xffffffffu, hi = 0u;
 #pragma unroll
-    for (int t = 0; t < kZPerLaneMax; ++t) {
+    for (int t = 0; t < ZN; ++t) {
         if (t < zn && (it.ok >> t & 1u)) {
             const int x0 = (int)floorf(it.fx[t]), y0 = (int)floorf(it.fy[t]);
             const unsigned l = ((unsigned)max(y0, 0) << 16) | (unsigned)max(x0, 0);
@@ -272,8 +274,8 @@ __device__ __forceinline__ bool merge_pays(const Patch& p, int zn, int merge_ste
 // t.  Cells whose patches do not fit the region get h = 0 and `overflow`.
 // Ends with the patch values readable by all lanes of the warp (fp32 at words
 // [off, off + h * w) of `region`).
-template <int L>
-__device__ __forceinline__ void merge_patches(Patch& p, const Items& it, const float (&rc)[kZPerLaneMax], int zn,
+template <int L, int ZN>
+__device__ __forceinline__ void merge_patches(Patch& p, const Items<ZN>& it, const float (&rc)[ZN], int zn,
                                               int sub, int ql, int Hf, int Wf, int* region) {
     int total;
     p.off = group_prefix<L>(p.h * p.w, sub, &total);
@@ -289,7 +291,7 @@ __device__ __forceinline__ void merge_patches(Patch& p, const Items& it, const f
     __syncwarp();
     if (n > 0) {
 #pragma unroll
-        for (int t = 0; t < kZPerLaneMax; ++t) {
+        for (int t = 0; t < ZN; ++t) {
             if (t < zn && (it.ok >> t & 1u)) {
                 const Corners c = bilinear_corners(it.fx[t], it.fy[t]);
                 const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
