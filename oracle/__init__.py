@@ -9,7 +9,9 @@ loop nest (FlashBEV reading notes, "Method" items 1 and 4): per height bin the
 mean over valid cameras of the bilinear samples, summed over height.  See the
 header comment of ``bev_oracle.c`` for every reading it takes.
 
-Also the lift-splat BEV pooling of the LSS tutorial ("Lift", "Splat"):
+Also the multi-scale form (``ms_forward`` / ``ms_backward``: several
+feature-pyramid levels sampled through one geometry and summed inside the
+valid mean; pins in ``tests/test_oracle_multiscale.py``), the lift-splat BEV pooling of the LSS tutorial ("Lift", "Splat"):
 ``lss_forward`` / ``lss_backward`` (pins in ``tests/test_oracle_lss.py``), and
 the deformable aggregation of the SparseDriveV2 notes ("Deformable
 Aggregation", steps 1-3): ``deform_forward`` / ``deform_backward`` (pins in
@@ -62,6 +64,10 @@ def _load():
         lib.oracle_forward.restype = None
         lib.oracle_backward.argtypes = [P, I, I, I, I, I, P, P, I, I, I, I, I, P, P, P, P, I]
         lib.oracle_backward.restype = None
+        lib.oracle_ms_forward.argtypes = [P, I, P, P, I, I, I, P, P, I, I, I, I, I, P, P, P, P, P, I]
+        lib.oracle_ms_forward.restype = None
+        lib.oracle_ms_backward.argtypes = [P, I, P, P, I, I, I, P, P, I, I, I, I, I, P, P, P, P, I]
+        lib.oracle_ms_backward.restype = None
         lib.oracle_deform_forward.argtypes = [P, I, I, I, I, I, P, P, I, I, P, P, P, I, I, P, P, I]
         lib.oracle_deform_forward.restype = None
         lib.oracle_deform_backward.argtypes = [P, P, I, I, I, I, I, P, P, I, I, P, P, P, I, I,
@@ -161,6 +167,48 @@ def backward(dout, N, Hf, Wf, K, E, img_h, img_w, grid: Grid, threads: int = 0):
     _load().oracle_backward(_ptr(G), B, N, C, Hf, Wf, _ptr(Kc), _ptr(Ec), img_h, img_w,
                             grid.X, grid.Y, grid.Z, _ptr(grid.lo), _ptr(grid.cell),
                             _ptr(dF), _ptr(dB), threads)
+    return dF, dB
+
+
+def _ptr_array(arrays):
+    return (ctypes.c_void_p * len(arrays))(*[a.ctypes.data for a in arrays])
+
+
+def ms_forward(levels, K, E, img_h, img_w, grid: Grid, threads: int = 0):
+    """Multi-scale forward: ``levels`` = list of [B,N,C,H_l,W_l] feature maps
+    (fp32 or bf16, widened exactly).  Returns (out, bound, count) as
+    ``forward`` does; the levels' samples are summed inside the valid mean."""
+    Fs = [_np(f, np.float64) for f in levels]
+    B, N, C = Fs[0].shape[:3]
+    assert all(f.shape[:3] == (B, N, C) for f in Fs)
+    H = np.array([f.shape[3] for f in Fs], dtype=np.int32)
+    W = np.array([f.shape[4] for f in Fs], dtype=np.int32)
+    Kc = _np(K, np.float32).reshape(B, N, 3, 3)
+    Ec = _np(E, np.float32).reshape(B, N, 4, 4)
+    out = np.zeros((B, C, grid.X, grid.Y), dtype=np.float64)
+    bound = np.zeros_like(out)
+    count = np.zeros((B, grid.X, grid.Y, grid.Z), dtype=np.int32)
+    _load().oracle_ms_forward(_ptr_array(Fs), len(Fs), _ptr(H), _ptr(W), B, N, C, _ptr(Kc), _ptr(Ec),
+                              img_h, img_w, grid.X, grid.Y, grid.Z, _ptr(grid.lo), _ptr(grid.cell),
+                              _ptr(out), _ptr(bound), _ptr(count), threads)
+    return out, bound, count
+
+
+def ms_backward(dout, N, sizes, K, E, img_h, img_w, grid: Grid, threads: int = 0):
+    """Multi-scale backward: ``sizes`` = [(H_l, W_l), ...].  Returns
+    (list of dF_l [B,N,C,H_l,W_l] f64, list of bounds)."""
+    G = _np(dout, np.float64)
+    B, C, X, Y = G.shape
+    assert (X, Y) == (grid.X, grid.Y)
+    H = np.array([h for h, _ in sizes], dtype=np.int32)
+    W = np.array([w for _, w in sizes], dtype=np.int32)
+    Kc = _np(K, np.float32).reshape(B, N, 3, 3)
+    Ec = _np(E, np.float32).reshape(B, N, 4, 4)
+    dF = [np.zeros((B, N, C, h, w), dtype=np.float64) for h, w in sizes]
+    dB = [np.zeros_like(d) for d in dF]
+    _load().oracle_ms_backward(_ptr(G), len(sizes), _ptr(H), _ptr(W), B, N, C, _ptr(Kc), _ptr(Ec),
+                               img_h, img_w, grid.X, grid.Y, grid.Z, _ptr(grid.lo), _ptr(grid.cell),
+                               _ptr_array(dF), _ptr_array(dB), threads)
     return dF, dB
 
 

@@ -258,6 +258,148 @@ void oracle_backward(const double* dout, int B, int N, int C, int Hf, int Wf,
 }
 
 /* ------------------------------------------------------------------------
+ * Multi-scale dense Sampling-VT (FlashBEV reading notes, "Takeaway" 4:
+ * multi-scale fused view transformation; SparseDriveV2 notes, "Image
+ * Encoder": an FPN gives each camera feature maps P_l at several resolutions
+ * with a common channel count).  The geometry of a voxel is that of the
+ * single-level operator above: one projection (u, v) in image pixels, one
+ * validity test, one count per height bin.  Each level l samples its own map
+ * at its own scale, fx_l = u * (W_l / W_img) - 0.5 (fy_l likewise), and the
+ * samples of all levels are summed inside the valid mean:
+ *
+ *   out[b,c,i,j] = sum_k [cnt_k > 0] (1 / cnt_k) sum_{n valid} sum_l bilinear(F_l[b,n,c], fx_l, fy_l)
+ *
+ * Readings (the notes name the direction only): the levels are combined by
+ * an unweighted sum, so that with one level this is the operator above; the
+ * count does not depend on the level (validity is an image-plane test); a
+ * corner outside level l's map contributes zero at that level only.
+ * ---------------------------------------------------------------------- */
+
+/* Forward.  F[l] = level l's features [B,N,C,H[l],W[l]] fp64; the rest as in
+ * oracle_forward. */
+void oracle_ms_forward(const double* const* F, int nlev, const int* H, const int* W, int B, int N, int C,
+                       const float* K, const float* E, int img_h, int img_w,
+                       int X, int Y, int Z, const float lo[3], const float cell[3],
+                       double* out, double* bound, int32_t* count, int threads)
+{
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic)
+#endif
+    for (long bi = 0; bi < (long)B * X; ++bi) {
+        int b = (int)(bi / X), i = (int)(bi % X);
+        double* acc = (double*)malloc(sizeof(double) * 4 * (size_t)C);
+        double* abs_acc = acc + C;
+        double* s = acc + 2 * C;
+        double* a = acc + 3 * C;
+        float x = centre(lo[0], i, cell[0]);
+        for (int j = 0; j < Y; ++j) {
+            float y = centre(lo[1], j, cell[1]);
+            for (int c = 0; c < C; ++c) { acc[c] = 0.0; abs_acc[c] = 0.0; }
+            for (int k = 0; k < Z; ++k) {
+                float z = centre(lo[2], k, cell[2]);
+                for (int c = 0; c < C; ++c) { s[c] = 0.0; a[c] = 0.0; }
+                int cnt = 0;
+                for (int n = 0; n < N; ++n) {
+                    const float* Kn = K + ((size_t)b * N + n) * 9;
+                    const float* En = E + ((size_t)b * N + n) * 16;
+                    float u, v, fx, fy;
+                    /* validity is the image-plane test: any level's sizes give it */
+                    if (!oracle_project(Kn, En, x, y, z, img_h, img_w, H[0], W[0], &u, &v, &fx, &fy))
+                        continue;
+                    ++cnt;
+                    for (int l = 0; l < nlev; ++l) {
+                        oracle_project(Kn, En, x, y, z, img_h, img_w, H[l], W[l], &u, &v, &fx, &fy);
+                        int ys[4], xs[4];
+                        float ws[4];
+                        corners(fx, fy, ys, xs, ws);
+                        for (int q = 0; q < 4; ++q) {
+                            if (ys[q] < 0 || ys[q] >= H[l] || xs[q] < 0 || xs[q] >= W[l]) continue;
+                            const double* Fp = F[l] + (((size_t)b * N + n) * C * H[l] + ys[q]) * W[l] + xs[q];
+                            for (int c = 0; c < C; ++c) {
+                                double term = (double)ws[q] * Fp[(size_t)c * H[l] * W[l]];
+                                s[c] += term;
+                                a[c] += fabs(term);
+                            }
+                        }
+                    }
+                }
+                count[(((size_t)b * X + i) * Y + j) * Z + k] = cnt;
+                if (cnt > 0) {
+                    for (int c = 0; c < C; ++c) {
+                        acc[c] += s[c] / cnt;
+                        abs_acc[c] += a[c] / cnt;
+                    }
+                }
+            }
+            for (int c = 0; c < C; ++c) {
+                size_t o = (((size_t)b * C + c) * X + i) * Y + j;
+                out[o] = acc[c];
+                bound[o] = abs_acc[c];
+            }
+        }
+        free(acc);
+    }
+}
+
+/* Backward: dF[l] and dbound[l] [B,N,C,H[l],W[l]] fp64 (overwritten). */
+void oracle_ms_backward(const double* dout, int nlev, const int* H, const int* W, int B, int N, int C,
+                        const float* K, const float* E, int img_h, int img_w,
+                        int X, int Y, int Z, const float lo[3], const float cell[3],
+                        double* const* dF, double* const* dbound, int threads)
+{
+    for (int l = 0; l < nlev; ++l) {
+        memset(dF[l], 0, sizeof(double) * (size_t)B * N * C * H[l] * W[l]);
+        memset(dbound[l], 0, sizeof(double) * (size_t)B * N * C * H[l] * W[l]);
+    }
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic)
+#endif
+    for (long bn = 0; bn < (long)B * N; ++bn) {
+        int b = (int)(bn / N), n = (int)(bn % N);
+        const float* Kn = K + ((size_t)b * N + n) * 9;
+        const float* En = E + ((size_t)b * N + n) * 16;
+        for (int i = 0; i < X; ++i) {
+            float x = centre(lo[0], i, cell[0]);
+            for (int j = 0; j < Y; ++j) {
+                float y = centre(lo[1], j, cell[1]);
+                for (int k = 0; k < Z; ++k) {
+                    float z = centre(lo[2], k, cell[2]);
+                    float u, v, fx, fy;
+                    int cnt = 0;
+                    for (int m = 0; m < N; ++m) {
+                        const float* Km = K + ((size_t)b * N + m) * 9;
+                        const float* Em = E + ((size_t)b * N + m) * 16;
+                        cnt += oracle_project(Km, Em, x, y, z, img_h, img_w, H[0], W[0], &u, &v, &fx, &fy);
+                    }
+                    if (!oracle_project(Kn, En, x, y, z, img_h, img_w, H[0], W[0], &u, &v, &fx, &fy))
+                        continue;
+                    for (int l = 0; l < nlev; ++l) {
+                        oracle_project(Kn, En, x, y, z, img_h, img_w, H[l], W[l], &u, &v, &fx, &fy);
+                        double* dFn = dF[l] + ((size_t)b * N + n) * C * H[l] * W[l];
+                        double* dBn = dbound[l] + ((size_t)b * N + n) * C * H[l] * W[l];
+                        int ys[4], xs[4];
+                        float ws[4];
+                        corners(fx, fy, ys, xs, ws);
+                        for (int q = 0; q < 4; ++q) {
+                            if (ys[q] < 0 || ys[q] >= H[l] || xs[q] < 0 || xs[q] >= W[l]) continue;
+                            for (int c = 0; c < C; ++c) {
+                                double g = dout[(((size_t)b * C + c) * X + i) * Y + j];
+                                double term = (double)ws[q] * g / cnt;
+                                size_t o = ((size_t)c * H[l] + ys[q]) * W[l] + xs[q];
+                                dFn[o] += term;
+                                dBn[o] += fabs(term);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------
  * Deformable aggregation (SparseDriveV2 notes, "Deformable Aggregation",
  * steps 1-3): a query with 3-D anchor a and keypoint offsets d_k samples the
  * cameras at its keypoints p_k = a + d_k (step 1), each projected as above

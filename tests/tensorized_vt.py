@@ -84,6 +84,40 @@ def tensorized_backward(dout, N, Hf, Wf, K, E, ranges, counts, img_h, img_w):
     return F.grad, amb
 
 
+def tensorized_ms_forward(levels, K, E, ranges, counts, img_h, img_w):
+    """Multi-scale form: one projection and mask, one grid_sample per level
+    (the normalised grid is the same for every level: align_corners=False
+    maps it to u * W_l / W_img - 0.5 on a map of width W_l), the levels'
+    samples summed before the masked mean over cameras.  Returns out, count,
+    ambiguous as ``tensorized_forward`` does."""
+    Fs = [torch.as_tensor(f).to(torch.float64) for f in levels]
+    B, N, C = Fs[0].shape[:3]
+    X, Y, Z = counts
+    u, v, depth, mask = project_all(K, E, ranges, counts, img_h, img_w)
+    grid = torch.stack([2.0 * u / img_w - 1.0, 2.0 * v / img_h - 1.0], dim=-1)
+    grid = torch.where(mask[..., None], grid, torch.zeros_like(grid)).reshape(B * N, X * Y * Z, 1, 2)
+    total = torch.zeros((B, N, C, X, Y, Z), dtype=torch.float64)
+    for F in Fs:
+        Hl, Wl = F.shape[3:]
+        s = Fn.grid_sample(F.reshape(B * N, C, Hl, Wl), grid, mode="bilinear", padding_mode="zeros",
+                           align_corners=False)
+        total = total + s.reshape(B, N, C, X, Y, Z)
+    total = total * mask[:, :, None].to(torch.float64)
+    count = mask.sum(dim=1)
+    out = (total.sum(dim=1) / count.clamp(min=1)[:, None].to(torch.float64)).sum(dim=-1)
+    return out, count, ambiguous(u, v, depth, img_h, img_w).any(dim=1)
+
+
+def tensorized_ms_backward(dout, N, sizes, K, E, ranges, counts, img_h, img_w):
+    """dL/dF_l of every level by autograd through the multi-scale form."""
+    dout = torch.as_tensor(dout, dtype=torch.float64)
+    B, C = dout.shape[:2]
+    Fs = [torch.zeros((B, N, C, h, w), dtype=torch.float64, requires_grad=True) for h, w in sizes]
+    out, _, amb = tensorized_ms_forward(Fs, K, E, ranges, counts, img_h, img_w)
+    (out * dout).sum().backward()
+    return [F.grad for F in Fs], amb
+
+
 # --------------------------------------------------------------------------
 # Deformable aggregation (SparseDriveV2 notes, "Deformable Aggregation"
 # steps 1-3), materialised: every (b, n, q, k) keypoint projected in float64,
