@@ -26,6 +26,11 @@ with "impl": "reference".
 "Splat"): one step = forward + backward (depth and feature gradients) of the
 ``lss`` workload (6 cameras, 8x22 features, 41 depth bins, C64, 200x200).
 
+--op ms measures the multi-scale form (FlashBEV reading notes, "Takeaway" 4):
+one step = channels-last copies of four FPN levels (64x176 .. 8x22 of a
+256x704 image), the fused multi-scale forward and every level's feature
+gradient, on a 200x200x8 grid (``ms`` workload).
+
 --op deform measures the deformable aggregation instead (SparseDriveV2 notes,
 "Deformable Aggregation"): one step = forward + backward (feature, weight and
 keypoint-offset gradients) over the queries of the ``deform`` workload (900
@@ -62,7 +67,7 @@ def parse_args():
     ap.add_argument("--workload", default="nuscenes")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--op", choices=["vt", "deform", "lss"], default="vt")
+    ap.add_argument("--op", choices=["vt", "deform", "lss", "ms"], default="vt")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the hot-L2 and back-to-back forward timings (for launch-list profiling)")
     args = ap.parse_args()
@@ -70,6 +75,8 @@ def parse_args():
         args.workload = "deform"
     if args.op == "lss" and args.workload == "nuscenes":
         args.workload = "lss"
+    if args.op == "ms" and args.workload == "nuscenes":
+        args.workload = "ms"
     return args
 
 
@@ -94,8 +101,14 @@ def hbm_peak():
 
 
 KERNEL_SOURCES = {
-    "sample_forward_kernel": ["bev_forward.cu", "bev_warp.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
-    "sample_backward_kernel": ["bev_backward.cu", "bev_warp.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
+    "sample_forward_kernel": ["bev_forward.cu", "bev_forward.cuh", "bev_warp.cuh", "bev_kernels.cuh",
+                              "bev_geometry.cuh"],
+    "sample_backward_kernel": ["bev_backward.cu", "bev_backward.cuh", "bev_warp.cuh", "bev_kernels.cuh",
+                               "bev_geometry.cuh"],
+    "sample_forward_ms_kernel": ["bev_forward_ms.cu", "bev_forward.cuh", "bev_warp.cuh", "bev_kernels.cuh",
+                                 "bev_geometry.cuh"],
+    "sample_backward_ms_kernel": ["bev_backward_ms.cu", "bev_backward.cuh", "bev_warp.cuh", "bev_kernels.cuh",
+                                  "bev_geometry.cuh"],
     "deform_forward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
     "deform_backward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
     "lss_forward_kernel": ["bev_lss.cu", "bev_lss.cuh"],
@@ -649,6 +662,167 @@ def run_deform(args):
     print(json.dumps(line), flush=True)
 
 
+MS_METRIC = "multi-scale BEV output elements/s (B·C·X·Y) and achieved HBM GB/s vs roofline, 1×B200"
+
+
+def ms_oracle_step(w, threads):
+    """One oracle forward + backward of the multi-scale operator over the
+    whole workload (same seeded inputs); returns seconds."""
+    import oracle
+    from camera_bev_view_b200 import inputs as I
+    Fs = I.make_ms_features(w)
+    K, E = I.make_rigs(w)
+    g = I.make_dout(w)
+    grid = oracle.Grid(w.ranges, w.res)
+    t0 = time.perf_counter()
+    oracle.ms_forward(Fs, K, E, w.img_h, w.img_w, grid, threads=threads)
+    oracle.ms_backward(g, w.N, w.levels, K, E, w.img_h, w.img_w, grid, threads=threads)
+    return time.perf_counter() - t0
+
+
+def run_ms(args):
+    import torch
+
+    from camera_bev_view_b200 import inputs as I
+    from camera_bev_view_b200 import ops
+
+    rank, world, local = dist_env()
+    w = I.MS_WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        threads = cpu_cores()
+        for _ in range(args.warmup):
+            ms_oracle_step(w, threads)
+        times = [ms_oracle_step(w, threads) for _ in range(args.steps)]
+        value = w.out_elems * len(times) / sum(times)
+        line = {"impl": "reference", "metric": MS_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded N(0,1) pyramid levels, 6-camera rig)",
+                "config": {"workload": w.name},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                 "sample": "whole workload, forward + backward, per step"},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    Fs = [f.to(dev) for f in I.make_ms_features(w, shard=rank)]
+    K_h, E_h = I.make_rigs(w, shard=rank)
+    K, E = K_h.to(dev), E_h.to(dev)
+    g = I.make_dout(w, shard=rank).to(dev)
+    B, N, C = Fs[0].shape[:3]
+    sizes = [tuple(f.shape[3:5]) for f in Fs]
+    esize = Fs[0].element_size()
+    grid = ops.bev_grid_spec(w.ranges, w.res)
+    Fcl = [torch.empty((B, N, h, wl, C), dtype=Fs[0].dtype, device=dev) for h, wl in sizes]
+    out = torch.empty((B, C, w.X, w.Y), device=dev)
+    dF = [torch.empty((B, N, C, h, wl), device=dev) for h, wl in sizes]
+    dt = ops.BF16 if esize == 2 else ops.F32
+    ws_f = torch.empty(max(256, ops.bev_multiscale_workspace_size(dt, ops.NHWC, B, N, C, sizes, 0)),
+                       dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(ops.bev_multiscale_workspace_size(ops.F32, ops.NCHW, B, N, C, sizes, 1),
+                       dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def repack():
+        for f, o in zip(Fs, Fcl):
+            ops.bev_features_to_channels_last(f, out=o)
+
+    stages = {
+        "to_channels_last": repack,
+        "forward": lambda: ops.bev_sample_forward_multiscale(Fcl, K, E, w.img_h, w.img_w, grid, layout=ops.NHWC,
+                                                             out=out, workspace=ws_f),
+        "backward": lambda: ops.bev_sample_backward_multiscale(g, K, E, w.img_h, w.img_w, grid, N, sizes, out=dF,
+                                                               workspace=ws_b),
+    }
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for f in stages.values():
+            f()
+        stream.synchronize()
+        for name, f in stages.items():
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                f()
+            graphs[name] = gr
+        for _ in range(args.warmup):
+            flush.zero_()
+            for gr in graphs.values():
+                gr.replay()
+        stream.synchronize()
+        names = list(stages)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        with ClockSampler(local) as clocks:
+            for k in range(args.steps):
+                flush.zero_()
+                ev[k][0].record(stream)
+                for si, name in enumerate(names):
+                    graphs[name].replay()
+                    ev[k][si + 1].record(stream)
+            torch.cuda.synchronize(dev)
+        per = {name: [ev[k][si].elapsed_time(ev[k][si + 1]) for k in range(args.steps)]
+               for si, name in enumerate(names)}
+    for gr in graphs.values():
+        gr.reset()
+    stage_ms = {name: sum(v) / len(v) for name, v in per.items()}
+    ms_step = sum(stage_ms.values())
+    elems = w.out_elems
+    rate = whole_job_rate(elems, world, max_over_ranks(ms_step, world, dev))
+    peak, peak_src = hbm_peak()
+    feat_bytes = sum(B * N * C * h * wl for h, wl in sizes)
+    fwd_bytes = feat_bytes * esize + elems * 4
+    bwd_bytes = elems * 4 + feat_bytes * 4
+    dom = "forward" if stage_ms["forward"] >= stage_ms["backward"] else "backward"
+    dom_bytes = fwd_bytes if dom == "forward" else bwd_bytes
+    kname = "sample_forward_ms_kernel" if dom == "forward" else "sample_backward_ms_kernel"
+    achieved = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
+    lv = ",".join(f"{h}x{wl}" for h, wl in sizes)
+    line = {
+        "metric": MS_METRIC, "value": rate, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if esize == 4 else "bf16",
+        "data": "synthetic (seeded N(0,1) pyramid levels, 6-camera rig)",
+        "config": {"workload": f"{w.name}: B{B} N{N} C{C} levels {lv} (img {w.img_h}x{w.img_w}) -> "
+                               f"BEV {w.X}x{w.Y}x{w.Z}",
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "timing": "CUDA events around CUDA-graph replays of each stage, launching stream"},
+        "stages_ms": stage_ms,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(kname, w.name), "kernel": kname, "stage": dom,
+                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "note": "forward: every level's features read once + out written once; backward: dout read "
+                             "once + every level's dF written once (whole call timed)",
+                     "peak_source": peak_src},
+        "gpu_launches": args.steps * (2 * len(sizes) + 2),
+        "clocks": clocks.summary(),
+    }
+    if args.cpu_seconds > 0 and rank == 0 and world == 1:
+        threads = cpu_cores()
+        spent, steps = 0.0, 0
+        while steps == 0 or spent < args.cpu_seconds:
+            spent += ms_oracle_step(w, threads)
+            steps += 1
+        line["cpu_baseline"] = {"value": elems * steps / spent, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{steps} whole forward+backward step(s) of the {w.name} workload "
+                                          f"({spent:.1f} s, OpenMP over BEV rows / (batch, camera))"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 LSS_METRIC = "lift-splat BEV pooling output elements/s (B·C·X·Y) and achieved HBM GB/s vs roofline, 1×B200"
 
 
@@ -789,6 +963,8 @@ def main():
     args = parse_args()
     if args.op == "lss":
         run_lss(args)
+    elif args.op == "ms":
+        run_ms(args)
     elif args.op == "deform":
         run_deform(args)
     elif args.impl == "reference":

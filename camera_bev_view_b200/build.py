@@ -9,6 +9,8 @@ import os
 import shutil
 import subprocess
 import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -44,14 +46,33 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    """Compile every .cu to an object in parallel (whole-program device code
+    per file, no relocatable device code), then link the shared library."""
     if not force and up_to_date():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *sources(), "-o", tmp]
-    if ptxas_verbose:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    tmpdir = tempfile.mkdtemp(prefix="bevsample-build-")
+    try:
+        compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+        extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+
+        def one(src):
+            obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
+            r = subprocess.run([nvcc(), *extra, *ARCH, *compile_flags, "-c", src, "-o", obj],
+                               capture_output=True, text=True)
+            return src, obj, r
+
+        with ThreadPoolExecutor(max_workers=max(1, min(len(sources()), os.cpu_count() or 1))) as ex:
+            results = list(ex.map(one, sources()))
+        for src, _, r in results:
+            sys.stdout.write(r.stdout)
+            sys.stderr.write(r.stderr)
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, f"nvcc -c {src}")
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *[o for _, o, _ in results]], check=True)
+        os.replace(tmp, LIB)
+    finally:
+        shutil.rmtree(tmpdir, ignore_errors=True)
     return LIB
 
 

@@ -343,6 +343,203 @@ BEV_API int bev_features_to_channels_last(const void* features, int dtype, int B
 }
 
 // ---------------------------------------------------------------------------
+// Multi-scale dense Sampling-VT
+// ---------------------------------------------------------------------------
+
+namespace {
+
+static_assert(bev::kMaxLevels == BEV_MAX_LEVELS, "level table size");
+
+bool levels_ok(int nlevels, const int* Hf, const int* Wf, int B, int N, int C) {
+    if (nlevels < 1 || nlevels > BEV_MAX_LEVELS || !Hf || !Wf) return false;
+    for (int l = 0; l < nlevels; ++l)
+        if (!dims_ok(B, N, C, Hf[l], Wf[l])) return false;
+    return true;
+}
+
+// Byte offset of level l's region in the workspace (each region 256-byte
+// aligned) and the total: forward = the channels-last copies, backward = the
+// fp32 channels-last gradient buffers.
+size_t ms_ws(int dtype, int layout, int B, int N, int C, int nlevels, const int* Hf, const int* Wf,
+             int for_backward, size_t* offsets) {
+    size_t total = 0;
+    for (int l = 0; l < nlevels; ++l) {
+        if (offsets) offsets[l] = total;
+        total += for_backward ? backward_ws(B, N, C, Hf[l], Wf[l]) : forward_ws(dtype, layout, B, N, C, Hf[l], Wf[l]);
+    }
+    return total;
+}
+
+bev::LevelTable level_table(int nlevels, const int* Hf, const int* Wf, int img_h, int img_w,
+                            const void* const* base) {
+    bev::LevelTable t;
+    memset(&t, 0, sizeof(t));
+    t.n = nlevels;
+    for (int l = 0; l < nlevels; ++l) {
+        t.Hf[l] = Hf[l];
+        t.Wf[l] = Wf[l];
+        t.sW[l] = (float)Wf[l] / (float)img_w;
+        t.sH[l] = (float)Hf[l] / (float)img_h;
+        t.base[l] = base[l];
+    }
+    return t;
+}
+
+}  // namespace
+
+BEV_API size_t bev_multiscale_workspace_size(int dtype, int layout, int B, int N, int C, int nlevels,
+                                             const int* Hf, const int* Wf, int for_backward) {
+    if (!levels_ok(nlevels, Hf, Wf, B, N, C)) return (size_t)-1;
+    if (!for_backward &&
+        ((dtype != BEV_F32 && dtype != BEV_BF16) || (layout != BEV_NCHW && layout != BEV_NHWC)))
+        return (size_t)-1;
+    return ms_ws(dtype, layout, B, N, C, nlevels, Hf, Wf, for_backward, nullptr);
+}
+
+BEV_API int bev_sample_forward_multiscale(const void* const* features, int nlevels, const int* Hf, const int* Wf,
+                                          int dtype, int layout, int B, int N, int C, const float* intrinsics,
+                                          const float* ego2cam, int img_h, int img_w, const bev_grid_t* grid,
+                                          float* out, uint8_t* valid_count, void* workspace,
+                                          size_t workspace_bytes, bev_stream_t stream) {
+    if (!features || !intrinsics || !ego2cam || !out || !grid) return BEV_ERR_INVALID_ARG;
+    if (!levels_ok(nlevels, Hf, Wf, B, N, C) || !grid_ok(grid)) return BEV_ERR_INVALID_ARG;
+    for (int l = 0; l < nlevels; ++l)
+        if (!features[l]) return BEV_ERR_INVALID_ARG;
+    if (img_h < 1 || img_w < 1 || img_h > BEV_MAX_DIM || img_w > BEV_MAX_DIM) return BEV_ERR_INVALID_ARG;
+    if (dtype != BEV_F32 && dtype != BEV_BF16) return BEV_ERR_UNSUPPORTED;
+    if (layout != BEV_NCHW && layout != BEV_NHWC) return BEV_ERR_UNSUPPORTED;
+    const bool repack = needs_repack(dtype, layout, C);
+    size_t off[BEV_MAX_LEVELS];
+    const size_t ws_need = ms_ws(dtype, layout, B, N, C, nlevels, Hf, Wf, 0, off);
+    if (ws_need > 0 && (!workspace || workspace_bytes < ws_need || ((uintptr_t)workspace % kAlign) != 0))
+        return BEV_ERR_WORKSPACE;
+    for (int l = 0; l < nlevels; ++l)
+        if (!repack && ((uintptr_t)features[l] % 16) != 0) return BEV_ERR_INVALID_ARG;
+
+    int dev;
+    int st = current_device(&dev);
+    if (st != BEV_OK) return st;
+    const void* ptrs[4] = {intrinsics, ego2cam, out, valid_count};
+    for (int k = 0; k < 4; ++k) {
+        if (k == 3 && !valid_count) continue;
+        if ((st = device_ptr(ptrs[k], dev)) != BEV_OK) return st;
+    }
+    for (int l = 0; l < nlevels; ++l)
+        if ((st = device_ptr(features[l], dev)) != BEV_OK) return st;
+    if (ws_need > 0 && (st = device_ptr(workspace, dev)) != BEV_OK) return BEV_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int cpc = chan_per_chunk(dtype);
+    const int Cp = round_up(C, cpc);
+    const void* base[BEV_MAX_LEVELS];
+    for (int l = 0; l < nlevels; ++l) {
+        base[l] = features[l];
+        if (repack) {
+            void* dst = static_cast<unsigned char*>(workspace) + off[l];
+            st = cuda_status(bev_launch_to_channels_last(features[l], layout, elem_size(dtype), B * N, C,
+                                                         Hf[l] * Wf[l], Cp, dst, s));
+            if (st != BEV_OK) return st;
+            base[l] = dst;
+        }
+    }
+    bev::SampleArgs a;
+    memset(&a, 0, sizeof(a));
+    a.feat = base[0];
+    a.K = intrinsics;
+    a.E = ego2cam;
+    a.out = out;
+    a.count = valid_count;
+    a.g = geo(grid, Hf[0], Wf[0], img_h, img_w);
+    a.lv = level_table(nlevels, Hf, Wf, img_h, img_w, base);
+    a.B = B;
+    a.N = N;
+    a.C = C;
+    a.Qtot = Cp / cpc;
+    a.chan_per_chunk = cpc;
+    const int max_chunks = bev::kSliceMax / cpc;
+    const int slices = (a.Qtot + max_chunks - 1) / max_chunks;
+    if (slices > 65535) return BEV_ERR_UNSUPPORTED;
+    a.slice_chunks = (a.Qtot + slices - 1) / slices;
+    int V;
+    pick_lanes(a.slice_chunks, &a.L, &V);
+    a.tile_j = bev::kTileJ;
+    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
+    a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
+    int sms;
+    if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
+    const long long ctas = (long long)a.tiles_i * a.tiles_j * B * slices;
+    a.cam_split = ctas < 2LL * sms * bev::kCtasPerSm;
+    if (a.cam_split) {
+        if ((st = cuda_status(cudaMemsetAsync(out, 0, (size_t)B * C * grid->X * grid->Y * sizeof(float), s))) !=
+            BEV_OK)
+            return st;
+    }
+    return cuda_status(bev_launch_forward_ms(a, dtype == BEV_BF16, V, slices, s));
+}
+
+BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const int* Hf, const int* Wf, int B,
+                                           int N, int C, const float* intrinsics, const float* ego2cam, int img_h,
+                                           int img_w, const bev_grid_t* grid, float* const* dfeatures,
+                                           void* workspace, size_t workspace_bytes, bev_stream_t stream) {
+    if (!dout || !intrinsics || !ego2cam || !dfeatures || !grid) return BEV_ERR_INVALID_ARG;
+    if (!levels_ok(nlevels, Hf, Wf, B, N, C) || !grid_ok(grid)) return BEV_ERR_INVALID_ARG;
+    for (int l = 0; l < nlevels; ++l)
+        if (!dfeatures[l]) return BEV_ERR_INVALID_ARG;
+    if (img_h < 1 || img_w < 1 || img_h > BEV_MAX_DIM || img_w > BEV_MAX_DIM) return BEV_ERR_INVALID_ARG;
+    size_t off[BEV_MAX_LEVELS];
+    const size_t ws_need = ms_ws(BEV_F32, BEV_NCHW, B, N, C, nlevels, Hf, Wf, 1, off);
+    if (!workspace || workspace_bytes < ws_need || ((uintptr_t)workspace % kAlign) != 0)
+        return BEV_ERR_WORKSPACE;
+
+    int dev;
+    int st = current_device(&dev);
+    if (st != BEV_OK) return st;
+    const void* ptrs[3] = {dout, intrinsics, ego2cam};
+    for (int k = 0; k < 3; ++k)
+        if ((st = device_ptr(ptrs[k], dev)) != BEV_OK) return st;
+    for (int l = 0; l < nlevels; ++l)
+        if ((st = device_ptr(dfeatures[l], dev)) != BEV_OK) return st;
+    if (device_ptr(workspace, dev) != BEV_OK) return BEV_ERR_WORKSPACE;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int Cp = round_up(C, 4);
+    if ((st = cuda_status(cudaMemsetAsync(workspace, 0, ws_need, s))) != BEV_OK) return st;
+    const void* base[BEV_MAX_LEVELS];
+    for (int l = 0; l < nlevels; ++l) base[l] = static_cast<unsigned char*>(workspace) + off[l];
+    bev::SampleArgs a;
+    memset(&a, 0, sizeof(a));
+    a.K = intrinsics;
+    a.E = ego2cam;
+    a.dout = dout;
+    a.dfeat = static_cast<float*>(workspace);
+    a.g = geo(grid, Hf[0], Wf[0], img_h, img_w);
+    a.lv = level_table(nlevels, Hf, Wf, img_h, img_w, base);
+    a.B = B;
+    a.N = N;
+    a.C = C;
+    a.Qtot = Cp / 4;
+    a.chan_per_chunk = 4;
+    const int max_chunks = bev::kSliceMax / 4;
+    const int slices = (a.Qtot + max_chunks - 1) / max_chunks;
+    if (slices > 65535) return BEV_ERR_UNSUPPORTED;
+    a.slice_chunks = (a.Qtot + slices - 1) / slices;
+    int V;
+    pick_lanes(a.slice_chunks, &a.L, &V);
+    int sms;
+    if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
+    a.tile_j = backward_tile_j(a.L, grid->X, grid->Y, B, slices, sms);
+    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
+    a.tiles_j = (grid->Y + a.tile_j - 1) / a.tile_j;
+    if ((st = cuda_status(bev_launch_backward_ms(a, V, slices, s))) != BEV_OK) return st;
+    for (int l = 0; l < nlevels; ++l) {
+        st = cuda_status(bev_launch_to_nchw(static_cast<const float*>(base[l]), B * N, C, Hf[l] * Wf[l], Cp,
+                                            dfeatures[l], s));
+        if (st != BEV_OK) return st;
+    }
+    return BEV_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Deformable aggregation
 // ---------------------------------------------------------------------------
 

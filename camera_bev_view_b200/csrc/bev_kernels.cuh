@@ -47,6 +47,20 @@ static_assert((int)sizeof(float) * kSliceMax * kStageStride <= kWarpBytes + 512,
 // of the SM's on-chip array serves as L1 for the tiles' texel windows.
 constexpr int kCtasPerSm = 3;
 
+// Feature-pyramid levels of the multi-scale operator.  Every level shares
+// the voxel's projection, validity and count; level l samples its own map at
+// its own scale.  The single-level kernels read g (Hf, Wf, sW, sH) and feat
+// instead.
+constexpr int kMaxLevels = 4;
+
+struct LevelTable {
+    int n;                            // levels, 1 .. kMaxLevels
+    int Hf[kMaxLevels], Wf[kMaxLevels];
+    float sW[kMaxLevels], sH[kMaxLevels];  // (float)W_l / img_w, (float)H_l / img_h, host IEEE divide
+    const void* base[kMaxLevels];     // forward: channels-last features of level l (16-byte chunks);
+                                      // backward: its fp32 channels-last gradient buffer
+};
+
 struct SampleArgs {
     const void* feat;       // channels-last [B*N][Hf*Wf][Qtot chunks of 16 bytes]
     const float* K;         // [B,N,3,3]
@@ -64,6 +78,7 @@ struct SampleArgs {
     int tile_j;             // cells per tile row: kTileJ (forward) or a multiple of 32 / L (backward)
     int tiles_i, tiles_j;   // tiles along X and Y
     int cam_split;          // forward: two CTAs per tile, each gathering every other camera
+    LevelTable lv;          // multi-scale kernels only
 };
 
 // Bytes of dynamic shared memory of one CTA (see carve_smem).
@@ -102,6 +117,10 @@ inline int carveout_percent(size_t smem) {
 cudaError_t bev_launch_forward(const bev::SampleArgs& a, bool bf16, int V, int slices,
                                cudaStream_t stream);
 cudaError_t bev_launch_backward(const bev::SampleArgs& a, int V, int slices, cudaStream_t stream);
+// Multi-scale forms (a.lv describes the levels).
+cudaError_t bev_launch_forward_ms(const bev::SampleArgs& a, bool bf16, int V, int slices,
+                                  cudaStream_t stream);
+cudaError_t bev_launch_backward_ms(const bev::SampleArgs& a, int V, int slices, cudaStream_t stream);
 cudaError_t bev_launch_to_channels_last(const void* src, int layout, int esize, int BN, int C,
                                         int HW, int Cp, void* dst, cudaStream_t stream);
 cudaError_t bev_launch_to_nchw(const float* src, int BN, int C, int HW, int Cp, float* dst,

@@ -196,8 +196,9 @@ struct Items {
 };
 
 // Project this lane's bins z = z0 + ql + L t (t < zn) of voxel column (x, y)
-// through one camera.
-template <int L, int ZN>
+// through one camera.  UV: keep the image-plane position (u, v) in the fx /
+// fy slots, for the multi-scale kernels to take to each level with at_level.
+template <int L, int ZN, bool UV = false>
 __device__ __forceinline__ Items<ZN> project_items(const float* cam, float x, float y, bool in_grid, int z0,
                                                int zn, int ql, const GeoParams& g) {
     Items<ZN> it;
@@ -209,12 +210,27 @@ __device__ __forceinline__ Items<ZN> project_items(const float* cam, float x, fl
         const int z = z0 + ql + L * t;
         if (t < zn && in_grid && z < g.Z) {
             float fx, fy;
-            if (project_voxel(cam, x, y, voxel_centre(g.zmin, z, g.dz), g, fx, fy)) {
-                it.fx[t] = fx;
-                it.fy[t] = fy;
+            ProjDetail det;
+            if (project_point(cam, x, y, voxel_centre(g.zmin, z, g.dz), g, fx, fy, det)) {
+                it.fx[t] = UV ? det.u : fx;
+                it.fy[t] = UV ? det.v : fy;
                 it.ok |= 1u << t;
             }
         }
+    }
+    return it;
+}
+
+// Sampling positions on one pyramid level from image-plane positions: the
+// same two roundings as project_point, fx = u * sW - 0.5.
+template <int ZN>
+__device__ __forceinline__ Items<ZN> at_level(const Items<ZN>& uv, float sW, float sH) {
+    Items<ZN> it;
+    it.ok = uv.ok;
+#pragma unroll
+    for (int t = 0; t < ZN; ++t) {
+        it.fx[t] = __fadd_rn(__fmul_rn(uv.fx[t], sW), -0.5f);
+        it.fy[t] = __fadd_rn(__fmul_rn(uv.fy[t], sH), -0.5f);
     }
     return it;
 }

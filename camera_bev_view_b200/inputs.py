@@ -32,6 +32,17 @@ as [-10, 10] m):
   lss       B1 N6 C64 D41 8x22  (img 128x352)  200x200 over +-50 m fp32
   lss_b4    B4 N6 C64 D41 16x44 (img 256x704)  200x200 over +-50 m fp32
 
+Multi-scale workloads (FlashBEV reading notes, "Takeaway" 4: multi-scale
+fused view transformation; SparseDriveV2 notes, "Image Encoder": an FPN
+gives P2..P5 at strides 4, 8, 16 and 32 with one channel count; 256x704
+images as in the nuScenes-like workload):
+
+  ms_tiny   B1 N6 C16  32x88,16x44,8x22,4x11 (img 128x352)  50x50x4   over +-25 m fp32
+  ms        B1 N6 C64  64x176,32x88,16x44,8x22 (img 256x704) 200x200x8 over +-50 m fp32
+  ms_bf16   B2 N6 C128 64x176,32x88,16x44,8x22 (img 256x704) 200x200x8 over +-50 m bf16
+
+Level l of the features is drawn i.i.d. N(0, 1) from its own seed.
+
 Depth distributions are a softmax over the bins of N(0, 1) * 2 logits;
 context features and the upstream gradient are N(0, 1).
 
@@ -137,6 +148,69 @@ DEFORM_WORKLOADS = {
     "deform": DeformWorkload("deform", 11, 1, 6, 256, 64, 176, 512, 1408, 900, 13, "f32"),
     "deform_bf16": DeformWorkload("deform_bf16", 12, 4, 6, 256, 64, 176, 512, 1408, 900, 13, "bf16"),
 }
+
+
+@dataclasses.dataclass(frozen=True)
+class MultiScaleWorkload:
+    name: str
+    index: int            # seed family
+    B: int
+    N: int
+    C: int
+    levels: tuple         # ((H_0, W_0), (H_1, W_1), ...)
+    img_h: int
+    img_w: int
+    X: int
+    Y: int
+    Z: int
+    xr: tuple
+    yr: tuple
+    zr: tuple
+    dtype: str            # "f32" or "bf16" feature storage
+
+    @property
+    def ranges(self):
+        return (self.xr[0], self.xr[1], self.yr[0], self.yr[1], self.zr[0], self.zr[1])
+
+    @property
+    def res(self):
+        return ((self.xr[1] - self.xr[0]) / self.X,
+                (self.yr[1] - self.yr[0]) / self.Y,
+                (self.zr[1] - self.zr[0]) / self.Z)
+
+    @property
+    def out_elems(self):
+        return self.B * self.C * self.X * self.Y
+
+    def scaled(self, **kw):
+        return dataclasses.replace(self, **kw)
+
+
+_P2_P5_256x704 = ((64, 176), (32, 88), (16, 44), (8, 22))
+
+MS_WORKLOADS = {
+    "ms_tiny": MultiScaleWorkload("ms_tiny", 30, 1, 6, 16, ((32, 88), (16, 44), (8, 22), (4, 11)), 128, 352,
+                                  50, 50, 4, (-25.0, 25.0), (-25.0, 25.0), (-5.0, 3.0), "f32"),
+    "ms": MultiScaleWorkload("ms", 31, 1, 6, 64, _P2_P5_256x704, 256, 704, 200, 200, 8,
+                             (-50.0, 50.0), (-50.0, 50.0), (-5.0, 3.0), "f32"),
+    "ms_bf16": MultiScaleWorkload("ms_bf16", 32, 2, 6, 128, _P2_P5_256x704, 256, 704, 200, 200, 8,
+                                  (-50.0, 50.0), (-50.0, 50.0), (-5.0, 3.0), "bf16"),
+}
+
+
+def make_ms_features(w: MultiScaleWorkload, shard: int = 0, layout: str = "nchw"):
+    """One i.i.d. N(0,1) feature map per level, [B,N,C,H_l,W_l] (or
+    [B,N,H_l,W_l,C] for ``nhwc``) on CPU; bf16 rounds the float32 draw."""
+    out = []
+    for l, (h, wl) in enumerate(w.levels):
+        g = torch.Generator().manual_seed(5000 + 10 * w.index + l + 100003 * shard)
+        f = torch.randn((w.B, w.N, w.C, h, wl), generator=g, dtype=torch.float32)
+        if w.dtype == "bf16":
+            f = f.to(torch.bfloat16)
+        if layout == "nhwc":
+            f = f.permute(0, 1, 3, 4, 2).contiguous()
+        out.append(f)
+    return out
 
 
 @dataclasses.dataclass(frozen=True)

@@ -102,6 +102,14 @@ def lib():
         L.bev_lss_backward.argtypes = [P, P, P, I, I, I, I, I, I, P, P, I, I, Fl, Fl, ctypes.POINTER(BevGrid),
                                        P, P, P, S, P]
         L.bev_lss_backward.restype = I
+        L.bev_multiscale_workspace_size.argtypes = [I, I, I, I, I, I, P, P, I]
+        L.bev_multiscale_workspace_size.restype = S
+        L.bev_sample_forward_multiscale.argtypes = [P, I, P, P, I, I, I, I, I, P, P, I, I,
+                                                    ctypes.POINTER(BevGrid), P, P, P, S, P]
+        L.bev_sample_forward_multiscale.restype = I
+        L.bev_sample_backward_multiscale.argtypes = [P, I, P, P, I, I, I, P, P, I, I, ctypes.POINTER(BevGrid),
+                                                     P, P, S, P]
+        L.bev_sample_backward_multiscale.restype = I
         L.bev_status_string.argtypes = [I]
         L.bev_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -194,6 +202,77 @@ def bev_sample_backward(dout: torch.Tensor, K: torch.Tensor, E: torch.Tensor, im
         _stream_ptr(stream))
     if st != 0:
         raise BevError(st, "bev_sample_backward")
+    return out
+
+
+def _int_array(vals):
+    return (ctypes.c_int * len(vals))(*[int(v) for v in vals])
+
+
+def _ptr_array(tensors):
+    return (ctypes.c_void_p * len(tensors))(*[t.data_ptr() for t in tensors])
+
+
+def bev_multiscale_workspace_size(dtype: int, layout: int, B: int, N: int, C: int, sizes,
+                                  for_backward: int) -> int:
+    """``sizes`` = [(H_l, W_l), ...]."""
+    v = lib().bev_multiscale_workspace_size(dtype, layout, B, N, C, len(sizes), _int_array([h for h, _ in sizes]),
+                                            _int_array([w for _, w in sizes]), for_backward)
+    if v == ctypes.c_size_t(-1).value:
+        raise BevError(-1, "bev_multiscale_workspace_size")
+    return int(v)
+
+
+def bev_sample_forward_multiscale(levels, K: torch.Tensor, E: torch.Tensor, img_h: int, img_w: int,
+                                  grid: BevGrid, layout: int = NCHW, out: torch.Tensor | None = None,
+                                  count: torch.Tensor | bool | None = None, workspace: torch.Tensor | None = None,
+                                  stream=None):
+    """Multi-scale forward.  ``levels`` = list of device tensors, level l
+    [B,N,C,H_l,W_l] (NCHW) or [B,N,H_l,W_l,C] (NHWC), one dtype.  Returns
+    (out [B,C,X,Y] fp32, count [B,X,Y,Z] uint8 or None)."""
+    levels = list(levels)
+    if layout == NCHW:
+        B, N, C = levels[0].shape[:3]
+        sizes = [tuple(f.shape[3:5]) for f in levels]
+    else:
+        B, N = levels[0].shape[:2]
+        C = levels[0].shape[4]
+        sizes = [tuple(f.shape[2:4]) for f in levels]
+    dev = levels[0].device
+    dtype = _dtype_code(levels[0])
+    if out is None:
+        out = torch.empty((B, C, grid.X, grid.Y), dtype=torch.float32, device=dev)
+    if count is True:
+        count = torch.empty((B, grid.X, grid.Y, grid.Z), dtype=torch.uint8, device=dev)
+    elif count is False:
+        count = None
+    ws, ws_bytes = _workspace(bev_multiscale_workspace_size(dtype, layout, B, N, C, sizes, 0), dev, workspace)
+    st = lib().bev_sample_forward_multiscale(
+        _ptr_array(levels), len(levels), _int_array([h for h, _ in sizes]), _int_array([w for _, w in sizes]),
+        dtype, layout, B, N, C, K.data_ptr(), E.data_ptr(), int(img_h), int(img_w), ctypes.byref(grid),
+        out.data_ptr(), count.data_ptr() if count is not None else None,
+        ws.data_ptr() if ws is not None else None, ws_bytes, _stream_ptr(stream))
+    if st != 0:
+        raise BevError(st, "bev_sample_forward_multiscale")
+    return out, count
+
+
+def bev_sample_backward_multiscale(dout: torch.Tensor, K: torch.Tensor, E: torch.Tensor, img_h: int, img_w: int,
+                                   grid: BevGrid, N: int, sizes, out=None, workspace: torch.Tensor | None = None,
+                                   stream=None):
+    """dL/dF_l for every level: list of [B,N,C,H_l,W_l] fp32 for dout [B,C,X,Y]."""
+    B, C = dout.shape[:2]
+    dev = dout.device
+    sizes = [tuple(s) for s in sizes]
+    if out is None:
+        out = [torch.empty((B, N, C, h, w), dtype=torch.float32, device=dev) for h, w in sizes]
+    ws, ws_bytes = _workspace(bev_multiscale_workspace_size(F32, NCHW, B, N, C, sizes, 1), dev, workspace)
+    st = lib().bev_sample_backward_multiscale(
+        dout.data_ptr(), len(sizes), _int_array([h for h, _ in sizes]), _int_array([w for _, w in sizes]),
+        B, N, C, K.data_ptr(), E.data_ptr(), int(img_h), int(img_w), ctypes.byref(grid),
+        _ptr_array(out), ws.data_ptr() if ws is not None else None, ws_bytes, _stream_ptr(stream))
+    if st != 0:
+        raise BevError(st, "bev_sample_backward_multiscale")
     return out
 
 

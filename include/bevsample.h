@@ -179,6 +179,60 @@ int bev_features_to_channels_last(const void* features, int dtype, int B, int N,
                                   void* out, bev_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Multi-scale dense Sampling-VT (FlashBEV reading notes, "Takeaway" 4:
+ * multi-scale fused view transformation; SparseDriveV2 notes, "Image
+ * Encoder": FPN levels P_l with one channel count).  Each voxel is projected
+ * once per camera, with the validity test and count of bev_sample_forward;
+ * level l samples its own map at its own scale, fx_l = u * (W_l / W_img) - 0.5
+ * (fy_l likewise), and the samples of all levels are summed inside the valid
+ * mean:
+ *   out[b, c, i, j] = sum_k [cnt > 0] (1 / cnt) sum_{valid n} sum_l bilinear(F_l[b, n, c], fx_l, fy_l)
+ * With one level this is bev_sample_forward.  The levels are combined by an
+ * unweighted sum (the notes name the direction, not a combination rule); a
+ * corner outside level l's map contributes zero at that level only.
+ * ------------------------------------------------------------------------- */
+
+/* Pyramid levels accepted by the multi-scale calls. */
+#define BEV_MAX_LEVELS 4
+
+/* Workspace bytes of bev_sample_forward_multiscale (for_backward = 0) or
+ * bev_sample_backward_multiscale (for_backward = 1): the per-level sizes of
+ * bev_workspace_size, each rounded up to 256 bytes, summed.  Hf, Wf are host
+ * arrays of nlevels entries.  Returns (size_t)-1 for invalid sizes. */
+size_t bev_multiscale_workspace_size(int dtype, int layout, int B, int N, int C, int nlevels,
+                                     const int* Hf, const int* Wf, int for_backward);
+
+/* Forward over nlevels (1..BEV_MAX_LEVELS) pyramid levels.
+ *   features    host array of nlevels device pointers; level l is
+ *               [B,N,C,Hf[l],Wf[l]] (BEV_NCHW) or [B,N,Hf[l],Wf[l],C] (BEV_NHWC),
+ *               all levels of one dtype and layout
+ *   Hf, Wf      host arrays of nlevels map sizes (any sizes; not necessarily halvings)
+ *   out         [B,C,X,Y] fp32, fully overwritten; valid_count as for bev_sample_forward
+ *   workspace   at least bev_multiscale_workspace_size(.., 0) bytes, 256-byte aligned
+ *               (may be NULL when that size is 0)
+ * Other arguments, checks and errors as for bev_sample_forward; nlevels
+ * outside 1..BEV_MAX_LEVELS or a NULL level pointer -> BEV_ERR_INVALID_ARG. */
+int bev_sample_forward_multiscale(const void* const* features, int nlevels, const int* Hf, const int* Wf,
+                                  int dtype, int layout, int B, int N, int C,
+                                  const float* intrinsics, const float* ego2cam,
+                                  int img_h, int img_w, const bev_grid_t* grid,
+                                  float* out, uint8_t* valid_count,
+                                  void* workspace, size_t workspace_bytes, bev_stream_t stream);
+
+/* Backward of bev_sample_forward_multiscale with respect to every level's
+ * features: dF_l[b, n, c, y, x] = sum of w_l * dout[b, c, i, j] / cnt_k over
+ * the valid samples whose level-l corners touch texel (y, x).
+ *   dfeatures   host array of nlevels device pointers, level l [B,N,C,Hf[l],Wf[l]]
+ *               fp32, fully overwritten
+ *   workspace   at least bev_multiscale_workspace_size(.., 1) bytes, 256-byte aligned
+ * Other arguments and errors as for bev_sample_backward. */
+int bev_sample_backward_multiscale(const float* dout, int nlevels, const int* Hf, const int* Wf,
+                                   int B, int N, int C, const float* intrinsics, const float* ego2cam,
+                                   int img_h, int img_w, const bev_grid_t* grid,
+                                   float* const* dfeatures, void* workspace, size_t workspace_bytes,
+                                   bev_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Deformable aggregation (SparseDriveV2 notes, "Deformable Aggregation",
  * steps 1-3).  Each query q of batch item b has a 3-D anchor a and Kp
  * keypoint offsets d_k; its keypoints p_k = a + d_k (fp32 sums, ego frame)

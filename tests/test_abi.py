@@ -256,3 +256,87 @@ def test_lss_argument_errors(L):
 def test_lss_valid_host_checks_then_cuda_error_without_device(L):
     assert _lfwd(L) == -4
     assert _lbwd(L) == -4
+
+
+# --------------------------------------------------------------------------
+# multi-scale dense Sampling-VT
+# --------------------------------------------------------------------------
+
+def test_header_declares_the_multiscale_calls():
+    names = declared_functions()
+    for n in ["bev_multiscale_workspace_size", "bev_sample_forward_multiscale", "bev_sample_backward_multiscale"]:
+        assert n in names
+    assert re.search(r"#define BEV_MAX_LEVELS 4\b", open(HEADER).read())
+
+
+P2_P5 = [(64, 176), (32, 88), (16, 44), (8, 22)]
+
+
+def test_multiscale_workspace_sizes(L):
+    per = [ops.bev_workspace_size(0, 0, 1, 6, 64, h, w, 0) for h, w in P2_P5]
+    assert ops.bev_multiscale_workspace_size(0, 0, 1, 6, 64, P2_P5, 0) == sum(per)
+    assert ops.bev_multiscale_workspace_size(0, 1, 1, 6, 64, P2_P5, 0) == 0          # NHWC in place
+    # per-level regions are 256-byte aligned: 1x1x3 channels of 2x2 texels -> 256 bytes each
+    assert ops.bev_multiscale_workspace_size(0, 0, 1, 1, 3, [(2, 2), (1, 1), (1, 2)], 0) == 3 * 256
+    bw = [ops.bev_workspace_size(0, 0, 2, 6, 64, h, w, 1) for h, w in P2_P5]
+    assert ops.bev_multiscale_workspace_size(0, 0, 2, 6, 64, P2_P5, 1) == sum(bw)
+    assert ops.bev_multiscale_workspace_size(0, 0, 1, 6, 64, P2_P5[:1], 0) == per[0]
+    for args in [(0, 0, 1, 6, 64, [], 0), (0, 0, 1, 6, 64, P2_P5 + [(4, 11)], 0),
+                 (0, 0, 1, 6, 64, [(16, 44), (0, 22)], 0), (2, 0, 1, 6, 64, P2_P5, 0), (0, 0, 1, 33, 64, P2_P5, 1)]:
+        with pytest.raises(ops.BevError):
+            ops.bev_multiscale_workspace_size(*args)
+
+
+def _ms_fwd(L, levels=P2_P5, feats=None, **kw):
+    g = ops.bev_grid_spec((-50, 50, -50, 50, -5, 3), (0.5, 0.5, 1.0))
+    n = len(levels)
+    fp = feats if feats is not None else (ctypes.c_void_p * max(n, 1))(*([FAKE] * max(n, 1)))
+    a = dict(features=fp, n=n, H=ops._int_array([h for h, _ in levels] or [0]),
+             W=ops._int_array([w for _, w in levels] or [0]), dtype=0, layout=0, B=1, N=6, C=64, K=FAKE, E=FAKE,
+             img_h=256, img_w=704, grid=ctypes.byref(g), out=FAKE, count=None, ws=FAKE, ws_bytes=1 << 30,
+             stream=None)
+    a.update(kw)
+    return L.bev_sample_forward_multiscale(a["features"], a["n"], a["H"], a["W"], a["dtype"], a["layout"], a["B"],
+                                           a["N"], a["C"], a["K"], a["E"], a["img_h"], a["img_w"], a["grid"],
+                                           a["out"], a["count"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def _ms_bwd(L, levels=P2_P5, grads=None, **kw):
+    g = ops.bev_grid_spec((-50, 50, -50, 50, -5, 3), (0.5, 0.5, 1.0))
+    n = len(levels)
+    gp = grads if grads is not None else (ctypes.c_void_p * max(n, 1))(*([FAKE] * max(n, 1)))
+    a = dict(dout=FAKE, n=n, H=ops._int_array([h for h, _ in levels] or [0]),
+             W=ops._int_array([w for _, w in levels] or [0]), B=2, N=6, C=64, K=FAKE, E=FAKE, img_h=256,
+             img_w=704, grid=ctypes.byref(g), dF=gp, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.bev_sample_backward_multiscale(a["dout"], a["n"], a["H"], a["W"], a["B"], a["N"], a["C"], a["K"],
+                                            a["E"], a["img_h"], a["img_w"], a["grid"], a["dF"], a["ws"],
+                                            a["ws_bytes"], a["stream"])
+
+
+def test_multiscale_argument_errors(L):
+    one_null = (ctypes.c_void_p * 4)(FAKE, FAKE, None, FAKE)
+    cases = [
+        (dict(features=None), -1), (dict(n=0), -1), (dict(n=5), -1), (dict(H=None), -1), (dict(W=None), -1),
+        (dict(K=None), -1), (dict(out=None), -1), (dict(grid=None), -1), (dict(N=33), -1), (dict(C=0), -1),
+        (dict(img_w=0), -1), (dict(feats=one_null), -1),
+        (dict(dtype=2), -2), (dict(layout=3), -2),
+        (dict(ws=None), -3), (dict(ws_bytes=1000), -3), (dict(ws=FAKE + 8), -3),
+    ]
+    for kw, want in cases:
+        feats = kw.pop("feats", None)
+        assert _ms_fwd(L, feats=feats, **kw) == want, kw
+    assert _ms_fwd(L, levels=[(16, 44), (0, 22)]) == -1
+    unaligned = (ctypes.c_void_p * 4)(FAKE, FAKE + 4, FAKE, FAKE)
+    assert _ms_fwd(L, feats=unaligned, layout=1, ws=None, ws_bytes=0) == -1   # NHWC in place must be 16B aligned
+    bwd = [(dict(dout=None), -1), (dict(dF=None), -1), (dict(n=0), -1), (dict(n=5), -1), (dict(N=40), -1),
+           (dict(grads=one_null), -1), (dict(ws=None), -3), (dict(ws_bytes=4096), -3), (dict(ws=FAKE + 16), -3)]
+    for kw, want in bwd:
+        grads = kw.pop("grads", None)
+        assert _ms_bwd(L, grads=grads, **kw) == want, kw
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_multiscale_valid_host_checks_then_cuda_error_without_device(L):
+    assert _ms_fwd(L) == -4
+    assert _ms_bwd(L) == -4
