@@ -138,7 +138,7 @@ int cuda_status(cudaError_t e) {
 // short second wave of the heaviest, near-rig tiles).  Must be a multiple
 // of the 32 / L cells a warp works on at once.
 int backward_tile_j(int L, int X, int Y, int B, int slices, int sms) {
-    const long long slots = (long long)sms * bev::kCtasPerSm;
+    const long long slots = (long long)sms * bev::kCtasPerSmBwd;
     const long long tiles = (long long)((X + bev::kTileI - 1) / bev::kTileI) *
                             ((Y + bev::kTileJ - 1) / bev::kTileJ) * B * slices;
     const int half = bev::kTileJ / 2;

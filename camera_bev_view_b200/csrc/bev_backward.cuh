@@ -207,14 +207,14 @@ __device__ __forceinline__ void backward_body(const SampleArgs& a) {
 }
 
 template <int L, int V>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_kernel(const SampleArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSmBwd) sample_backward_kernel(const SampleArgs a) {
     backward_body<L, V, false>(a);
 }
 
 // The level table is indexed at run time: __grid_constant__ lets the body
 // read it in place from the parameter space.
 template <int L, int V>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_backward_ms_kernel(const __grid_constant__ SampleArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSmBwd) sample_backward_ms_kernel(const __grid_constant__ SampleArgs a) {
     backward_body<L, V, true>(a);
 }
 
@@ -227,7 +227,7 @@ static cudaError_t launch_one(const SampleArgs& a, dim3 grid, size_t smem, cudaS
         k = sample_backward_kernel<L, V>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, carveout_percent(smem));
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, carveout_percent(smem, kCtasPerSmBwd));
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, smem, st>>>(a);
     return cudaGetLastError();

@@ -46,6 +46,8 @@ static_assert((int)sizeof(float) * kSliceMax * kStageStride <= kWarpBytes + 512,
 // CTAs kept resident per SM; shared memory stays small (~34 KB) so that most
 // of the SM's on-chip array serves as L1 for the tiles' texel windows.
 constexpr int kCtasPerSm = 3;
+// The backward holds dout instead of accumulators and fits more CTAs.
+constexpr int kCtasPerSmBwd = 3;
 
 // Feature-pyramid levels of the multi-scale operator.  Every level shares
 // the voxel's projection, validity and count; level l samples its own map at
@@ -100,12 +102,12 @@ __host__ __device__ inline SmemLayout smem_layout(int N) {
 
 __host__ __device__ inline size_t sample_smem_bytes(int N) { return smem_layout(N).total; }
 
-// Preferred shared-memory carveout for kCtasPerSm CTAs of `smem` bytes each:
+// Preferred shared-memory carveout for `ctas` CTAs of `smem` bytes each:
 // the smallest shared-memory configuration of the SM (KB) that holds them,
 // as a percentage of the 228 KB maximum; the rest of the array is L1.
-inline int carveout_percent(size_t smem) {
+inline int carveout_percent(size_t smem, int ctas = kCtasPerSm) {
     const int sizes_kb[] = {0, 8, 16, 32, 64, 100, 132, 164, 196, 228};
-    const size_t need = (size_t)kCtasPerSm * (smem + 1024);
+    const size_t need = (size_t)ctas * (smem + 1024);
     for (int kb : sizes_kb)
         if ((size_t)kb * 1024 >= need) return (100 * kb + 227) / 228;
     return 100;

@@ -3,10 +3,10 @@
 // to_channels_last: features [BN][C][HW] (or [BN][HW][C]) -> [BN][HW][Cp] with
 //   zero padding channels, so that one texel's channel vector is contiguous
 //   and 16-byte aligned for the gather kernels.  Pure HBM-bound copies: the
-//   NCHW case moves 4x4 blocks with 16-byte loads and stores for 4-byte
-//   elements when the shapes allow it, else a 32x32 shared-memory tiled
-//   transpose (coalesced on both sides); the unaligned-NHWC case is a straight
-//   strided copy.
+//   NCHW case moves 4x4 blocks (4-byte elements) or 8x8 blocks (2-byte
+//   elements) with 16-byte loads and stores when the shapes allow it, else a
+//   32x32 shared-memory tiled transpose (coalesced on both sides); the
+//   unaligned-NHWC case is a straight strided copy.
 // to_nchw: the fp32 channels-last gradient buffer [BN][HW][Cp] -> [BN][C][HW].
 //   When HW is a multiple of 4 and the output is 16-byte aligned, each thread
 //   moves a 4 texel x 4 channel block with 16-byte loads and 16-byte stores
@@ -92,6 +92,41 @@ __global__ void __launch_bounds__(256) nchw_to_nhwc_v4_kernel(const float* __res
     *reinterpret_cast<float4*>(d + 3 * (size_t)Cp) = make_float4(r[0].w, r[1].w, r[2].w, r[3].w);
 }
 
+// 8x8 register-blocked NCHW -> channels-last copy for 2-byte elements: block
+// (16 x 16 threads) covers 128 channels x 128 texels; thread (tx, ty) reads
+// channels 8 ty .. 8 ty + 7 at texels 8 tx .. 8 tx + 7 (eight 16-byte loads)
+// and writes eight texel rows of 8 channels (eight 16-byte stores); each
+// output word pairs the same texel of two channels (a byte permute).
+// Padding channels are written as 0.  HW % 8 == 0, Cp % 8 == 0, both
+// pointers 16-byte aligned.
+__global__ void __launch_bounds__(256) nchw_to_nhwc_16x8_kernel(const uint16_t* __restrict__ src, int C, int HW,
+                                                                int Cp, uint16_t* __restrict__ dst) {
+    const size_t bn = blockIdx.z;
+    const int c = blockIdx.y * 128 + 8 * threadIdx.y;
+    const int p = blockIdx.x * 128 + 8 * threadIdx.x;
+    if (p >= HW || c >= Cp) return;
+    uint4 r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        r[i] = c + i < C ? __ldg(reinterpret_cast<const uint4*>(src + (bn * C + c + i) * (size_t)HW + p))
+                         : make_uint4(0u, 0u, 0u, 0u);
+    uint16_t* d = dst + (bn * HW + p) * (size_t)Cp + c;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        // texel j sits in word j / 2 of every channel row, low half for even j
+        const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
+        unsigned w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint4& v = r[i];
+            w[i] = (j >> 1) == 0 ? v.x : (j >> 1) == 1 ? v.y : (j >> 1) == 2 ? v.z : v.w;
+        }
+        const uint4 o = make_uint4(__byte_perm(w[0], w[1], sel), __byte_perm(w[2], w[3], sel),
+                                   __byte_perm(w[4], w[5], sel), __byte_perm(w[6], w[7], sel));
+        *reinterpret_cast<uint4*>(d + (size_t)j * Cp) = o;
+    }
+}
+
 // 4x4 register-blocked transpose: block (16 x 16 threads) covers 64 texels x
 // 64 channels; thread (tx, ty) reads texels 4 ty .. 4 ty + 3 at channels
 // 4 tx .. 4 tx + 3 and writes them back as four channel rows.  HW % 4 == 0,
@@ -125,6 +160,11 @@ cudaError_t bev_launch_to_channels_last(const void* src, int layout, int esize, 
         ((uintptr_t)dst % 16) == 0) {
         const dim3 grid((HW + 63) / 64, (Cp + 63) / 64, BN);
         bev::nchw_to_nhwc_v4_kernel<<<grid, dim3(16, 16), 0, stream>>>((const float*)src, C, HW, Cp, (float*)dst);
+    } else if (layout == 0 && esize == 2 && HW % 8 == 0 && Cp % 8 == 0 && ((uintptr_t)src % 16) == 0 &&
+               ((uintptr_t)dst % 16) == 0) {
+        const dim3 grid((HW + 127) / 128, (Cp + 127) / 128, BN);
+        bev::nchw_to_nhwc_16x8_kernel<<<grid, dim3(16, 16), 0, stream>>>((const uint16_t*)src, C, HW, Cp,
+                                                                         (uint16_t*)dst);
     } else if (layout == 0) {  // NCHW
         const dim3 grid((HW + bev::kT - 1) / bev::kT, (Cp + bev::kT - 1) / bev::kT, BN);
         const dim3 block(bev::kT, 8);
