@@ -225,9 +225,8 @@ static cudaError_t launch_one(const SampleArgs& a, dim3 grid, size_t smem, cudaS
         k = sample_backward_ms_kernel<L, V>;
     else
         k = sample_backward_kernel<L, V>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, carveout_percent(smem, kCtasPerSmBwd));
+    static std::atomic<long long> attrs[kAttrDevices];
+    const cudaError_t e = set_smem_attributes(k, smem, carveout_percent(smem, kCtasPerSmBwd), attrs);
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, smem, st>>>(a);
     return cudaGetLastError();

@@ -28,6 +28,7 @@
 // accumulators are added in warp order at the end (deterministic).  The feature gradient is reduced into an fp32
 // channels-last buffer with 16-byte vector reductions.
 #include "bev_deform.cuh"
+#include "bev_kernels.cuh"
 
 namespace bev {
 
@@ -350,10 +351,12 @@ __global__ void __launch_bounds__(kDeformWarps * 32) deform_backward_kernel(cons
 
 namespace {
 
-template <typename Kernel>
-cudaError_t launch(Kernel k, const DeformArgs& a, cudaStream_t st) {
+template <auto K>
+cudaError_t launch(const DeformArgs& a, cudaStream_t st) {
+    const auto k = K;
     const size_t smem = deform_smem_bytes(a.N, a.C, a.Kp);
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<long long> attrs[kAttrDevices];
+    const cudaError_t e = set_smem_attributes(k, smem, -1, attrs);
     if (e != cudaSuccess) return e;
     const dim3 grid(a.Q, a.B);
     k<<<grid, kDeformWarps * 32, smem, st>>>(a);
@@ -367,14 +370,14 @@ cudaError_t launch(Kernel k, const DeformArgs& a, cudaStream_t st) {
 cudaError_t bev_launch_deform_forward(const bev::DeformArgs& a, bool bf16, int V, cudaStream_t stream) {
     using namespace bev;
     switch ((bf16 ? 16 : 0) + V) {
-        case 1: return launch(deform_forward_kernel<false, 1>, a, stream);
-        case 2: return launch(deform_forward_kernel<false, 2>, a, stream);
-        case 3: return launch(deform_forward_kernel<false, 3>, a, stream);
-        case 4: return launch(deform_forward_kernel<false, 4>, a, stream);
-        case 16 + 1: return launch(deform_forward_kernel<true, 1>, a, stream);
-        case 16 + 2: return launch(deform_forward_kernel<true, 2>, a, stream);
-        case 16 + 3: return launch(deform_forward_kernel<true, 3>, a, stream);
-        case 16 + 4: return launch(deform_forward_kernel<true, 4>, a, stream);
+        case 1: return launch<deform_forward_kernel<false, 1>>(a, stream);
+        case 2: return launch<deform_forward_kernel<false, 2>>(a, stream);
+        case 3: return launch<deform_forward_kernel<false, 3>>(a, stream);
+        case 4: return launch<deform_forward_kernel<false, 4>>(a, stream);
+        case 16 + 1: return launch<deform_forward_kernel<true, 1>>(a, stream);
+        case 16 + 2: return launch<deform_forward_kernel<true, 2>>(a, stream);
+        case 16 + 3: return launch<deform_forward_kernel<true, 3>>(a, stream);
+        case 16 + 4: return launch<deform_forward_kernel<true, 4>>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -382,14 +385,14 @@ cudaError_t bev_launch_deform_forward(const bev::DeformArgs& a, bool bf16, int V
 cudaError_t bev_launch_deform_backward(const bev::DeformArgs& a, bool bf16, int V, cudaStream_t stream) {
     using namespace bev;
     switch ((bf16 ? 16 : 0) + V) {
-        case 1: return launch(deform_backward_kernel<false, 1>, a, stream);
-        case 2: return launch(deform_backward_kernel<false, 2>, a, stream);
-        case 3: return launch(deform_backward_kernel<false, 3>, a, stream);
-        case 4: return launch(deform_backward_kernel<false, 4>, a, stream);
-        case 16 + 1: return launch(deform_backward_kernel<true, 1>, a, stream);
-        case 16 + 2: return launch(deform_backward_kernel<true, 2>, a, stream);
-        case 16 + 3: return launch(deform_backward_kernel<true, 3>, a, stream);
-        case 16 + 4: return launch(deform_backward_kernel<true, 4>, a, stream);
+        case 1: return launch<deform_backward_kernel<false, 1>>(a, stream);
+        case 2: return launch<deform_backward_kernel<false, 2>>(a, stream);
+        case 3: return launch<deform_backward_kernel<false, 3>>(a, stream);
+        case 4: return launch<deform_backward_kernel<false, 4>>(a, stream);
+        case 16 + 1: return launch<deform_backward_kernel<true, 1>>(a, stream);
+        case 16 + 2: return launch<deform_backward_kernel<true, 2>>(a, stream);
+        case 16 + 3: return launch<deform_backward_kernel<true, 3>>(a, stream);
+        case 16 + 4: return launch<deform_backward_kernel<true, 4>>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -327,9 +327,8 @@ static cudaError_t launch_one(const SampleArgs& a, dim3 grid, size_t smem, cudaS
         k = sample_forward_ms_kernel<BF16, L, V>;
     else
         k = sample_forward_kernel<BF16, L, V>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, carveout_percent(smem));
+    static std::atomic<long long> attrs[kAttrDevices];
+    const cudaError_t e = set_smem_attributes(k, smem, carveout_percent(smem), attrs);
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, smem, st>>>(a);
     return cudaGetLastError();

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "bev_geometry.cuh"
 
 namespace bev {
@@ -111,6 +113,28 @@ inline int carveout_percent(size_t smem, int ctas = kCtasPerSm) {
     for (int kb : sizes_kb)
         if ((size_t)kb * 1024 >= need) return (100 * kb + 227) / 228;
     return 100;
+}
+
+// A kernel's dynamic shared-memory limit and carveout preference, set once
+// per device and size rather than on every launch (cudaFuncSetAttribute is a
+// driver call that costs microseconds of host time).  `cache` is one static
+// array per kernel; carveout < 0 leaves the preference alone.
+constexpr int kAttrDevices = 64;
+
+template <typename Kernel>
+inline cudaError_t set_smem_attributes(Kernel* k, size_t smem, int carveout,
+                                       std::atomic<long long> (&cache)[kAttrDevices]) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const long long key = (((long long)carveout + 1) << 32) | (long long)smem;
+    const bool cached = dev >= 0 && dev < kAttrDevices;
+    if (cached && cache[dev].load(std::memory_order_relaxed) == key) return cudaSuccess;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess && carveout >= 0)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, carveout);
+    if (e == cudaSuccess && cached) cache[dev].store(key, std::memory_order_relaxed);
+    return e;
 }
 
 }  // namespace bev
