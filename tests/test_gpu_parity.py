@@ -251,3 +251,43 @@ def test_host_pointers_are_rejected_without_launch():
                                 w.img_w, g, 6, w.Hf, w.Wf)                # K on the host
     assert e.value.status == -1
     torch.cuda.synchronize()
+
+
+# --------------------------------------------------------------------------
+# the largest sizes the boundary accepts along each axis (small elsewhere)
+# --------------------------------------------------------------------------
+
+def test_maximum_height_bins():
+    """Z = 1024 (the limit): 64 height chunks per cell in the forward."""
+    K, E = I.make_rig(51, 6, 128, 352)
+    K, E = torch.from_numpy(K)[None], torch.from_numpy(E)[None]
+    F = torch.randn((1, 6, 8, 8, 22), generator=torch.Generator().manual_seed(51))
+    ranges, res = (-8, 8, -8, 8, -5, 3), (2.0, 2.0, 8.0 / 1024)
+    out, ref, cnt, _ = check_forward(F, K, E, 128, 352, ranges, res, 1e-5)
+    assert cnt.shape[-1] == 1024 and cnt.sum() > 10000
+    dout = torch.randn((1, 8, 8, 8), generator=torch.Generator().manual_seed(52))
+    check_backward(dout, K, E, 128, 352, ranges, res, 6, 8, 22)
+
+
+def test_two_thousand_channels_in_sixteen_slices():
+    K, E = I.make_rig(53, 6, 128, 352)
+    K, E = torch.from_numpy(K)[None], torch.from_numpy(E)[None]
+    F = torch.randn((1, 6, 2048, 4, 11), generator=torch.Generator().manual_seed(53))
+    ranges, res = (-12, 12, -12, 12, -4, 4), (1.5, 1.5, 2.0)
+    check_forward(F, K, E, 128, 352, ranges, res, 1e-5)
+    dout = torch.randn((1, 2048, 16, 16), generator=torch.Generator().manual_seed(54))
+    check_backward(dout, K, E, 128, 352, ranges, res, 6, 4, 11)
+
+
+def test_widest_feature_map():
+    """Wf = 16384 (the limit) on a 2048 x 16384 image: texel offsets beyond
+    2^16 within one row."""
+    K = np.array([[[[4000.0, 0, 8192], [0, 4000.0, 1024], [0, 0, 1]]]], np.float32)
+    E = np.array([[[[0, -1, 0, 0], [0, 0, -1, 0], [1, 0, 0, 0], [0, 0, 0, 1]]]], np.float32)
+    K, E = torch.from_numpy(K), torch.from_numpy(E)
+    F = torch.randn((1, 1, 4, 2, 16384), generator=torch.Generator().manual_seed(55))
+    ranges, res = (5, 25, -20, 20, -1, 1), (1.0, 0.25, 0.5)
+    out, ref, cnt, _ = check_forward(F, K, E, 2048, 16384, ranges, res, 1e-5)
+    assert cnt.sum() > 1000
+    dout = torch.randn((1, 4, 20, 160), generator=torch.Generator().manual_seed(56))
+    check_backward(dout, K, E, 2048, 16384, ranges, res, 1, 2, 16384)
