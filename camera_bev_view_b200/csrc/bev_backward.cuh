@@ -132,11 +132,11 @@ __device__ __forceinline__ void backward_body(const SampleArgs& a) {
 
     const int b = blockIdx.y;
     int ti0, tj0;
-    tile_origin(a, s.act + 40, ti0, tj0);
+    tile_origin(a, s, b, s.act + 40, ti0, tj0);
     const int chunk0 = blockIdx.z * a.slice_chunks;
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
     const int c_base = chunk0 * 4;
-    setup_tile(a, s, b, ti0, tj0);
+    setup_tile(a, s, ti0, tj0);
     const int nA = s.act[32];
     if (nA == 0) return;
 

@@ -177,10 +177,10 @@ __device__ __forceinline__ void forward_body(const SampleArgs& a) {
 
     const int b = blockIdx.y;
     int ti0, tj0;
-    tile_origin(a, s.act + 40, ti0, tj0);
+    tile_origin(a, s, b, s.act + 40, ti0, tj0);
     const int chunk0 = blockIdx.z * a.slice_chunks;
     const int nchunks = min(a.slice_chunks, a.Qtot - chunk0);
-    setup_tile(a, s, b, ti0, tj0);
+    setup_tile(a, s, ti0, tj0);
     const int nA = s.act[32];
     // camera split: half h of the tile gathers the active cameras aa with
     // aa % 2 == h (both halves count over all of them); a tile seen by one

@@ -43,15 +43,27 @@ __device__ __forceinline__ CtaSmem carve_smem(unsigned char* smem, int N) {
     return s;
 }
 
+// Calibrations of batch item b into shared memory: E rows 0..2, then K rows
+// 0..1, per camera; threads first .. kThreads - 1 take one float at a time.
+// Only the per-CTA set-up reads them from global memory.
+__device__ __forceinline__ void stage_cams(const SampleArgs& a, const CtaSmem& s, int b, int first) {
+    for (int t = (int)threadIdx.x - first; t < a.N * kCamFloats; t += kThreads - first) {
+        const int n = t / kCamFloats, r = t - n * kCamFloats;
+        s.cams[t] = r < 12 ? a.E[((size_t)b * a.N + n) * 16 + r]
+                           : a.K[((size_t)b * a.N + n) * 9 + (r - 12)];
+    }
+}
+
 // Tile of this CTA (with a camera split, CTAs 2t and 2t + 1 share tile t).
 // Tiles are issued in rings of increasing Chebyshev
 // distance from the centre tile of the grid: for rigs mounted near the grid
 // centre the nearest voxels see the most texels, so the heaviest tiles start
 // first and the light outer ring fills the tail of the launch.  Any order
 // gives the same results.  Warp 0 maps the block index (the rank) to its
-// ring, then finds the position inside the ring with ballots over 32 ring
-// positions at a time.
-__device__ inline void tile_origin(const SampleArgs& a, int* slot, int& ti0, int& tj0) {
+// ring -- its lanes test 32 candidate rings at a time -- then finds the
+// position inside the ring with ballots over 32 ring positions at a time.
+// The other warps meanwhile stage batch item b's calibrations.
+__device__ inline void tile_origin(const SampleArgs& a, const CtaSmem& s, int b, int* slot, int& ti0, int& tj0) {
     const int Ti = a.tiles_i, Tj = a.tiles_j;
     if (threadIdx.x < 32) {
         const int ci = (Ti - 1) >> 1, cj = (Tj - 1) >> 1;
@@ -61,14 +73,19 @@ __device__ inline void tile_origin(const SampleArgs& a, int* slot, int& ti0, int
             const int w = min(cj + r, Tj - 1) - max(cj - r, 0) + 1;
             return h * w;
         };
-        // ring r of rank k: the smallest r with area(r) > k (binary search)
-        int lo = 0, hi = max(max(ci, Ti - 1 - ci), max(cj, Tj - 1 - cj));
+        // ring r of rank k: the smallest r with area(r) > k (area grows with
+        // r and area(rmax) is every tile)
+        const int rmax = max(max(ci, Ti - 1 - ci), max(cj, Tj - 1 - cj));
         const int rank = a.cam_split ? blockIdx.x >> 1 : blockIdx.x;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (area(mid) > rank) hi = mid; else lo = mid + 1;
+        int r = rmax;
+        for (int r0 = 0; r0 <= rmax; r0 += 32) {
+            const int cand = r0 + (int)threadIdx.x;
+            const unsigned m = __ballot_sync(0xffffffffu, cand <= rmax && area(cand) > rank);
+            if (m) {
+                r = r0 + __ffs(m) - 1;
+                break;
+            }
         }
-        const int r = lo;
         int k = rank - area(r - 1);
         const int ring = r == 0 ? 1 : 8 * r;
         int found = -1;
@@ -94,23 +111,19 @@ __device__ inline void tile_origin(const SampleArgs& a, int* slot, int& ti0, int
                 k -= __popc(m);
             }
         }
+    } else {
+        stage_cams(a, s, b, 32);
     }
     __syncthreads();
     ti0 = slot[0];
     tj0 = slot[1];
 }
 
-// Stage camera constants of batch item b and cull cameras against the tile.
+// Cull the cameras (staged by tile_origin) against the tile.
 // One thread per (camera, corner of the tile's voxel-centre box); the five
 // visibility margins are max-reduced over the eight corners with shuffles.
-__device__ inline void setup_tile(const SampleArgs& a, const CtaSmem& s, int b, int ti0, int tj0) {
+__device__ inline void setup_tile(const SampleArgs& a, const CtaSmem& s, int ti0, int tj0) {
     const int tid = threadIdx.x;
-    for (int t = tid; t < a.N * kCamFloats; t += kThreads) {
-        const int n = t / kCamFloats, r = t - n * kCamFloats;
-        s.cams[t] = r < 12 ? a.E[((size_t)b * a.N + n) * 16 + r]
-                           : a.K[((size_t)b * a.N + n) * 9 + (r - 12)];
-    }
-    __syncthreads();
     const GeoParams& g = a.g;
     const int n = tid >> 3, v = tid & 7;  // kThreads == 8 * BEV_MAX_CAMERAS
     if ((tid >> 5) * 4 < a.N) {           // warps holding at least one camera
