@@ -151,6 +151,33 @@ int sm_count(int dev, int* sms) {
     return BEV_OK;
 }
 
+// Channel slices and lanes per cell for Cp channels in chunks of cpc
+// channels: fills a.Qtot, a.chan_per_chunk, a.slice_chunks and a.L, and
+// returns the chunks per lane V (0 when the slices exceed the grid limit).
+int channel_layout(bev::SampleArgs& a, int Cp, int cpc, int* slices) {
+    a.Qtot = Cp / cpc;
+    a.chan_per_chunk = cpc;
+    const int max_chunks = bev::kSliceMax / cpc;
+    *slices = (a.Qtot + max_chunks - 1) / max_chunks;
+    if (*slices > 65535) return 0;
+    a.slice_chunks = (a.Qtot + *slices - 1) / *slices;
+    int V;
+    pick_lanes(a.slice_chunks, &a.L, &V);
+    return V;
+}
+
+// Tiles of a launch.  Forward: 8x8 tiles, and when they fill fewer than two
+// waves of resident CTAs the launch would end on a short wave of the
+// heaviest, near-rig tiles, so every tile's cameras are split over two CTAs
+// that add into the zeroed output.  Backward: the width of backward_tile_j.
+void tile_layout(bev::SampleArgs& a, const bev_grid_t* grid, int B, int slices, int sms, bool backward) {
+    a.tile_j = backward ? backward_tile_j(a.L, grid->X, grid->Y, B, slices, sms) : bev::kTileJ;
+    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
+    a.tiles_j = (grid->Y + a.tile_j - 1) / a.tile_j;
+    const long long ctas = (long long)a.tiles_i * a.tiles_j * B * slices;
+    a.cam_split = !backward && ctas < 2LL * sms * bev::kCtasPerSm;
+}
+
 }  // namespace
 
 BEV_API const char* bev_status_string(int status) {
@@ -252,24 +279,11 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
     a.B = B;
     a.N = N;
     a.C = C;
-    a.Qtot = Cp / cpc;
-    a.chan_per_chunk = cpc;
-    const int max_chunks = bev::kSliceMax / cpc;
-    const int slices = (a.Qtot + max_chunks - 1) / max_chunks;
-    if (slices > 65535) return BEV_ERR_UNSUPPORTED;
-    a.slice_chunks = (a.Qtot + slices - 1) / slices;
-    int V;
-    pick_lanes(a.slice_chunks, &a.L, &V);
-    a.tile_j = bev::kTileJ;
-    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
-    a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
-    // Few tiles (under two waves of resident CTAs): the launch would end on a
-    // short wave of the heaviest, near-rig tiles, so split every tile's
-    // cameras over two CTAs that add into the zeroed output.
-    int sms;
+    int slices, sms;
+    const int V = channel_layout(a, Cp, cpc, &slices);
+    if (V == 0) return BEV_ERR_UNSUPPORTED;
     if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
-    const long long ctas = (long long)a.tiles_i * a.tiles_j * B * slices;
-    a.cam_split = ctas < 2LL * sms * bev::kCtasPerSm;
+    tile_layout(a, grid, B, slices, sms, false);
     if (a.cam_split) {
         if ((st = cuda_status(cudaMemsetAsync(out, 0, (size_t)B * C * grid->X * grid->Y * sizeof(float), s))) !=
             BEV_OK)
@@ -310,19 +324,11 @@ BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, 
     a.B = B;
     a.N = N;
     a.C = C;
-    a.Qtot = Cp / 4;
-    a.chan_per_chunk = 4;
-    const int max_chunks = bev::kSliceMax / 4;
-    const int slices = (a.Qtot + max_chunks - 1) / max_chunks;
-    if (slices > 65535) return BEV_ERR_UNSUPPORTED;
-    a.slice_chunks = (a.Qtot + slices - 1) / slices;
-    int V;
-    pick_lanes(a.slice_chunks, &a.L, &V);
-    int sms;
+    int slices, sms;
+    const int V = channel_layout(a, Cp, 4, &slices);
+    if (V == 0) return BEV_ERR_UNSUPPORTED;
     if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
-    a.tile_j = backward_tile_j(a.L, grid->X, grid->Y, B, slices, sms);
-    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
-    a.tiles_j = (grid->Y + a.tile_j - 1) / a.tile_j;
+    tile_layout(a, grid, B, slices, sms, true);
     if ((st = cuda_status(bev_launch_backward(a, V, slices, s))) != BEV_OK) return st;
     return cuda_status(bev_launch_to_nchw(static_cast<const float*>(workspace), B * N, C, Hf * Wf, Cp,
                                           dfeatures, s));
@@ -370,8 +376,7 @@ size_t ms_ws(int dtype, int layout, int B, int N, int C, int nlevels, const int*
     return total;
 }
 
-bev::LevelTable level_table(int nlevels, const int* Hf, const int* Wf, int img_h, int img_w,
-                            const void* const* base) {
+bev::LevelTable level_table(int nlevels, const int* Hf, const int* Wf, int img_h, int img_w) {
     bev::LevelTable t;
     memset(&t, 0, sizeof(t));
     t.n = nlevels;
@@ -380,7 +385,6 @@ bev::LevelTable level_table(int nlevels, const int* Hf, const int* Wf, int img_h
         t.Wf[l] = Wf[l];
         t.sW[l] = (float)Wf[l] / (float)img_w;
         t.sH[l] = (float)Hf[l] / (float)img_h;
-        t.base[l] = base[l];
     }
     return t;
 }
@@ -450,25 +454,16 @@ BEV_API int bev_sample_forward_multiscale(const void* const* features, int nleve
     a.out = out;
     a.count = valid_count;
     a.g = geo(grid, Hf[0], Wf[0], img_h, img_w);
-    a.lv = level_table(nlevels, Hf, Wf, img_h, img_w, base);
+    a.lv = level_table(nlevels, Hf, Wf, img_h, img_w);
+    for (int l = 0; l < nlevels; ++l) a.lv.feat[l] = base[l];
     a.B = B;
     a.N = N;
     a.C = C;
-    a.Qtot = Cp / cpc;
-    a.chan_per_chunk = cpc;
-    const int max_chunks = bev::kSliceMax / cpc;
-    const int slices = (a.Qtot + max_chunks - 1) / max_chunks;
-    if (slices > 65535) return BEV_ERR_UNSUPPORTED;
-    a.slice_chunks = (a.Qtot + slices - 1) / slices;
-    int V;
-    pick_lanes(a.slice_chunks, &a.L, &V);
-    a.tile_j = bev::kTileJ;
-    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
-    a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
-    int sms;
+    int slices, sms;
+    const int V = channel_layout(a, Cp, cpc, &slices);
+    if (V == 0) return BEV_ERR_UNSUPPORTED;
     if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
-    const long long ctas = (long long)a.tiles_i * a.tiles_j * B * slices;
-    a.cam_split = ctas < 2LL * sms * bev::kCtasPerSm;
+    tile_layout(a, grid, B, slices, sms, false);
     if (a.cam_split) {
         if ((st = cuda_status(cudaMemsetAsync(out, 0, (size_t)B * C * grid->X * grid->Y * sizeof(float), s))) !=
             BEV_OK)
@@ -504,8 +499,8 @@ BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int Cp = round_up(C, 4);
     if ((st = cuda_status(cudaMemsetAsync(workspace, 0, ws_need, s))) != BEV_OK) return st;
-    const void* base[BEV_MAX_LEVELS];
-    for (int l = 0; l < nlevels; ++l) base[l] = static_cast<unsigned char*>(workspace) + off[l];
+    float* base[BEV_MAX_LEVELS];
+    for (int l = 0; l < nlevels; ++l) base[l] = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + off[l]);
     bev::SampleArgs a;
     memset(&a, 0, sizeof(a));
     a.K = intrinsics;
@@ -513,26 +508,19 @@ BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const
     a.dout = dout;
     a.dfeat = static_cast<float*>(workspace);
     a.g = geo(grid, Hf[0], Wf[0], img_h, img_w);
-    a.lv = level_table(nlevels, Hf, Wf, img_h, img_w, base);
+    a.lv = level_table(nlevels, Hf, Wf, img_h, img_w);
+    for (int l = 0; l < nlevels; ++l) a.lv.grad[l] = base[l];
     a.B = B;
     a.N = N;
     a.C = C;
-    a.Qtot = Cp / 4;
-    a.chan_per_chunk = 4;
-    const int max_chunks = bev::kSliceMax / 4;
-    const int slices = (a.Qtot + max_chunks - 1) / max_chunks;
-    if (slices > 65535) return BEV_ERR_UNSUPPORTED;
-    a.slice_chunks = (a.Qtot + slices - 1) / slices;
-    int V;
-    pick_lanes(a.slice_chunks, &a.L, &V);
-    int sms;
+    int slices, sms;
+    const int V = channel_layout(a, Cp, 4, &slices);
+    if (V == 0) return BEV_ERR_UNSUPPORTED;
     if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
-    a.tile_j = backward_tile_j(a.L, grid->X, grid->Y, B, slices, sms);
-    a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
-    a.tiles_j = (grid->Y + a.tile_j - 1) / a.tile_j;
+    tile_layout(a, grid, B, slices, sms, true);
     if ((st = cuda_status(bev_launch_backward_ms(a, V, slices, s))) != BEV_OK) return st;
     for (int l = 0; l < nlevels; ++l) {
-        st = cuda_status(bev_launch_to_nchw(static_cast<const float*>(base[l]), B * N, C, Hf[l] * Wf[l], Cp,
+        st = cuda_status(bev_launch_to_nchw(base[l], B * N, C, Hf[l] * Wf[l], Cp,
                                             dfeatures[l], s));
         if (st != BEV_OK) return st;
     }

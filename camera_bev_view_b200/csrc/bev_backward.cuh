@@ -195,7 +195,7 @@ __device__ __forceinline__ void backward_body(const SampleArgs& a) {
                 } else {
                     for (int l = 0; l < a.lv.n; ++l) {
                         const int Hl = a.lv.Hf[l], Wl = a.lv.Wf[l];
-                        float* Gn = static_cast<float*>(const_cast<void*>(a.lv.base[l])) + (size_t)(chunk0 + ql) * 4 +
+                        float* Gn = a.lv.grad[l] + (size_t)(chunk0 + ql) * 4 +
                                     ((size_t)b * a.N + cam) * ((size_t)Hl * Wl) * tstride;
                         scatter_camera<L, V, ZN>(d, at_level(it, a.lv.sW[l], a.lv.sH[l]), rc, zn, sub, ql, Gn, Hl, Wl,
                                                  tstride, nchunks, region);

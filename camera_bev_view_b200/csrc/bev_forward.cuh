@@ -246,7 +246,7 @@ __device__ __forceinline__ void forward_body(const SampleArgs& a) {
                 } else {
                     for (int l = 0; l < a.lv.n; ++l) {
                         const int Hl = a.lv.Hf[l], Wl = a.lv.Wf[l];
-                        const uint4* Fn = reinterpret_cast<const uint4*>(a.lv.base[l]) + chunk0 + ql +
+                        const uint4* Fn = reinterpret_cast<const uint4*>(a.lv.feat[l]) + chunk0 + ql +
                                           ((size_t)b * a.N + cam) * ((size_t)Hl * Wl) * a.Qtot;
                         gather_camera<BF16, L, V, ZN>(acc[q], at_level(it, a.lv.sW[l], a.lv.sH[l]), rc, zn, sub, ql,
                                                       Fn, Hl, Wl, a.Qtot, nchunks, region);

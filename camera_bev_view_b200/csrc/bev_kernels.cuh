@@ -61,8 +61,8 @@ struct LevelTable {
     int n;                            // levels, 1 .. kMaxLevels
     int Hf[kMaxLevels], Wf[kMaxLevels];
     float sW[kMaxLevels], sH[kMaxLevels];  // (float)W_l / img_w, (float)H_l / img_h, host IEEE divide
-    const void* base[kMaxLevels];     // forward: channels-last features of level l (16-byte chunks);
-                                      // backward: its fp32 channels-last gradient buffer
+    const void* feat[kMaxLevels];     // forward: channels-last features of level l (16-byte chunks)
+    float* grad[kMaxLevels];          // backward: fp32 channels-last gradient buffer of level l
 };
 
 struct SampleArgs {
