@@ -23,10 +23,13 @@ constexpr int kCellsPerWarp = kTile / kWarps;
 static_assert(kCellsPerWarp == kTileJ && kWarps == kTileI, "one warp per tile row");
 // Height bins a lane projects per chunk (chunk = lanes per cell * this).  The
 // projections of a chunk stay in registers (two of them cached per cell
-// group), so the forward, whose accumulators already fill the register file,
-// takes two; the backward, which holds dout instead, takes four.  Taller
-// grids take more chunks.
-constexpr int kZPerLaneFwd = 2;
+// group), and taller grids take more chunks.  The forward's accumulators
+// already fill the register file: fp32 slices with eight or more lanes per
+// cell take one bin per lane (two spill), bf16 slices and four-lane cells
+// take two (one is slower there).  The backward, which holds dout instead,
+// takes four.
+template <bool BF16, int L>
+constexpr int z_per_lane_fwd() { return (!BF16 && L >= 8) ? 1 : 2; }
 constexpr int kZPerLaneBwd = 4;
 constexpr int kZPerLaneMax = kZPerLaneBwd;
 // Merged-weight entries of one warp for one (camera, height chunk): the
