@@ -83,3 +83,31 @@ def test_two_gloo_ranks_shard_and_aggregate(tmp_path):
     assert res["rate"] == pytest.approx(2 * w.out_elems / 2e-3)
     s0, s1 = res["sums"]
     assert not np.allclose(s0, s1)                           # each rank transforms its own batch
+
+
+def test_recorded_traffic_names_known_kernels_and_sources():
+    """Every kernel in the committed traffic table maps to source files that
+    exist, so a stale entry is detected by its digest rather than by a crash;
+    entries whose digest matches the sources are returned, others are not."""
+    table = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for kernel, per_workload in table.items():
+        assert kernel in bench.KERNEL_SOURCES, kernel
+        for f in bench.KERNEL_SOURCES[kernel]:
+            assert os.path.exists(os.path.join(ROOT, "camera_bev_view_b200", "csrc", f)), f
+        for workload, entry in per_workload.items():
+            got = bench.recorded_traffic(kernel, workload)
+            if entry.get("source_digest") == bench.source_digest(kernel):
+                assert got == float(entry["dram_bytes_per_launch"]) and got > 0
+            else:
+                assert got is None
+
+
+@pytest.mark.parametrize("op,workload", [("ms", "ms_tiny"), ("deform", "deform_tiny"), ("lss", "lss_tiny")])
+def test_reference_arm_of_the_further_operators(op, workload):
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--op", op, "--impl", "reference",
+                        "--steps", "1", "--warmup", "0", "--workload", workload], capture_output=True, text=True,
+                       env=env, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
