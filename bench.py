@@ -102,14 +102,8 @@ def hbm_peak():
 
 
 KERNEL_SOURCES = {
-    "sample_forward_kernel": ["bev_forward.cu", "bev_forward.cuh", "bev_warp.cuh", "bev_kernels.cuh",
-                              "bev_geometry.cuh"],
-    "sample_backward_kernel": ["bev_backward.cu", "bev_backward.cuh", "bev_warp.cuh", "bev_kernels.cuh",
-                               "bev_geometry.cuh"],
-    "sample_forward_ms_kernel": ["bev_forward_ms.cu", "bev_forward.cuh", "bev_warp.cuh", "bev_kernels.cuh",
-                                 "bev_geometry.cuh"],
-    "sample_backward_ms_kernel": ["bev_backward_ms.cu", "bev_backward.cuh", "bev_warp.cuh", "bev_kernels.cuh",
-                                  "bev_geometry.cuh"],
+    "sample_forward_kernel": ["bev_forward.cu", "bev_tile.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
+    "sample_backward_kernel": ["bev_backward.cu", "bev_tile.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
     "deform_forward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
     "deform_backward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
     "lss_forward_kernel": ["bev_lss.cu", "bev_lss.cuh"],
@@ -841,7 +835,7 @@ def run_ms(args):
     bwd_bytes = elems * 4 + feat_bytes * 4
     dom = "forward" if stage_ms["forward"] >= stage_ms["backward"] else "backward"
     dom_bytes = fwd_bytes if dom == "forward" else bwd_bytes
-    kname = "sample_forward_ms_kernel" if dom == "forward" else "sample_backward_ms_kernel"
+    kname = "sample_forward_kernel" if dom == "forward" else "sample_backward_kernel"
     achieved = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
     lv = ",".join(f"{h}x{wl}" for h, wl in sizes)
     line = {

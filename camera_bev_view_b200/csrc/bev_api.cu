@@ -78,35 +78,6 @@ size_t backward_ws(int B, int N, int C, int Hf, int Wf) {
     return align_up((size_t)B * N * Hf * Wf * (size_t)round_up(C, 4) * sizeof(float));
 }
 
-// Lanes per cell L and 16-byte chunks per lane V (<= 8) for a slice of qs
-// chunks (qs <= 32).  Eight lanes per cell is preferred: each load
-// instruction then covers whole 128-byte lines of four cells, and each lane
-// keeps 2V packed accumulators busy per texel.  Wider or narrower groups are
-// used only when eight lanes would leave more than a fifth of the lanes idle.
-void pick_lanes(int qs, int* L, int* V) {
-    const int order[4] = {8, 16, 32, 4};
-    for (int k = 0; k < 4; ++k) {
-        const int l = order[k], v = (qs + l - 1) / l;
-        if (v <= 8 && 5 * (l * v - qs) <= l * v) {
-            *L = l;
-            *V = v;
-            return;
-        }
-    }
-    int best_l = 4, best_v = (qs + 3) / 4, best_waste = 1 << 30;
-    for (int k = 0; k < 4; ++k) {
-        const int l = order[k], v = (qs + l - 1) / l;
-        if (v > 8) continue;
-        if (l * v - qs < best_waste) {
-            best_waste = l * v - qs;
-            best_l = l;
-            best_v = v;
-        }
-    }
-    *L = best_l;
-    *V = best_v;
-}
-
 bev::GeoParams geo(const bev_grid_t* g, int Hf, int Wf, int img_h, int img_w) {
     bev::GeoParams p;
     p.xmin = g->xmin;
@@ -133,49 +104,29 @@ int cuda_status(cudaError_t e) {
     return BEV_ERR_CUDA;
 }
 
-// Backward tile width: kTileJ cells, or half that when kTileJ-wide tiles
-// would not fill two waves of resident CTAs (the launch would then end on a
-// short second wave of the heaviest, near-rig tiles).  Must be a multiple
-// of the 32 / L cells a warp works on at once.
-int backward_tile_j(int L, int X, int Y, int B, int slices, int sms) {
-    const long long slots = (long long)sms * bev::kCtasPerSmBwd;
-    const long long tiles = (long long)((X + bev::kTileI - 1) / bev::kTileI) *
-                            ((Y + bev::kTileJ - 1) / bev::kTileJ) * B * slices;
-    const int half = bev::kTileJ / 2;
-    return (tiles < 2 * slots && half % (32 / L) == 0) ? half : bev::kTileJ;
+// Channel slices of the dense kernels: each lane of a warp owns cpl
+// consecutive channels, so a CTA covers 32 * cpl channels of the Cp padded
+// channels per texel (4-, 8- or 16-byte loads per lane).  Fills a.cpl and
+// a.cpad and returns the number of slices.
+int channel_slices(bev::SampleArgs& a, bool bf16, int Cp) {
+    a.cpl = bf16 ? (Cp <= 64 ? 2 : 4) : (Cp <= 32 ? 1 : Cp <= 64 ? 2 : 4);
+    a.cpad = Cp;
+    return (Cp + 32 * a.cpl - 1) / (32 * a.cpl);
 }
 
-int sm_count(int dev, int* sms) {
-    if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *sms < 1)
-        return cuda_status(cudaErrorInvalidDevice);
-    return BEV_OK;
-}
-
-// Channel slices and lanes per cell for Cp channels in chunks of cpc
-// channels: fills a.Qtot, a.chan_per_chunk, a.slice_chunks and a.L, and
-// returns the chunks per lane V (0 when the slices exceed the grid limit).
-int channel_layout(bev::SampleArgs& a, int Cp, int cpc, int* slices) {
-    a.Qtot = Cp / cpc;
-    a.chan_per_chunk = cpc;
-    const int max_chunks = bev::kSliceMax / cpc;
-    *slices = (a.Qtot + max_chunks - 1) / max_chunks;
-    if (*slices > 65535) return 0;
-    a.slice_chunks = (a.Qtot + *slices - 1) / *slices;
-    int V;
-    pick_lanes(a.slice_chunks, &a.L, &V);
-    return V;
-}
-
-// Tiles of a launch.  Forward: 8x8 tiles, and when they fill fewer than two
-// waves of resident CTAs the launch would end on a short wave of the
-// heaviest, near-rig tiles, so every tile's cameras are split over two CTAs
-// that add into the zeroed output.  Backward: the width of backward_tile_j.
-void tile_layout(bev::SampleArgs& a, const bev_grid_t* grid, int B, int slices, int sms, bool backward) {
-    a.tile_j = backward ? backward_tile_j(a.L, grid->X, grid->Y, B, slices, sms) : bev::kTileJ;
+// 8x8 tiles of the grid.
+void tile_grid(bev::SampleArgs& a, const bev_grid_t* grid) {
     a.tiles_i = (grid->X + bev::kTileI - 1) / bev::kTileI;
-    a.tiles_j = (grid->Y + a.tile_j - 1) / a.tile_j;
-    const long long ctas = (long long)a.tiles_i * a.tiles_j * B * slices;
-    a.cam_split = !backward && ctas < 2LL * sms * bev::kCtasPerSm;
+    a.tiles_j = (grid->Y + bev::kTileJ - 1) / bev::kTileJ;
+}
+
+// A single-level table: the level is the feature map itself.
+void single_level(bev::SampleArgs& a, int Hf, int Wf, int img_h, int img_w) {
+    a.lv.n = 1;
+    a.lv.Hf[0] = Hf;
+    a.lv.Wf[0] = Wf;
+    a.lv.sW[0] = (float)Wf / (float)img_w;
+    a.lv.sH[0] = (float)Hf / (float)img_h;
 }
 
 }  // namespace
@@ -270,7 +221,6 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
     }
     bev::SampleArgs a;
     memset(&a, 0, sizeof(a));
-    a.feat = feat;
     a.K = intrinsics;
     a.E = ego2cam;
     a.out = out;
@@ -279,17 +229,13 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
     a.B = B;
     a.N = N;
     a.C = C;
-    int slices, sms;
-    const int V = channel_layout(a, Cp, cpc, &slices);
-    if (V == 0) return BEV_ERR_UNSUPPORTED;
-    if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
-    tile_layout(a, grid, B, slices, sms, false);
-    if (a.cam_split) {
-        if ((st = cuda_status(cudaMemsetAsync(out, 0, (size_t)B * C * grid->X * grid->Y * sizeof(float), s))) !=
-            BEV_OK)
-            return st;
-    }
-    return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, V, slices, s));
+    single_level(a, Hf, Wf, img_h, img_w);
+    a.lv.feat[0] = feat;
+    a.texel_bytes = Cp * elem_size(dtype);
+    a.out_vec = ((uintptr_t)out % 16) == 0 && (grid->Y % 4) == 0;
+    const int slices = channel_slices(a, dtype == BEV_BF16, Cp);
+    tile_grid(a, grid);
+    return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, slices, s));
 }
 
 BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, int Wf,
@@ -319,17 +265,15 @@ BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, 
     a.K = intrinsics;
     a.E = ego2cam;
     a.dout = dout;
-    a.dfeat = static_cast<float*>(workspace);
     a.g = geo(grid, Hf, Wf, img_h, img_w);
     a.B = B;
     a.N = N;
     a.C = C;
-    int slices, sms;
-    const int V = channel_layout(a, Cp, 4, &slices);
-    if (V == 0) return BEV_ERR_UNSUPPORTED;
-    if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
-    tile_layout(a, grid, B, slices, sms, true);
-    if ((st = cuda_status(bev_launch_backward(a, V, slices, s))) != BEV_OK) return st;
+    single_level(a, Hf, Wf, img_h, img_w);
+    a.lv.grad[0] = static_cast<float*>(workspace);
+    const int slices = channel_slices(a, false, Cp);
+    tile_grid(a, grid);
+    if ((st = cuda_status(bev_launch_backward(a, slices, s))) != BEV_OK) return st;
     return cuda_status(bev_launch_to_nchw(static_cast<const float*>(workspace), B * N, C, Hf * Wf, Cp,
                                           dfeatures, s));
 }
@@ -448,7 +392,6 @@ BEV_API int bev_sample_forward_multiscale(const void* const* features, int nleve
     }
     bev::SampleArgs a;
     memset(&a, 0, sizeof(a));
-    a.feat = base[0];
     a.K = intrinsics;
     a.E = ego2cam;
     a.out = out;
@@ -459,17 +402,11 @@ BEV_API int bev_sample_forward_multiscale(const void* const* features, int nleve
     a.B = B;
     a.N = N;
     a.C = C;
-    int slices, sms;
-    const int V = channel_layout(a, Cp, cpc, &slices);
-    if (V == 0) return BEV_ERR_UNSUPPORTED;
-    if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
-    tile_layout(a, grid, B, slices, sms, false);
-    if (a.cam_split) {
-        if ((st = cuda_status(cudaMemsetAsync(out, 0, (size_t)B * C * grid->X * grid->Y * sizeof(float), s))) !=
-            BEV_OK)
-            return st;
-    }
-    return cuda_status(bev_launch_forward_ms(a, dtype == BEV_BF16, V, slices, s));
+    a.texel_bytes = Cp * elem_size(dtype);
+    a.out_vec = ((uintptr_t)out % 16) == 0 && (grid->Y % 4) == 0;
+    const int slices = channel_slices(a, dtype == BEV_BF16, Cp);
+    tile_grid(a, grid);
+    return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, slices, s));
 }
 
 BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const int* Hf, const int* Wf, int B,
@@ -506,19 +443,15 @@ BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const
     a.K = intrinsics;
     a.E = ego2cam;
     a.dout = dout;
-    a.dfeat = static_cast<float*>(workspace);
     a.g = geo(grid, Hf[0], Wf[0], img_h, img_w);
     a.lv = level_table(nlevels, Hf, Wf, img_h, img_w);
     for (int l = 0; l < nlevels; ++l) a.lv.grad[l] = base[l];
     a.B = B;
     a.N = N;
     a.C = C;
-    int slices, sms;
-    const int V = channel_layout(a, Cp, 4, &slices);
-    if (V == 0) return BEV_ERR_UNSUPPORTED;
-    if ((st = sm_count(dev, &sms)) != BEV_OK) return st;
-    tile_layout(a, grid, B, slices, sms, true);
-    if ((st = cuda_status(bev_launch_backward_ms(a, V, slices, s))) != BEV_OK) return st;
+    const int slices = channel_slices(a, false, Cp);
+    tile_grid(a, grid);
+    if ((st = cuda_status(bev_launch_backward(a, slices, s))) != BEV_OK) return st;
     for (int l = 0; l < nlevels; ++l) {
         st = cuda_status(bev_launch_to_nchw(base[l], B * N, C, Hf[l] * Wf[l], Cp,
                                             dfeatures[l], s));
