@@ -271,6 +271,7 @@ BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, 
     a.C = C;
     single_level(a, Hf, Wf, img_h, img_w);
     a.lv.grad[0] = static_cast<float*>(workspace);
+    a.out_vec = ((uintptr_t)dout % 16) == 0 && (grid->Y % 4) == 0;
     const int slices = channel_slices(a, false, Cp);
     tile_grid(a, grid);
     if ((st = cuda_status(bev_launch_backward(a, slices, s))) != BEV_OK) return st;
@@ -446,6 +447,7 @@ BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const
     a.g = geo(grid, Hf[0], Wf[0], img_h, img_w);
     a.lv = level_table(nlevels, Hf, Wf, img_h, img_w);
     for (int l = 0; l < nlevels; ++l) a.lv.grad[l] = base[l];
+    a.out_vec = ((uintptr_t)dout % 16) == 0 && (grid->Y % 4) == 0;
     a.B = B;
     a.N = N;
     a.C = C;

@@ -47,23 +47,23 @@ __device__ __forceinline__ void load_tile(float (&v)[CPL], const float* t) {
     }
 }
 
-// Scatter of one group over its union box, two rows by two columns per step.
+// Scatter of one group over its union box, two rows by two columns per
+// step; weights [texel][member] with S per texel.
 template <int CPL, int G>
-__device__ __forceinline__ void backward_group(const TileSm& s, const Group& gp, float* gl, size_t rowf, int tf,
-                                               bool on, int lane) {
+__device__ __forceinline__ void backward_group(const TileSm& s, const Members& m, const float* wb, float* gl,
+                                               size_t rowf, int tf, bool on, int lane) {
     constexpr int S = G == 1 ? 1 : G == 2 ? 2 : G <= 4 ? 4 : 8;
     float d[G][CPL];
 #pragma unroll
-    for (int gg = 0; gg < G; ++gg) load_tile<CPL>(d[gg], s.tile + gp.cell[gg] * s.tile_stride + lane * CPL);
-    const int h = gp.h, w = gp.w;
-    const float* wb = s.wf + gp.off;
-    float* fb = gl + (size_t)gp.y0 * rowf + (size_t)gp.x0 * tf;
+    for (int gg = 0; gg < G; ++gg) load_tile<CPL>(d[gg], s.tile + m.cell[gg] * s.tile_stride + lane * CPL);
+    const int h = m.h, w = m.w;
+    float* fb = gl + (size_t)m.y0 * rowf + (size_t)m.x0 * tf;
     for (int c0 = 0; c0 < w; c0 += 2) {
-        const bool c1 = c0 + 1 < w;
+        const bool c1 = m.even || c0 + 1 < w;
         float* p = fb + (size_t)c0 * tf;
         const float* q = wb + c0 * S;
         for (int r0 = 0; r0 < h; r0 += 2, p += 2 * rowf, q += 2 * w * S) {
-            const bool r1 = r0 + 1 < h;
+            const bool r1 = m.even || r0 + 1 < h;
             const bool in[4] = {true, c1, r1, r1 && c1};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -87,62 +87,92 @@ __device__ __forceinline__ void backward_group(const TileSm& s, const Group& gp,
     }
 }
 
-// A group too large to merge: each member cell's valid bins, corner by
-// corner, with weight w / cnt.
+// Merge the members' weights in the warp's region, scatter, clear the region.
 template <int CPL>
-__device__ __noinline__ void backward_direct(const TileSm& s, int gi, int zc, int Hl, int Wl, float sW,
-                                             float sH, float* gl, size_t rowf, int tf, bool on, int lane) {
-    const Group& gp = s.grp[gi];
-    for (int m = 0; m < gp.n; ++m) {
-        const int cell = gp.cell[m];
-        float d[CPL];
-        load_tile<CPL>(d, s.tile + cell * s.tile_stride + lane * CPL);
-        for (int zz = 0; zz < zc; ++zz) {
-            const float2 uv = s.uv[cell * kZc + zz];
-            if (isnan(uv.x)) continue;
-            float fx, fy;
-            level_position(uv, sW, sH, fx, fy);
-            const Corners c = bilinear_corners(fx, fy);
-            const float rc = s.rc[cell * kZc + zz];
-            const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+__device__ __forceinline__ void backward_members(const TileSm& s, const Members& m, const GroupItems& it, int zc,
+                                                 int Hl, int Wl, float sW, float sH, float* gl, size_t rowf, int tf,
+                                                 bool on, int lane, unsigned* wh, unsigned* wl) {
+    merge_members(s, m, it, zc, Hl, Wl, sW, sH, wh, wl);
+    const float* wb = reinterpret_cast<const float*>(wh);
+    switch (m.n) {
+        case 1: backward_group<CPL, 1>(s, m, wb, gl, rowf, tf, on, lane); break;
+        case 2: backward_group<CPL, 2>(s, m, wb, gl, rowf, tf, on, lane); break;
+        case 3: backward_group<CPL, 3>(s, m, wb, gl, rowf, tf, on, lane); break;
+        case 4: backward_group<CPL, 4>(s, m, wb, gl, rowf, tf, on, lane); break;
+        case 5: backward_group<CPL, 5>(s, m, wb, gl, rowf, tf, on, lane); break;
+        case 6: backward_group<CPL, 6>(s, m, wb, gl, rowf, tf, on, lane); break;
+        case 7: backward_group<CPL, 7>(s, m, wb, gl, rowf, tf, on, lane); break;
+        default: backward_group<CPL, 8>(s, m, wb, gl, rowf, tf, on, lane); break;
+    }
+    clear_members(m, wh);
+}
+
+// A cell whose box does not fit a warp's region: its valid bins (lanes
+// 0 .. zc-1 of `one`, a one-cell projection), corner by corner, with weight
+// w / cnt.
+template <int CPL>
+__device__ __forceinline__ void backward_direct(const TileSm& s, const GroupItems& one, int cell, int zc, int Hl,
+                                                int Wl, float sW, float sH, float* gl, size_t rowf, int tf, bool on,
+                                                int lane) {
+    float d[CPL];
+    load_tile<CPL>(d, s.tile + cell * s.tile_stride + lane * CPL);
+    for (int zz = 0; zz < zc; ++zz) {
+        const float2 uv = make_float2(__shfl_sync(0xffffffffu, one.uv[0].x, zz), __shfl_sync(0xffffffffu, one.uv[0].y, zz));
+        if (isnan(uv.x)) continue;
+        float fx, fy;
+        level_position(uv, sW, sH, fx, fy);
+        const Corners c = bilinear_corners(fx, fy);
+        const float rc = s.rc[cell * kZc + zz];
+        const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
-                if ((unsigned)yy >= (unsigned)Hl || (unsigned)xx >= (unsigned)Wl) continue;
-                const float wk = __fmul_rn(ws[k], rc);
-                if (wk == 0.0f || !on) continue;
-                float v[CPL];
+        for (int k = 0; k < 4; ++k) {
+            const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
+            if ((unsigned)yy >= (unsigned)Hl || (unsigned)xx >= (unsigned)Wl) continue;
+            const float wk = __fmul_rn(ws[k], rc);
+            if (wk == 0.0f || !on) continue;
+            float v[CPL];
 #pragma unroll
-                for (int q = 0; q < CPL; ++q) v[q] = __fmul_rn(wk, d[q]);
-                red_add<CPL>(gl + (size_t)yy * rowf + (size_t)xx * tf, v);
-            }
+            for (int q = 0; q < CPL; ++q) v[q] = __fmul_rn(wk, d[q]);
+            red_add<CPL>(gl + (size_t)yy * rowf + (size_t)xx * tf, v);
         }
     }
 }
 
+// Warps take camera slot aa's groups in turn (largest first) until none is
+// left; each group is projected once and scattered on every level.
 template <int CPL>
-__device__ __forceinline__ void sweep_backward(const TileSm& s, int r, int zc, int Hl, int Wl, float sW, float sH,
-                                               float* gl, size_t rowf, int tf, bool on, int lane) {
-    const int rend = s.ctl[kCtlRstart + r + 1];
+__device__ __forceinline__ void sweep_backward(const SampleArgs& a, const TileSm& s, int aa, int b, int ti0, int tj0,
+                                               int z0, int zc, int c_base, bool on, int lane, int warp) {
+    unsigned* wh = s.wqh + warp * kWarpEntries;
+    unsigned* wl = s.wql + warp * kWarpEntries;
+    const int ng = s.ctl[kCtlGroups];
+    const int cam = s.ctl[kCtlActive + aa];
+    const int tf = a.cpad;  // floats per texel of the gradient buffers
     for (;;) {
-        int gi = 0;
-        if (lane == 0) gi = atomicAdd(&s.ctl[kCtlNext], 1);
-        gi = __shfl_sync(0xffffffffu, gi, 0);
-        if (gi >= rend) break;
-        const Group gp = s.grp[gi];
-        if (gp.direct) {
-            backward_direct<CPL>(s, gi, zc, Hl, Wl, sW, sH, gl, rowf, tf, on, lane);
-            continue;
-        }
-        switch (gp.n) {
-            case 1: backward_group<CPL, 1>(s, gp, gl, rowf, tf, on, lane); break;
-            case 2: backward_group<CPL, 2>(s, gp, gl, rowf, tf, on, lane); break;
-            case 3: backward_group<CPL, 3>(s, gp, gl, rowf, tf, on, lane); break;
-            case 4: backward_group<CPL, 4>(s, gp, gl, rowf, tf, on, lane); break;
-            case 5: backward_group<CPL, 5>(s, gp, gl, rowf, tf, on, lane); break;
-            case 6: backward_group<CPL, 6>(s, gp, gl, rowf, tf, on, lane); break;
-            case 7: backward_group<CPL, 7>(s, gp, gl, rowf, tf, on, lane); break;
-            default: backward_group<CPL, 8>(s, gp, gl, rowf, tf, on, lane); break;
+        int k = 0;
+        if (lane == 0) k = atomicAdd(&s.ctl[kCtlNext], 1);
+        k = __shfl_sync(0xffffffffu, k, 0);
+        if (k >= ng) break;
+        const Group& gp = s.grp[s.ctl[kCtlOrder + k]];
+        const GroupItems it = project_members(a, s, gp.cell, gp.n, cam, ti0, tj0, z0, zc);
+        for (int l = 0; l < a.lv.n; ++l) {
+            const int Hl = a.lv.Hf[l], Wl = a.lv.Wf[l];
+            const float sW = a.lv.sW[l], sH = a.lv.sH[l];
+            const size_t rowf = (size_t)Wl * tf;
+            float* gl = a.lv.grad[l] + ((size_t)b * a.N + cam) * Hl * rowf + c_base + lane * CPL;
+            const Members m = members_box(it, gp.cell, gp.n, Hl, Wl, sW, sH);
+            if (m.entries <= kWarpEntries) {
+                backward_members<CPL>(s, m, it, zc, Hl, Wl, sW, sH, gl, rowf, tf, on, lane, wh, wl);
+                continue;
+            }
+            for (int q = 0; q < gp.n; ++q) {  // too large together: cell by cell
+                const GroupItems one = project_members(a, s, gp.cell + q, 1, cam, ti0, tj0, z0, zc);
+                const Members m1 = members_box(one, gp.cell + q, 1, Hl, Wl, sW, sH);
+                if (m1.entries <= kWarpEntries)
+                    backward_members<CPL>(s, m1, one, zc, Hl, Wl, sW, sH, gl, rowf, tf, on, lane, wh, wl);
+                else
+                    backward_direct<CPL>(s, one, gp.cell[q], zc, Hl, Wl, sW, sH, gl, rowf, tf, on, lane);
+            }
         }
     }
 }
@@ -156,7 +186,10 @@ __global__ void __launch_bounds__(kThreads, kTileCtas) sample_backward_kernel(co
     const int c_base = blockIdx.z * 32 * CPL;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    for (int e = threadIdx.x; e < kEntries; e += kThreads) s.wq[e] = 0ull;
+    for (int e = 4 * threadIdx.x; e < kWarps * kWarpEntries; e += 4 * kThreads) {
+        *reinterpret_cast<uint4*>(s.wqh + e) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(s.wql + e) = make_uint4(0u, 0u, 0u, 0u);
+    }
     int ti0, tj0;
     locate_tile(a, s, b, ti0, tj0);
     cull_cameras(a, s, ti0, tj0);
@@ -164,55 +197,55 @@ __global__ void __launch_bounds__(kThreads, kTileCtas) sample_backward_kernel(co
     if (nA == 0) return;  // no camera sees the tile: nothing to add
 
     // dout of the tile: thread (channel, tile row) reads the row's 8 cells
-    // along y; absent cells and channels are 0.
-    const int nch = min(32 * CPL, a.C - c_base);
-    for (int idx = threadIdx.x; idx < 32 * CPL * kTileI; idx += kThreads) {
-        const int ci = idx / (32 * CPL), c = idx - ci * (32 * CPL);
-        const int i = ti0 + ci;
-        float v[kTileJ];
+    // along y (two 16-byte loads where dout allows); absent cells and
+    // channels are 0.  The loads are issued here and land in shared memory
+    // after the count pass, which hides their latency.
+    constexpr int SL = 32 * CPL;  // channels of a slice (a power of two)
+    constexpr int kIt = (SL * kTileI + kThreads - 1) / kThreads;
+    const int nch = min(SL, a.C - c_base);
+    float dv[kIt][kTileJ];
 #pragma unroll
-        for (int cj = 0; cj < kTileJ; ++cj) v[cj] = 0.0f;
-        if (c < nch && i < g.X) {
+    for (int it = 0; it < kIt; ++it) {
+        const int idx = threadIdx.x + it * kThreads;
+        const int c = idx & (SL - 1), i = ti0 + idx / SL;
+#pragma unroll
+        for (int cj = 0; cj < kTileJ; ++cj) dv[it][cj] = 0.0f;
+        if (idx < SL * kTileI && c < nch && i < g.X) {
             const float* dp = a.dout + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0;
+            if (a.out_vec && tj0 + kTileJ <= g.Y) {
 #pragma unroll
-            for (int cj = 0; cj < kTileJ; ++cj)
-                if (tj0 + cj < g.Y) v[cj] = __ldg(dp + cj);
+                for (int q = 0; q < kTileJ / 4; ++q) {
+                    const float4 u4 = __ldg(reinterpret_cast<const float4*>(dp) + q);
+                    dv[it][4 * q] = u4.x; dv[it][4 * q + 1] = u4.y; dv[it][4 * q + 2] = u4.z; dv[it][4 * q + 3] = u4.w;
+                }
+            } else {
+#pragma unroll
+                for (int cj = 0; cj < kTileJ; ++cj)
+                    if (tj0 + cj < g.Y) dv[it][cj] = __ldg(dp + cj);
+            }
         }
-        float* tp = s.tile + ci * kTileJ * s.tile_stride + c;
-#pragma unroll
-        for (int cj = 0; cj < kTileJ; ++cj) tp[cj * s.tile_stride] = v[cj];
     }
     const bool on = c_base + lane * CPL < a.cpad;
-    const int tf = a.cpad;  // floats per texel of the gradient buffers
 
     for (int z0 = 0; z0 < g.Z; z0 += kZc) {
         const int zc = min(kZc, g.Z - z0);
         count_pass(a, s, b, ti0, tj0, z0, zc, false);
+        if (z0 == 0) {
+#pragma unroll
+            for (int it = 0; it < kIt; ++it) {
+                const int idx = threadIdx.x + it * kThreads;
+                if (idx >= SL * kTileI) break;
+                float* tp = s.tile + (idx / SL) * kTileJ * s.tile_stride + (idx & (SL - 1));
+#pragma unroll
+                for (int cj = 0; cj < kTileJ; ++cj) tp[cj * s.tile_stride] = dv[it][cj];
+            }
+        }
         __syncthreads();
         for (int aa = 0; aa < nA; ++aa) {
-            project_pass(a, s, ti0, tj0, z0, zc, aa);
+            if (warp == 0) form_groups(s, s.xlo + aa * kCells);
             __syncthreads();
-            const int cam = s.ctl[kCtlActive + aa];
-            for (int l = 0; l < a.lv.n; ++l) {
-                const int Hl = a.lv.Hf[l], Wl = a.lv.Wf[l];
-                const float sW = a.lv.sW[l], sH = a.lv.sH[l];
-                box_pass(s, zc, Hl, Wl, sW, sH);
-                __syncthreads();
-                if (warp == 0) form_groups(s);
-                __syncthreads();
-                const int nr = s.ctl[kCtlRounds];
-                const size_t rowf = (size_t)Wl * tf;
-                float* gl = a.lv.grad[l] + ((size_t)b * a.N + cam) * Hl * rowf + c_base + lane * CPL;
-                for (int r = 0; r < nr; ++r) {
-                    merge_pass(s, zc, Hl, Wl, sW, sH, r);
-                    __syncthreads();
-                    convert_pass(s, r);
-                    if (threadIdx.x == 0) s.ctl[kCtlNext] = s.ctl[kCtlRstart + r];
-                    __syncthreads();
-                    sweep_backward<CPL>(s, r, zc, Hl, Wl, sW, sH, gl, rowf, tf, on, lane);
-                }
-                __syncthreads();
-            }
+            sweep_backward<CPL>(a, s, aa, b, ti0, tj0, z0, zc, c_base, on, lane, warp);
+            __syncthreads();
         }
     }
 }

@@ -19,46 +19,82 @@
 
 namespace bev {
 
-// Sweep of one group's union box, two rows by two columns per step.
-template <bool BF16, int CPL, int G>
-__device__ __forceinline__ void gather_group(float (&acc)[G][CPL], const Group& gp, const float* wf,
-                                             const unsigned char* fl, size_t rowb, int tb, bool on) {
+// Sweep of one group's union box, two rows by two columns per step; weights
+// [texel][member] with S per texel.  An even box needs no edge predicates;
+// lanes past the slice's channels load channel 0 (harmless, never stored).
+template <bool BF16, int CPL, int G, bool EVEN>
+__device__ __forceinline__ void gather_walk(float (&acc)[G][CPL], const Members& m, const float* wb,
+                                            const unsigned char* fl, size_t rowb, int tb) {
     constexpr int S = G == 1 ? 1 : G == 2 ? 2 : G <= 4 ? 4 : 8;
-    const int h = gp.h, w = gp.w;
-    const float* wb = wf + gp.off;
-    const unsigned char* fb = fl + (size_t)gp.y0 * rowb + (size_t)gp.x0 * tb;
+    const int h = m.h, w = m.w;
+    const unsigned char* fb = fl + (size_t)m.y0 * rowb + (size_t)m.x0 * tb;
     for (int c0 = 0; c0 < w; c0 += 2) {
-        const bool c1 = c0 + 1 < w;
+        const bool c1 = EVEN || c0 + 1 < w;
         const unsigned char* p = fb + (size_t)c0 * tb;
         const float* q = wb + c0 * S;
-        for (int r0 = 0; r0 < h; r0 += 2, p += 2 * rowb, q += 2 * w * S) {
-            const bool r1 = r0 + 1 < h;
-            const bool in[4] = {true, c1, r1, r1 && c1};
+        if constexpr (EVEN && G * CPL <= 0) {
+            // two rows by two columns per step; the next step's texels are
+            // loaded before this step's FMAs, so two steps of loads are in
+            // flight per warp (where the accumulators leave room for them)
             LaneVec<BF16, CPL> d[4];
-            float wt[4][S];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (in[u]) {
-                    load_weights<S>(wt[u], q + ((u >> 1) * w + (u & 1)) * S);
-                } else {
+            for (int u = 0; u < 4; ++u) d[u].load(p + (u >> 1) * rowb + (u & 1) * tb);
+            for (int r0 = 0; r0 < h; r0 += 2, p += 2 * rowb, q += 2 * w * S) {
+                LaneVec<BF16, CPL> nx[4];
+                if (r0 + 2 < h) {
 #pragma unroll
-                    for (int k = 0; k < S; ++k) wt[u][k] = 0.0f;
+                    for (int u = 0; u < 4; ++u) nx[u].load(p + (2 + (u >> 1)) * rowb + (u & 1) * tb);
                 }
-                if (in[u] && on)
-                    d[u].load(p + (u >> 1) * rowb + (u & 1) * tb);
-                else
-                    d[u].zero();
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float wt[S];
+                    load_weights<S>(wt, q + ((u >> 1) * w + (u & 1)) * S);
+                    float v[CPL];
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) v[c] = d[u].get(c);
+#pragma unroll
+                    for (int gg = 0; gg < G; ++gg) fma_lane<CPL>(acc[gg], wt[gg], v);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) d[u] = nx[u];
             }
+        } else {
+            for (int r0 = 0; r0 < h; r0 += 2, p += 2 * rowb, q += 2 * w * S) {
+                const bool r1 = EVEN || r0 + 1 < h;
+                const bool in[4] = {true, c1, r1, r1 && c1};
+                LaneVec<BF16, CPL> d[4];
+                float wt[4][S];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float v[CPL];
+                for (int u = 0; u < 4; ++u) {
+                    if (in[u]) {
+                        load_weights<S>(wt[u], q + ((u >> 1) * w + (u & 1)) * S);
+                        d[u].load(p + (u >> 1) * rowb + (u & 1) * tb);
+                    } else {
 #pragma unroll
-                for (int c = 0; c < CPL; ++c) v[c] = d[u].get(c);
+                        for (int k = 0; k < S; ++k) wt[u][k] = 0.0f;
+                        d[u].zero();
+                    }
+                }
 #pragma unroll
-                for (int gg = 0; gg < G; ++gg) fma_lane<CPL>(acc[gg], wt[u][gg], v);
+                for (int u = 0; u < 4; ++u) {
+                    float v[CPL];
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) v[c] = d[u].get(c);
+#pragma unroll
+                    for (int gg = 0; gg < G; ++gg) fma_lane<CPL>(acc[gg], wt[u][gg], v);
+                }
             }
         }
     }
+}
+
+template <bool BF16, int CPL, int G>
+__device__ __forceinline__ void gather_members(float (&acc)[G][CPL], const Members& m, const float* wb,
+                                               const unsigned char* fl, size_t rowb, int tb) {
+    if (m.even)
+        gather_walk<BF16, CPL, G, true>(acc, m, wb, fl, rowb, tb);
+    else
+        gather_walk<BF16, CPL, G, false>(acc, m, wb, fl, rowb, tb);
 }
 
 // Add a lane's channels of one cell into the output tile.
@@ -78,83 +114,110 @@ __device__ __forceinline__ void add_to_tile(float* t, const float (&v)[CPL]) {
 }
 
 template <bool BF16, int CPL, int G>
-__device__ __forceinline__ void forward_group(const TileSm& s, const Group& gp, const unsigned char* fl, size_t rowb,
-                                              int tb, bool on, int lane) {
+__device__ __forceinline__ void forward_group(const TileSm& s, const Members& m, const float* wb,
+                                              const unsigned char* fl, size_t rowb, int tb, bool on, int lane) {
     float acc[G][CPL];
 #pragma unroll
     for (int gg = 0; gg < G; ++gg)
 #pragma unroll
         for (int c = 0; c < CPL; ++c) acc[gg][c] = 0.0f;
-    gather_group<BF16, CPL, G>(acc, gp, s.wf, fl, rowb, tb, on);
+    gather_members<BF16, CPL, G>(acc, m, wb, fl, rowb, tb);
     if (on) {
 #pragma unroll
-        for (int gg = 0; gg < G; ++gg) add_to_tile<CPL>(s.tile + gp.cell[gg] * s.tile_stride + lane * CPL, acc[gg]);
+        for (int gg = 0; gg < G; ++gg) add_to_tile<CPL>(s.tile + m.cell[gg] * s.tile_stride + lane * CPL, acc[gg]);
     }
 }
 
-// A group too large to merge: each member cell's valid bins, corner by
-// corner, with weight w / cnt.
+// Merge the members' weights in the warp's region, sweep, clear the region.
 template <bool BF16, int CPL>
-__device__ __noinline__ void forward_direct(const TileSm& s, int gi, int zc, int Hl, int Wl, float sW,
-                                            float sH, const unsigned char* fl, size_t rowb, int tb, bool on,
-                                            int lane) {
-    const Group& gp = s.grp[gi];
-    for (int m = 0; m < gp.n; ++m) {
-        const int cell = gp.cell[m];
-        float acc[CPL];
+__device__ __forceinline__ void forward_members(const TileSm& s, const Members& m, const GroupItems& it, int zc,
+                                                int Hl, int Wl, float sW, float sH, const unsigned char* fl,
+                                                size_t rowb, int tb, bool on, int lane, unsigned* wh, unsigned* wl) {
+    merge_members(s, m, it, zc, Hl, Wl, sW, sH, wh, wl);
+    const float* wb = reinterpret_cast<const float*>(wh);
+    switch (m.n) {
+        case 1: forward_group<BF16, CPL, 1>(s, m, wb, fl, rowb, tb, on, lane); break;
+        case 2: forward_group<BF16, CPL, 2>(s, m, wb, fl, rowb, tb, on, lane); break;
+        case 3: forward_group<BF16, CPL, 3>(s, m, wb, fl, rowb, tb, on, lane); break;
+        case 4: forward_group<BF16, CPL, 4>(s, m, wb, fl, rowb, tb, on, lane); break;
+        case 5: forward_group<BF16, CPL, 5>(s, m, wb, fl, rowb, tb, on, lane); break;
+        case 6: forward_group<BF16, CPL, 6>(s, m, wb, fl, rowb, tb, on, lane); break;
+        case 7: forward_group<BF16, CPL, 7>(s, m, wb, fl, rowb, tb, on, lane); break;
+        default: forward_group<BF16, CPL, 8>(s, m, wb, fl, rowb, tb, on, lane); break;
+    }
+    clear_members(m, wh);
+}
+
+// A cell whose box does not fit a warp's region: its valid bins (lanes
+// 0 .. zc-1 of `one`, a one-cell projection), corner by corner, with weight
+// w / cnt.
+template <bool BF16, int CPL>
+__device__ __forceinline__ void forward_direct(const TileSm& s, const GroupItems& one, int cell, int zc, int Hl,
+                                               int Wl, float sW, float sH, const unsigned char* fl, size_t rowb,
+                                               int tb, bool on, int lane) {
+    float acc[CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[c] = 0.0f;
-        for (int zz = 0; zz < zc; ++zz) {
-            const float2 uv = s.uv[cell * kZc + zz];
-            if (isnan(uv.x)) continue;
-            float fx, fy;
-            level_position(uv, sW, sH, fx, fy);
-            const Corners c = bilinear_corners(fx, fy);
-            const float rc = s.rc[cell * kZc + zz];
-            const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+    for (int c = 0; c < CPL; ++c) acc[c] = 0.0f;
+    for (int zz = 0; zz < zc; ++zz) {
+        const float2 uv = make_float2(__shfl_sync(0xffffffffu, one.uv[0].x, zz), __shfl_sync(0xffffffffu, one.uv[0].y, zz));
+        if (isnan(uv.x)) continue;
+        float fx, fy;
+        level_position(uv, sW, sH, fx, fy);
+        const Corners c = bilinear_corners(fx, fy);
+        const float rc = s.rc[cell * kZc + zz];
+        const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
-                if ((unsigned)yy >= (unsigned)Hl || (unsigned)xx >= (unsigned)Wl) continue;
-                LaneVec<BF16, CPL> d;
-                if (on)
-                    d.load(fl + (size_t)yy * rowb + (size_t)xx * tb);
-                else
-                    d.zero();
-                float v[CPL];
+        for (int k = 0; k < 4; ++k) {
+            const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
+            if ((unsigned)yy >= (unsigned)Hl || (unsigned)xx >= (unsigned)Wl) continue;
+            LaneVec<BF16, CPL> d;
+            d.load(fl + (size_t)yy * rowb + (size_t)xx * tb);
+            float v[CPL];
 #pragma unroll
-                for (int q = 0; q < CPL; ++q) v[q] = d.get(q);
-                fma_lane<CPL>(acc, __fmul_rn(ws[k], rc), v);
-            }
+            for (int q = 0; q < CPL; ++q) v[q] = d.get(q);
+            fma_lane<CPL>(acc, __fmul_rn(ws[k], rc), v);
         }
-        if (on) add_to_tile<CPL>(s.tile + cell * s.tile_stride + lane * CPL, acc);
     }
+    if (on) add_to_tile<CPL>(s.tile + cell * s.tile_stride + lane * CPL, acc);
 }
 
-// Warps take the groups of round r in turn until none is left.
+// Warps take camera slot aa's groups in turn (largest first) until none is
+// left; each group is projected once and swept on every level.
 template <bool BF16, int CPL>
-__device__ __forceinline__ void sweep_forward(const TileSm& s, int r, int zc, int Hl, int Wl, float sW, float sH,
-                                              const unsigned char* fl, size_t rowb, int tb, bool on, int lane) {
-    const int rend = s.ctl[kCtlRstart + r + 1];
+__device__ __forceinline__ void sweep_forward(const SampleArgs& a, const TileSm& s, int aa, int b, int ti0, int tj0,
+                                              int z0, int zc, int lane_c, bool on, int lane, int warp) {
+    constexpr int esize = BF16 ? 2 : 4;
+    unsigned* wh = s.wqh + warp * kWarpEntries;
+    unsigned* wl = s.wql + warp * kWarpEntries;
+    const int ng = s.ctl[kCtlGroups];
+    const int cam = s.ctl[kCtlActive + aa];
+    const int tb = a.texel_bytes;
     for (;;) {
-        int gi = 0;
-        if (lane == 0) gi = atomicAdd(&s.ctl[kCtlNext], 1);
-        gi = __shfl_sync(0xffffffffu, gi, 0);
-        if (gi >= rend) break;
-        const Group gp = s.grp[gi];
-        if (gp.direct) {
-            forward_direct<BF16, CPL>(s, gi, zc, Hl, Wl, sW, sH, fl, rowb, tb, on, lane);
-            continue;
-        }
-        switch (gp.n) {
-            case 1: forward_group<BF16, CPL, 1>(s, gp, fl, rowb, tb, on, lane); break;
-            case 2: forward_group<BF16, CPL, 2>(s, gp, fl, rowb, tb, on, lane); break;
-            case 3: forward_group<BF16, CPL, 3>(s, gp, fl, rowb, tb, on, lane); break;
-            case 4: forward_group<BF16, CPL, 4>(s, gp, fl, rowb, tb, on, lane); break;
-            case 5: forward_group<BF16, CPL, 5>(s, gp, fl, rowb, tb, on, lane); break;
-            case 6: forward_group<BF16, CPL, 6>(s, gp, fl, rowb, tb, on, lane); break;
-            case 7: forward_group<BF16, CPL, 7>(s, gp, fl, rowb, tb, on, lane); break;
-            default: forward_group<BF16, CPL, 8>(s, gp, fl, rowb, tb, on, lane); break;
+        int k = 0;
+        if (lane == 0) k = atomicAdd(&s.ctl[kCtlNext], 1);
+        k = __shfl_sync(0xffffffffu, k, 0);
+        if (k >= ng) break;
+        const Group& gp = s.grp[s.ctl[kCtlOrder + k]];
+        const GroupItems it = project_members(a, s, gp.cell, gp.n, cam, ti0, tj0, z0, zc);
+        for (int l = 0; l < a.lv.n; ++l) {
+            const int Hl = a.lv.Hf[l], Wl = a.lv.Wf[l];
+            const float sW = a.lv.sW[l], sH = a.lv.sH[l];
+            const size_t rowb = (size_t)Wl * tb;
+            const unsigned char* fl = static_cast<const unsigned char*>(a.lv.feat[l]) +
+                                      ((size_t)b * a.N + cam) * Hl * rowb + (size_t)lane_c * esize;
+            const Members m = members_box(it, gp.cell, gp.n, Hl, Wl, sW, sH);
+            if (m.entries <= kWarpEntries) {
+                forward_members<BF16, CPL>(s, m, it, zc, Hl, Wl, sW, sH, fl, rowb, tb, on, lane, wh, wl);
+                continue;
+            }
+            for (int q = 0; q < gp.n; ++q) {  // too large together: cell by cell
+                const GroupItems one = project_members(a, s, gp.cell + q, 1, cam, ti0, tj0, z0, zc);
+                const Members m1 = members_box(one, gp.cell + q, 1, Hl, Wl, sW, sH);
+                if (m1.entries <= kWarpEntries)
+                    forward_members<BF16, CPL>(s, m1, one, zc, Hl, Wl, sW, sH, fl, rowb, tb, on, lane, wh, wl);
+                else
+                    forward_direct<BF16, CPL>(s, one, gp.cell[q], zc, Hl, Wl, sW, sH, fl, rowb, tb, on, lane);
+            }
         }
     }
 }
@@ -169,66 +232,51 @@ __global__ void __launch_bounds__(kThreads, kTileCtas) sample_forward_kernel(con
     const int b = blockIdx.y;
     const int c_base = blockIdx.z * 32 * CPL;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int esize = BF16 ? 2 : 4;
 
-    for (int e = threadIdx.x; e < kEntries; e += kThreads) s.wq[e] = 0ull;
-    for (int e = threadIdx.x; e < kCells * s.tile_stride; e += kThreads) s.tile[e] = 0.0f;
+    for (int e = 4 * threadIdx.x; e < kWarps * kWarpEntries; e += 4 * kThreads) {
+        *reinterpret_cast<uint4*>(s.wqh + e) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(s.wql + e) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int e = 4 * threadIdx.x; e < kCells * s.tile_stride; e += 4 * kThreads)
+        *reinterpret_cast<float4*>(s.tile + e) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     int ti0, tj0;
     locate_tile(a, s, b, ti0, tj0);
     cull_cameras(a, s, ti0, tj0);
     const int nA = s.ctl[kCtlNA];
     const bool on = c_base + lane * CPL < a.cpad;
+    const int lane_c = on ? c_base + lane * CPL : c_base;  // lanes past the channels read channel c_base
     const bool write_count = a.count != nullptr && blockIdx.z == 0;
-    const int tb = a.texel_bytes;
 
     for (int z0 = 0; z0 < g.Z; z0 += kZc) {
         const int zc = min(kZc, g.Z - z0);
         count_pass(a, s, b, ti0, tj0, z0, zc, write_count);
         __syncthreads();
         for (int aa = 0; aa < nA; ++aa) {
-            project_pass(a, s, ti0, tj0, z0, zc, aa);
+            if (warp == 0) form_groups(s, s.xlo + aa * kCells);
             __syncthreads();
-            const int cam = s.ctl[kCtlActive + aa];
-            for (int l = 0; l < a.lv.n; ++l) {
-                const int Hl = a.lv.Hf[l], Wl = a.lv.Wf[l];
-                const float sW = a.lv.sW[l], sH = a.lv.sH[l];
-                box_pass(s, zc, Hl, Wl, sW, sH);
-                __syncthreads();
-                if (warp == 0) form_groups(s);
-                __syncthreads();
-                const int nr = s.ctl[kCtlRounds];
-                const size_t rowb = (size_t)Wl * tb;
-                const unsigned char* fl = static_cast<const unsigned char*>(a.lv.feat[l]) +
-                                          ((size_t)b * a.N + cam) * Hl * rowb + (size_t)(c_base + lane * CPL) * esize;
-                for (int r = 0; r < nr; ++r) {
-                    merge_pass(s, zc, Hl, Wl, sW, sH, r);
-                    __syncthreads();
-                    convert_pass(s, r);
-                    if (threadIdx.x == 0) s.ctl[kCtlNext] = s.ctl[kCtlRstart + r];
-                    __syncthreads();
-                    sweep_forward<BF16, CPL>(s, r, zc, Hl, Wl, sW, sH, fl, rowb, tb, on, lane);
-                }
-                __syncthreads();
-            }
+            sweep_forward<BF16, CPL>(a, s, aa, b, ti0, tj0, z0, zc, lane_c, on, lane, warp);
+            __syncthreads();
         }
     }
     __syncthreads();
 
     // Store: each thread takes (channel, tile row) pairs and writes the row's
     // 8 cells along y (two 16-byte stores where out allows).
-    const int nch = min(32 * CPL, a.C - c_base);
-    for (int idx = threadIdx.x; idx < nch * kTileI; idx += kThreads) {
-        const int ci = idx / nch, c = idx - ci * nch;
+    constexpr int SL = 32 * CPL;  // channels of a slice (a power of two)
+    const int nch = min(SL, a.C - c_base);
+    for (int idx = threadIdx.x; idx < SL * kTileI; idx += kThreads) {
+        const int c = idx & (SL - 1), ci = idx / SL;
         const int i = ti0 + ci;
-        if (i >= g.X) continue;
+        if (c >= nch || i >= g.X) continue;
         const float* tp = s.tile + ci * kTileJ * s.tile_stride + c;
         float v[kTileJ];
 #pragma unroll
         for (int cj = 0; cj < kTileJ; ++cj) v[cj] = tp[cj * s.tile_stride];
         float* op = a.out + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0;
         if (a.out_vec && tj0 + kTileJ <= g.Y) {
-            *reinterpret_cast<float4*>(op) = make_float4(v[0], v[1], v[2], v[3]);
-            *reinterpret_cast<float4*>(op + 4) = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+            for (int q = 0; q < kTileJ / 4; ++q)
+                *reinterpret_cast<float4*>(op + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         } else {
 #pragma unroll
             for (int cj = 0; cj < kTileJ; ++cj)

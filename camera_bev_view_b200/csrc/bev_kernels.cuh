@@ -16,6 +16,7 @@ constexpr int kTileI = 8;
 constexpr int kTileJ = 8;
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+static_assert(kTileJ % 4 == 0, "tile rows are stored as 16-byte vectors");
 
 // Feature-pyramid levels.  Every level shares the voxel's projection,
 // validity and count; level l samples its own map at its own scale.  The
@@ -41,7 +42,7 @@ struct SampleArgs {
     int cpl;                // channels per lane: a channel slice is 32 * cpl channels
     int cpad;               // channels per texel in the channels-last buffers (padded)
     int texel_bytes;        // forward: bytes per texel of the channels-last features
-    int out_vec;            // forward: out is 16-byte aligned and Y % 4 == 0
+    int out_vec;            // out (forward) / dout (backward) is 16-byte aligned and Y % 4 == 0
     int tiles_i, tiles_j;   // tiles along X and Y
     LevelTable lv;          // feature levels
 };

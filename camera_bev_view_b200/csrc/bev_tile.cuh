@@ -8,29 +8,31 @@
 // item and one channel slice, and works camera by camera:
 //
 //   count    every (cell, height bin) voxel of the tile is tested against
-//            every camera that can see the tile; the valid cameras per bin
-//            give the mean's 1 / cnt.
-//   project  per camera, the image-plane position (u, v) of every voxel the
-//            camera sees, in the fixed fp32 order of the public header.
-//   boxes    per camera and feature level, the texel box each cell's valid
-//            samples touch (bilinear corners inside the map).
-//   groups   cells whose boxes start at the same feature column are grouped,
-//            up to kGmax at a time.  A vertical column of voxels projects to
-//            a near-vertical segment, so cells of one group share nearly all
-//            of their texels (the union box is ~94% filled on the seeded
-//            rigs): a texel's channel vector is then loaded once for the
-//            whole group and applied to every member cell from registers.
-//   merge    the bilinear weights w / cnt of all bins of a cell are summed
-//            per (cell, texel) into a dense [texel][slot] array per group,
-//            with integer atomics on an exact 2^-40 fixed point (order of the
-//            additions does not matter), then rounded once to fp32.
-//   sweep    warps take groups in turn and walk each union box once (the
-//            forward gathers, the backward scatters).
+//            every camera that can see the tile (exactly as the fixed fp32
+//            order of the public header decides it); the valid cameras per
+//            bin give the mean's 1 / cnt.  The same pass notes, per camera,
+//            the leftmost feature column each cell's valid voxels reach.
+//   groups   per camera, cells whose voxels start at the same feature column
+//            are grouped, up to kGmax at a time.  A vertical column of voxels
+//            projects to a near-vertical segment, so cells of one group share
+//            nearly all of their texels (the union box is ~94% filled on the
+//            seeded rigs): a texel's channel vector is then loaded once for
+//            the whole group and applied to every member cell from registers.
+//   sweep    warps take groups in turn, largest first.  For its group a warp
+//            projects the members' voxels exactly (image-plane positions held
+//            in registers), bounds their texels, sums the bilinear weights
+//            w / cnt of the members' bins per
+//            (cell, texel) into a dense [texel][member] array of its own
+//            shared-memory region -- 32-bit integer atomics on an exact fixed
+//            point split in two words (2^-20 and 2^-40), so the order of the
+//            additions does not matter -- rounds them once to fp32, and walks
+//            the union box once (the forward gathers, the backward scatters).
 //
-// A group's merged weights that would not fit the shared-memory budget go
-// in further rounds; a group whose box alone is too large for a round is
-// swept bin by bin instead ("direct").  Every step is deterministic except
-// the order of the backward's global reductions.
+// A group whose merged weights would not fit the warp's region is taken
+// cell by cell; a cell whose box alone does not fit is swept bin by bin
+// ("direct").  With several feature levels, a group is swept level by
+// level on the same projections.  Every step is deterministic except the order of the
+// backward's global reductions.
 #pragma once
 
 #include <limits.h>
@@ -43,21 +45,17 @@ namespace bev {
 constexpr int kCells = kTileI * kTileJ;  // cell = ci * kTileJ + cj
 constexpr int kZc = 16;                  // height bins per chunk of the count
 constexpr int kGmax = 8;                 // cells per group
-constexpr int kEntries = 2048;           // merged-weight entries per round
+constexpr int kWarpEntries = 512;        // merged-weight entries of a warp's region
 constexpr int kTileCtas = 2;             // CTAs per SM
+constexpr int kMaxActive = 32;           // active cameras of a tile (at most BEV_MAX_CAMERAS)
 static_assert(kThreads == 256 && kCells == 64, "the tile machinery assumes 256 threads and 64 cells");
 
 struct Group {
-    int y0, x0, h, w;  // union box of the member cells' texel boxes
-    int off;           // first fp32 weight of the group in its round
-    int n;             // member cells, 1 .. kGmax
-    int slots;         // weights stored per texel: 1, 2, 4 or 8 (>= n)
-    int round;         // merge round
-    int direct;        // 1: swept bin by bin (box too large for a round)
-    int pad[3];
-    unsigned char cell[kGmax];
+    int n;                     // member cells, 1 .. kGmax
+    unsigned char cell[kGmax];  // member cell indices
+    int pad;
 };
-static_assert(sizeof(Group) == 56, "group descriptor size");
+static_assert(sizeof(Group) == 16, "group descriptor size");
 
 // Control words (ints) of the CTA.
 enum {
@@ -65,20 +63,18 @@ enum {
     kCtlNA = 32,       // number of active cameras
     kCtlOrigin = 40,   // [40, 41] tile origin
     kCtlGroups = 48,   // groups of the current view
-    kCtlRounds = 49,   // merge rounds of the current view
     kCtlNext = 50,     // next group to sweep (warps take groups in turn)
+    kCtlSizeHist = 52, // [52, 61) groups per size, then per-size cursors
     kCtlCull = 64,     // [64, 96) per-camera visibility flags of the cull
-    kCtlRstart = 128,  // [128, 128 + 65) first group of each round
-    kCtlNent = 208,    // [208, 208 + 64) weight entries of each round
-    kCtlBucket = 288,  // [288, 352) per-column bucket counters
-    kCtlGbase = 352,   // [352, 416) first group of each bucket
-    kCtlBounds = 416,  // [416, 416 + 4 * 64) union bounds while grouping
-    kCtlWords = 672,
+    kCtlOrder = 96,    // [96, 160) groups, largest first
+    kCtlBucket = 160,  // [160, 224) per-column bucket counters
+    kCtlGbase = 224,   // [224, 288) first group of each bucket
+    kCtlWords = 288,
 };
 
 // Byte offsets of the CTA's shared-memory regions.  cpl = channels per lane.
 struct TileLayout {
-    size_t cams, ctl, rc, vmask, uv, box, cellg, grp, wq, wf, tile, total;
+    size_t cams, ctl, rc, xlo, grp, wqh, wql, tile, total;
     int tile_stride;  // floats per cell row of the [cell][channel] tile
 };
 
@@ -93,13 +89,10 @@ __host__ __device__ inline TileLayout tile_layout(int N, int cpl) {
     l.cams = take(sizeof(float) * N * kCamFloats);
     l.ctl = take(sizeof(int) * kCtlWords);
     l.rc = take(sizeof(float) * kCells * kZc);
-    l.vmask = take(sizeof(unsigned) * kCells * kZc);
-    l.uv = take(sizeof(float2) * kCells * kZc);
-    l.box = take(sizeof(unsigned) * 2 * kCells);
-    l.cellg = take(sizeof(int) * kCells);
+    l.xlo = take(sizeof(unsigned short) * kMaxActive * kCells);
     l.grp = take(sizeof(Group) * kCells);
-    l.wq = take(sizeof(unsigned long long) * kEntries);
-    l.wf = take(sizeof(float) * kEntries);
+    l.wqh = take(sizeof(unsigned) * kWarps * kWarpEntries);
+    l.wql = take(sizeof(unsigned) * kWarps * kWarpEntries);
     l.tile_stride = 32 * cpl + 4;
     l.tile = take(sizeof(float) * kCells * l.tile_stride);
     l.total = b;
@@ -109,14 +102,11 @@ __host__ __device__ inline TileLayout tile_layout(int N, int cpl) {
 struct TileSm {
     float* cams;
     int* ctl;
-    float* rc;
-    unsigned* vmask;
-    float2* uv;
-    unsigned* box;
-    int* cellg;
+    float* rc;            // [cell * kZc + bin]: 1 / cnt (0 when no camera sees the voxel)
+    unsigned short* xlo;  // [active camera][cell]: leftmost level-0 column of its valid voxels (0xffff: none)
     Group* grp;
-    unsigned long long* wq;
-    float* wf;
+    unsigned* wqh;   // per warp: merge words in 2^-20 units, then the fp32 weights
+    unsigned* wql;   // per warp: merge words in 2^-40 units
     float* tile;
     int tile_stride;
 };
@@ -127,13 +117,10 @@ __device__ __forceinline__ TileSm carve_tile(unsigned char* smem, int N, int cpl
     s.cams = reinterpret_cast<float*>(smem + l.cams);
     s.ctl = reinterpret_cast<int*>(smem + l.ctl);
     s.rc = reinterpret_cast<float*>(smem + l.rc);
-    s.vmask = reinterpret_cast<unsigned*>(smem + l.vmask);
-    s.uv = reinterpret_cast<float2*>(smem + l.uv);
-    s.box = reinterpret_cast<unsigned*>(smem + l.box);
-    s.cellg = reinterpret_cast<int*>(smem + l.cellg);
+    s.xlo = reinterpret_cast<unsigned short*>(smem + l.xlo);
     s.grp = reinterpret_cast<Group*>(smem + l.grp);
-    s.wq = reinterpret_cast<unsigned long long*>(smem + l.wq);
-    s.wf = reinterpret_cast<float*>(smem + l.wf);
+    s.wqh = reinterpret_cast<unsigned*>(smem + l.wqh);
+    s.wql = reinterpret_cast<unsigned*>(smem + l.wql);
     s.tile = reinterpret_cast<float*>(smem + l.tile);
     s.tile_stride = l.tile_stride;
     return s;
@@ -272,13 +259,28 @@ __device__ __forceinline__ ItemMap item_map(int zc) {
     return m;
 }
 
+// One camera's constants (E rows 0..2, K rows 0..1) held in registers.
+struct CamRegs {
+    float c[kCamFloats];
+};
+
+__device__ __forceinline__ CamRegs load_cam(const float* cam) {
+    CamRegs r;
+#pragma unroll
+    for (int k = 0; k < kCamFloats; ++k) r.c[k] = cam[k];
+    return r;
+}
+
 // Validity of one voxel in one camera, decided exactly as the fixed fp32
 // order of project_point decides it.  Depth and the homogeneous image
 // coordinates are computed in that order; the divides are taken with an
 // approximate quotient first and settled by the IEEE divide only when the
 // approximate position lies within 1e-5 (relative, at least 1e-5 px) of an
-// image edge, far outside the error of the approximation.
-__device__ __forceinline__ bool voxel_visible(const float* cam, float x, float y, float z, const GeoParams& g) {
+// image edge, far outside the error of the approximation.  `uv` receives the
+// position the decision used (approximate or exact).
+__device__ __forceinline__ bool voxel_visible(const CamRegs& cr, float x, float y, float z, const GeoParams& g,
+                                              float2& uv) {
+    const float* cam = cr.c;
     const float pcx = cam_row(cam + 0, x, y, z);
     const float pcy = cam_row(cam + 4, x, y, z);
     const float depth = cam_row(cam + 8, x, y, z);
@@ -291,67 +293,24 @@ __device__ __forceinline__ bool voxel_visible(const float* cam, float x, float y
     if (depth < 1e30f) {
         const float ua = __fdividef(uh, depth), va = __fdividef(vh, depth);
         const float mu = 1e-5f * fmaxf(fabsf(ua), 1.0f), mv = 1e-5f * fmaxf(fabsf(va), 1.0f);
-        const bool out_u = ua < -mu || ua > g.img_w + mu, out_v = va < -mv || va > g.img_h + mv;
-        if (out_u || out_v) return false;
+        uv = make_float2(ua, va);
+        if (ua < -mu || ua > g.img_w + mu || va < -mv || va > g.img_h + mv) return false;
         if (ua > mu && ua < g.img_w - mu && va > mv && va < g.img_h - mv) return true;
     }
     const float u = __fdiv_rn(uh, depth), v = __fdiv_rn(vh, depth);
+    uv = make_float2(u, v);
     return u >= 0.0f && u <= g.img_w && v >= 0.0f && v <= g.img_h;
 }
 
-// Count pass over the bins [z0, z0 + zc): 1 / cnt per item, a bit per
-// active camera that sees the item, and the optional uint8 count output.
-__device__ inline void count_pass(const SampleArgs& a, const TileSm& s, int b, int ti0, int tj0, int z0, int zc,
-                                  bool write_count) {
-    const GeoParams& g = a.g;
-    const ItemMap im = item_map(zc);
-    const int nA = s.ctl[kCtlNA];
-    const int zz = threadIdx.x % im.LZ;
-    for (int p = 0; p < im.passes; ++p) {
-        const int cell = p * im.cpp + (int)threadIdx.x / im.LZ;
-        if (cell >= kCells || zz >= zc) continue;
-        const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ, z = z0 + zz;
-        const bool in = i < g.X && j < g.Y;
-        unsigned m = 0;
-        int cnt = 0;
-        if (in) {
-            const float x = voxel_centre(g.xmin, i, g.dx), y = voxel_centre(g.ymin, j, g.dy);
-            const float zf = voxel_centre(g.zmin, z, g.dz);
-            for (int aa = 0; aa < nA; ++aa) {
-                if (voxel_visible(s.cams + s.ctl[kCtlActive + aa] * kCamFloats, x, y, zf, g)) {
-                    m |= 1u << aa;
-                    ++cnt;
-                }
-            }
-            if (write_count) a.count[(((size_t)b * g.X + i) * g.Y + j) * g.Z + z] = (uint8_t)cnt;
-        }
-        s.rc[cell * kZc + zz] = cnt > 0 ? __frcp_rn((float)cnt) : 0.0f;
-        s.vmask[cell * kZc + zz] = m;
-    }
-}
+__device__ __forceinline__ float2 no_uv() { return make_float2(__int_as_float(0x7fc00000), 0.0f); }
 
-// Image-plane positions of the voxels that active camera slot aa sees (x =
-// NaN elsewhere), in the fixed order of project_point.
-__device__ inline void project_pass(const SampleArgs& a, const TileSm& s, int ti0, int tj0, int z0, int zc, int aa) {
-    const GeoParams& g = a.g;
-    const ItemMap im = item_map(zc);
-    const float* cam = s.cams + s.ctl[kCtlActive + aa] * kCamFloats;
-    const int zz = threadIdx.x % im.LZ;
-    for (int p = 0; p < im.passes; ++p) {
-        const int cell = p * im.cpp + (int)threadIdx.x / im.LZ;
-        if (cell >= kCells || zz >= zc) continue;
-        const int item = cell * kZc + zz;
-        float2 uv = make_float2(__int_as_float(0x7fc00000), 0.0f);
-        if ((s.vmask[item] >> aa) & 1u) {
-            const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
-            float fx, fy;
-            ProjDetail det;
-            if (project_point(cam, voxel_centre(g.xmin, i, g.dx), voxel_centre(g.ymin, j, g.dy),
-                              voxel_centre(g.zmin, z0 + zz, g.dz), g, fx, fy, det))
-                uv = make_float2(det.u, det.v);
-        }
-        s.uv[item] = uv;
-    }
+// Exact image-plane position of a voxel when it is valid (as project_point
+// gives it), else x = NaN.
+__device__ __forceinline__ float2 voxel_exact(const CamRegs& cr, float x, float y, float z, const GeoParams& g) {
+    float fx, fy;
+    ProjDetail det;
+    if (project_point(cr.c, x, y, z, g, fx, fy, det)) return make_float2(det.u, det.v);
+    return no_uv();
 }
 
 // Sampling position of an image-plane position on a level of scale (sW, sH):
@@ -361,32 +320,62 @@ __device__ __forceinline__ void level_position(float2 uv, float sW, float sH, fl
     fy = __fadd_rn(__fmul_rn(uv.y, sH), -0.5f);
 }
 
-// Texel box of each cell on one level: (ylo, xlo) and (yhi, xhi) exclusive,
-// as 16-bit fields; an empty box is lo = 0xffffffff, hi = 0.
-__device__ inline void box_pass(const TileSm& s, int zc, int Hf, int Wf, float sW, float sH) {
+// Count pass over the bins [z0, z0 + zc): 1 / cnt per item, the optional
+// uint8 count output, and per (active camera, cell) the leftmost level-0
+// feature column the cell's valid voxels reach (from the position the
+// validity test used; it only steers the grouping).  Cameras are the outer
+// loop, so each camera's constants are read once per thread.
+constexpr int kMaxPasses = kCells * 16 / kThreads;  // item passes at 16 lanes per cell
+
+__device__ inline void count_pass(const SampleArgs& a, const TileSm& s, int b, int ti0, int tj0, int z0, int zc,
+                                  bool write_count) {
+    const GeoParams& g = a.g;
     const ItemMap im = item_map(zc);
+    const int nA = s.ctl[kCtlNA];
     const int zz = threadIdx.x % im.LZ;
-    for (int p = 0; p < im.passes; ++p) {
+    const float sW0 = a.lv.sW[0];
+    const int W0 = a.lv.Wf[0];
+    bool in[kMaxPasses];
+    float px[kMaxPasses], py[kMaxPasses], pz[kMaxPasses];
+    int cnt[kMaxPasses];
+#pragma unroll
+    for (int p = 0; p < kMaxPasses; ++p) {
         const int cell = p * im.cpp + (int)threadIdx.x / im.LZ;
-        unsigned lo = 0xffffffffu, hi = 0u;
-        if (cell < kCells && zz < zc) {
-            const float2 uv = s.uv[cell * kZc + zz];
-            if (!isnan(uv.x)) {
-                float fx, fy;
-                level_position(uv, sW, sH, fx, fy);
-                const int x0 = (int)floorf(fx), y0 = (int)floorf(fy);
-                lo = ((unsigned)max(y0, 0) << 16) | (unsigned)max(x0, 0);
-                hi = ((unsigned)min(y0 + 2, Hf) << 16) | (unsigned)min(x0 + 2, Wf);
+        const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
+        in[p] = p < im.passes && cell < kCells && zz < zc && i < g.X && j < g.Y;
+        px[p] = voxel_centre(g.xmin, i, g.dx);
+        py[p] = voxel_centre(g.ymin, j, g.dy);
+        pz[p] = voxel_centre(g.zmin, z0 + zz, g.dz);
+        cnt[p] = 0;
+    }
+    for (int aa = 0; aa < nA; ++aa) {
+        const CamRegs cr = load_cam(s.cams + s.ctl[kCtlActive + aa] * kCamFloats);
+#pragma unroll
+        for (int p = 0; p < kMaxPasses; ++p) {
+            if (p >= im.passes) break;
+            float2 uv;
+            unsigned x0 = 0xffffu;
+            if (in[p] && voxel_visible(cr, px[p], py[p], pz[p], g, uv)) {
+                ++cnt[p];
+                x0 = (unsigned)min(max((int)floorf(__fmaf_rn(uv.x, sW0, -0.5f)), 0), W0 - 1);
             }
+            // leftmost column over the cell's lanes (warps with none skip it)
+            if (__any_sync(0xffffffffu, x0 != 0xffffu)) {
+                for (int o = 1; o < im.LZ; o <<= 1) x0 = min(x0, __shfl_xor_sync(0xffffffffu, x0, o));
+            }
+            const int cell = p * im.cpp + (int)threadIdx.x / im.LZ;
+            if (zz == 0 && cell < kCells) s.xlo[aa * kCells + cell] = (unsigned short)x0;
         }
-        for (int o = 1; o < im.LZ; o <<= 1) {
-            lo = __vminu2(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-            hi = __vmaxu2(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+#pragma unroll
+    for (int p = 0; p < kMaxPasses; ++p) {
+        if (p >= im.passes) break;
+        const int cell = p * im.cpp + (int)threadIdx.x / im.LZ;
+        if (in[p] && write_count) {
+            const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
+            a.count[(((size_t)b * g.X + i) * g.Y + j) * g.Z + z0 + zz] = (uint8_t)cnt[p];
         }
-        if (zz == 0 && cell < kCells) {
-            s.box[2 * cell] = lo;
-            s.box[2 * cell + 1] = hi;
-        }
+        if (cell < kCells && zz < zc) s.rc[cell * kZc + zz] = cnt[p] > 0 ? __frcp_rn((float)cnt[p]) : 0.0f;
     }
 }
 
@@ -404,36 +393,30 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
     return v;
 }
 
-__device__ __forceinline__ int slots_for(int n) { return n == 1 ? 1 : n == 2 ? 2 : n <= 4 ? 4 : 8; }
 
 // Groups of the current view from the cells' boxes: cells whose boxes start
 // at the same feature column form buckets, split into groups of at most
 // kGmax cells; cells more than 63 columns right of the leftmost form groups
-// of their own.  Then the union boxes, the weight layout and the merge
-// rounds.  Warp 0 only.
-__device__ inline void form_groups(const TileSm& s) {
+// of their own.  The groups are listed largest first, so that the warps that
+// take them in turn finish close together.  Warp 0 only.
+__device__ inline void form_groups(const TileSm& s, const unsigned short* xl) {
     const int lane = threadIdx.x & 31;
     int* ctl = s.ctl;
     int* bcnt = ctl + kCtlBucket;
     int* gbase = ctl + kCtlGbase;
-    int* gy0 = ctl + kCtlBounds;
-    int* gx0 = gy0 + kCells;
-    int* gy1 = gx0 + kCells;
-    int* gx1 = gy1 + kCells;
-    unsigned lo[2], hi[2];
+    int* hist = ctl + kCtlSizeHist;  // [0, kGmax]: count per size, reused as cursors
     bool val[2];
     int xlo[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         const int c = lane + 32 * k;
-        lo[k] = s.box[2 * c];
-        hi[k] = s.box[2 * c + 1];
-        val[k] = hi[k] != 0u;
-        xlo[k] = (int)(lo[k] & 0xffffu);
+        xlo[k] = (int)xl[c];
+        val[k] = xlo[k] != 0xffff;
     }
     const int xm = __reduce_min_sync(0xffffffffu, (unsigned)min(val[0] ? xlo[0] : 0xffff, val[1] ? xlo[1] : 0xffff));
     bcnt[lane] = 0;
     bcnt[lane + 32] = 0;
+    if (lane <= kGmax) hist[lane] = 0;
     __syncwarp();
     int key[2], rank[2] = {0, 0};
 #pragma unroll
@@ -454,158 +437,215 @@ __device__ inline void form_groups(const TileSm& s) {
     const int ng = nbg + __popc(far0) + __popc(far1);
     __syncwarp();
     const unsigned lt = (1u << lane) - 1u;
-    int grp[2] = {-1, -1}, slot[2] = {0, 0};
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         const int c = lane + 32 * k;
-        int cg = -1;
         if (val[k]) {
-            int gi, n;
+            int gi, slot, n;
             if (key[k] < 64) {
                 gi = gbase[key[k]] + rank[k] / kGmax;
-                slot[k] = rank[k] % kGmax;
+                slot = rank[k] % kGmax;
                 n = min(kGmax, bcnt[key[k]] - (rank[k] / kGmax) * kGmax);
             } else {
                 gi = nbg + (k == 0 ? __popc(far0 & lt) : __popc(far0) + __popc(far1 & lt));
-                slot[k] = 0;
+                slot = 0;
                 n = 1;
             }
-            grp[k] = gi;
-            cg = (gi << 8) | slot[k];
-            s.grp[gi].cell[slot[k]] = (unsigned char)c;
-            if (slot[k] == 0) {
+            s.grp[gi].cell[slot] = (unsigned char)c;
+            if (slot == 0) {
                 s.grp[gi].n = n;
-                gy0[gi] = (int)(lo[k] >> 16);
-                gx0[gi] = (int)(lo[k] & 0xffffu);
-                gy1[gi] = (int)(hi[k] >> 16);
-                gx1[gi] = (int)(hi[k] & 0xffffu);
-            }
-        }
-        s.cellg[c] = cg;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        if (grp[k] >= 0 && slot[k] != 0) {
-            atomicMin(&gy0[grp[k]], (int)(lo[k] >> 16));
-            atomicMin(&gx0[grp[k]], (int)(lo[k] & 0xffffu));
-            atomicMax(&gy1[grp[k]], (int)(hi[k] >> 16));
-            atomicMax(&gx1[grp[k]], (int)(hi[k] & 0xffffu));
-        }
-    }
-    __syncwarp();
-    // weight entries per group; boxes too large for half a round go direct
-    int e[2], sl[2], h[2], w[2], dir[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int gi = lane + 32 * k;
-        e[k] = 0;
-        sl[k] = 1;
-        h[k] = w[k] = 0;
-        dir[k] = 0;
-        if (gi < ng) {
-            h[k] = gy1[gi] - gy0[gi];
-            w[k] = gx1[gi] - gx0[gi];
-            sl[k] = slots_for(s.grp[gi].n);
-            // padded to 4 entries so that every group's weights start 16-byte aligned
-            const long long ent = ((long long)h[k] * w[k] * sl[k] + 3) & ~3ll;
-            if (ent > kEntries / 2) {
-                dir[k] = 1;
-            } else {
-                e[k] = (int)ent;
+                atomicAdd(&hist[n], 1);
             }
         }
     }
-    const int emax = __reduce_max_sync(0xffffffffu, (unsigned)max(e[0], e[1]));
-    const int step = kEntries - emax;  // >= kEntries / 2
-    const int s0 = warp_inclusive_scan(e[0]), s1 = warp_inclusive_scan(e[1]);
-    const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
-    const int off[2] = {s0 - e[0], tot0 + s1 - e[1]};
-    int* rstart = ctl + kCtlRstart;
-    int* nent = ctl + kCtlNent;
-    nent[lane] = 0;
-    nent[lane + 32] = 0;
     __syncwarp();
-    int rnd[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int gi = lane + 32 * k;
-        rnd[k] = off[k] / step;
-        if (gi < ng) {
-            Group& gp = s.grp[gi];
-            gp.y0 = gy0[gi];
-            gp.x0 = gx0[gi];
-            gp.h = h[k];
-            gp.w = w[k];
-            gp.slots = sl[k];
-            gp.round = rnd[k];
-            gp.off = off[k] - rnd[k] * step;
-            gp.direct = dir[k];
-            atomicMax(&nent[rnd[k]], gp.off + e[k]);
-        }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int gi = lane + 32 * k;
-        if (gi < ng && (gi == 0 || s.grp[gi - 1].round != rnd[k])) rstart[rnd[k]] = gi;
-    }
+    // largest first: groups of size n start after all larger ones
     if (lane == 0) {
-        const int nr = ng > 0 ? s.grp[ng - 1].round + 1 : 0;
-        rstart[nr] = ng;
+        int at = 0;
+        for (int n = kGmax; n >= 1; --n) {
+            const int c = hist[n];
+            hist[n] = at;
+            at += c;
+        }
         ctl[kCtlGroups] = ng;
-        ctl[kCtlRounds] = nr;
+        ctl[kCtlNext] = 0;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int gi = lane + 32 * k;
+        if (gi < ng) ctl[kCtlOrder + atomicAdd(&hist[s.grp[gi].n], 1)] = gi;
     }
 }
 
 // ---------------------------------------------------------------------------
-// Merge of one round's weights
+// Per-warp merge of one group's weights
 // ---------------------------------------------------------------------------
 
-constexpr float kFix = 1099511627776.0f;  // 2^40: fixed point of the merged weights
-constexpr double kFixInv = 9.094947017729282379150390625e-13;  // 2^-40
+// Exact fixed point of the merged weights.  A contribution v = w / cnt (in
+// [0, 1], fp32) is split into hi = RN(v 2^20) and lo = RN((v - hi 2^-20)
+// 2^40), |lo| <= 2^19; both splits are exact integer roundings done by adding
+// 1.5 * 2^23 in fp32 (the sum lies in [2^23, 2^24), where the spacing of fp32
+// is 1, so the addition rounds to an integer) and the residual is exact.  At
+// most kZc contributions reach one entry, so the word sums stay within 2^24 in
+// magnitude and convert to fp32 exactly: the merged weight
+// hi 2^-20 + lo 2^-40 does not depend on the order of the additions and is
+// rounded once.
+constexpr float kTwo20 = 1048576.0f;
+constexpr float kTwoM20 = 9.5367431640625e-07f;
+constexpr float kTwoM40 = 9.094947017729282379150390625e-13f;
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+static_assert(kZc * (1 << 20) <= (1 << 24), "merge words must stay exact in fp32");
 
-// Sum w / cnt of every valid bin into its cell's slot of its group's
-// [texel][slot] array (groups of round r that are not direct).
-__device__ inline void merge_pass(const TileSm& s, int zc, int Hf, int Wf, float sW, float sH, int r) {
+__device__ __forceinline__ void split_weight(float v, int& hi, int& lo) {
+    const float t = __fmaf_rn(v, kTwo20, kRound);
+    hi = __float_as_int(t) - __float_as_int(kRound);
+    const float r = __fmaf_rn(v, kTwo20, -__fsub_rn(t, kRound));  // exact residual, |r| <= 0.5
+    lo = __float_as_int(__fmaf_rn(r, kTwo20, kRound)) - __float_as_int(kRound);
+}
+
+// A group's voxels, as the warp that sweeps the group holds them: lane l
+// takes bin l % LZ of member cell t * (32 / LZ) + l / LZ at step t.
+constexpr int kItemSteps = kGmax * kZc / 32;
+
+struct GroupItems {
+    float2 uv[kItemSteps];  // exact image-plane position; x = NaN when the camera does not see the voxel
+};
+
+// Exact projections of the members' voxels through one camera.
+__device__ inline GroupItems project_members(const SampleArgs& a, const TileSm& s, const unsigned char* cells, int n,
+                                             int cam, int ti0, int tj0, int z0, int zc) {
+    const GeoParams& g = a.g;
+    const int lane = threadIdx.x & 31;
     const ItemMap im = item_map(zc);
-    const int zz = threadIdx.x % im.LZ;
-    for (int p = 0; p < im.passes; ++p) {
-        const int cell = p * im.cpp + (int)threadIdx.x / im.LZ;
-        if (cell >= kCells || zz >= zc) continue;
-        const int item = cell * kZc + zz;
-        const float2 uv = s.uv[item];
-        const int cg = s.cellg[cell];
-        if (isnan(uv.x) || cg < 0) continue;
-        const Group& gp = s.grp[cg >> 8];
-        if (gp.round != r || gp.direct) continue;
-        float fx, fy;
-        level_position(uv, sW, sH, fx, fy);
-        const Corners c = bilinear_corners(fx, fy);
-        const float rc = s.rc[item];
-        const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
-        const int slot = cg & 255;
+    const int zz = lane % im.LZ, per = 32 / im.LZ;
+    const CamRegs cr = load_cam(s.cams + cam * kCamFloats);
+    GroupItems it;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
-            if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
-            const unsigned long long q = __float2ull_rn(__fmul_rn(ws[k], rc) * kFix);
-            if (q == 0ull) continue;
-            const int e = gp.off + ((yy - gp.y0) * gp.w + (xx - gp.x0)) * gp.slots + slot;
-            atomicAdd(&s.wq[e], q);
+    for (int t = 0; t < kItemSteps; ++t) {
+        it.uv[t] = no_uv();
+        const int k = t * per + lane / im.LZ;
+        if (t * per < n && k < n && zz < zc) {
+            const int cell = cells[k];
+            const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
+            it.uv[t] = voxel_exact(cr, voxel_centre(g.xmin, i, g.dx), voxel_centre(g.ymin, j, g.dy),
+                                   voxel_centre(g.zmin, z0 + zz, g.dz), g);
         }
     }
+    return it;
 }
 
-// Round r's fixed-point sums to fp32 (one rounding each); the fixed-point
-// words are cleared for the next round.
-__device__ __forceinline__ void convert_pass(const TileSm& s, int r) {
-    const int n = s.ctl[kCtlNent + r];
-    for (int e = threadIdx.x; e < n; e += kThreads) {
-        const unsigned long long q = s.wq[e];
-        s.wq[e] = 0ull;
-        s.wf[e] = __double2float_rn(__ull2double_rn(q) * kFixInv);
+// A set of member cells and the union of their texel boxes on the current
+// level, as one warp processes it.  When the map allows, the box is widened
+// to even height and width inside the map (extra rows and columns carry zero
+// weight), so that the sweep's two-by-two steps need no edge predicates.
+struct Members {
+    int n;                      // cells (1 .. kGmax)
+    int slots;                  // weights per texel (1, 2, 4 or 8)
+    int y0, x0, h, w;           // union box
+    bool even;                  // h and w are even
+    const unsigned char* cell;  // member cell indices (shared memory)
+    int entries;                // h * w * slots rounded up to 4
+};
+
+__device__ __forceinline__ int slots_for(int n) { return n == 1 ? 1 : n == 2 ? 2 : n <= 4 ? 4 : 8; }
+
+// Union of the bilinear corners (inside the map) of the group's valid voxels
+// on one level; warp-uniform.  Every member has a valid voxel, so the box is
+// not empty.
+__device__ __forceinline__ Members members_box(const GroupItems& it, const unsigned char* cells, int n, int Hf, int Wf,
+                                               float sW, float sH) {
+    unsigned lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+    for (int t = 0; t < kItemSteps; ++t) {
+        if (!isnan(it.uv[t].x)) {
+            float fx, fy;
+            level_position(it.uv[t], sW, sH, fx, fy);
+            const int x0 = (int)floorf(fx), y0 = (int)floorf(fy);
+            lo = __vminu2(lo, ((unsigned)max(y0, 0) << 16) | (unsigned)max(x0, 0));
+            hi = __vmaxu2(hi, ((unsigned)min(y0 + 2, Hf) << 16) | (unsigned)min(x0 + 2, Wf));
+        }
     }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        lo = __vminu2(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = __vmaxu2(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    Members m;
+    m.n = n;
+    m.slots = slots_for(n);
+    m.y0 = (int)(lo >> 16);
+    m.x0 = (int)(lo & 0xffffu);
+    m.h = (int)(hi >> 16) - m.y0;
+    m.w = (int)(hi & 0xffffu) - m.x0;
+    const int h2 = (m.h + 1) & ~1, w2 = (m.w + 1) & ~1;
+    m.even = h2 <= Hf && w2 <= Wf;
+    if (m.even) {  // the widened box still covers the union and stays inside the map
+        m.y0 = min(m.y0, Hf - h2);
+        m.x0 = min(m.x0, Wf - w2);
+        m.h = h2;
+        m.w = w2;
+    }
+    m.cell = cells;
+    m.entries = (m.h * m.w * m.slots + 3) & ~3;
+    return m;
+}
+
+// Sum w / cnt of every valid voxel of the members into the warp's region
+// ([texel of the union box][member] words), then round each entry to fp32
+// in place (the weights replace the 2^-20 words; the 2^-40 words are
+// cleared).  Ends with the weights readable by the whole warp.
+__device__ inline void merge_members(const TileSm& s, const Members& m, const GroupItems& it, int zc, int Hf, int Wf,
+                                     float sW, float sH, unsigned* wh, unsigned* wl) {
+    const int lane = threadIdx.x & 31;
+    const ItemMap im = item_map(zc);
+    const int zz = lane % im.LZ, per = 32 / im.LZ;
+    const int rowe = m.w * m.slots;
+#pragma unroll
+    for (int t = 0; t < kItemSteps; ++t) {
+        const int k = t * per + lane / im.LZ;
+        if (isnan(it.uv[t].x) || k >= m.n) continue;
+        float fx, fy;
+        level_position(it.uv[t], sW, sH, fx, fy);
+        const Corners c = bilinear_corners(fx, fy);
+        const float rc = s.rc[m.cell[k] * kZc + zz];
+        const bool cx0 = (unsigned)c.x0 < (unsigned)Wf, cx1 = (unsigned)(c.x0 + 1) < (unsigned)Wf;
+        const bool cy0 = (unsigned)c.y0 < (unsigned)Hf, cy1 = (unsigned)(c.y0 + 1) < (unsigned)Hf;
+        const int e = ((c.y0 - m.y0) * m.w + (c.x0 - m.x0)) * m.slots + k;
+        const float ws[4] = {c.w00, c.w01, c.w10, c.w11};
+        const bool ok[4] = {cy0 && cx0, cy0 && cx1, cy1 && cx0, cy1 && cx1};
+        const int off[4] = {0, m.slots, rowe, rowe + m.slots};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float v = __fmul_rn(ws[q], rc);
+            if (!ok[q] || v == 0.0f) continue;
+            int hi, lo;
+            split_weight(v, hi, lo);
+            if (hi != 0) atomicAdd(&wh[e + off[q]], (unsigned)hi);
+            if (lo != 0) atomicAdd(reinterpret_cast<int*>(wl) + e + off[q], lo);
+        }
+    }
+    __syncwarp();
+    for (int e = 4 * lane; e < m.entries; e += 128) {
+        const uint4 qh = *reinterpret_cast<const uint4*>(wh + e);
+        const int4 ql = *reinterpret_cast<const int4*>(wl + e);
+        *reinterpret_cast<uint4*>(wl + e) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<float4*>(wh + e) =
+            make_float4(__fadd_rn((float)qh.x * kTwoM20, (float)ql.x * kTwoM40),
+                        __fadd_rn((float)qh.y * kTwoM20, (float)ql.y * kTwoM40),
+                        __fadd_rn((float)qh.z * kTwoM20, (float)ql.z * kTwoM40),
+                        __fadd_rn((float)qh.w * kTwoM20, (float)ql.w * kTwoM40));
+    }
+    __syncwarp();
+}
+
+// Clear the weights of the warp's region after its sweep (the region must be
+// zero before the next merge).
+__device__ __forceinline__ void clear_members(const Members& m, unsigned* wh) {
+    __syncwarp();
+    const int lane = threadIdx.x & 31;
+    for (int e = 4 * lane; e < m.entries; e += 128) *reinterpret_cast<uint4*>(wh + e) = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
