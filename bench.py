@@ -3,8 +3,13 @@
 
 One step = the whole hot path over one batch: channels-last copy of the
 features, fused forward gather-reduction, and the feature gradient (zero-init,
-scatter, layout back), on the nuScenes-like workload (B1, 6 cameras, C64,
-16x44 features from 256x704 images, BEV 200x200x8 over +-50 m, fp32).
+scatter, layout back).  The default workload is the largest single-GPU one,
+``batched_bf16`` (B4, 6 cameras, C128 bf16 features of 32x88 from 512x1408
+images, BEV 200x200x16 over +-50 m, fp32 accumulation and output);
+--workload picks another (tiny, nuscenes, large, backward).  The line's
+``by_workload`` block adds the forward and backward of ``large`` (B1 C80
+fp32, 400x400x16) and ``nuscenes`` (B1 C64 fp32, 200x200x8), timed outside
+the main timed region.
 
 Timing: inputs resident in HBM; L2 flushed (256 MiB write) before every timed
 step; the step (repack, forward, backward) captured once as a CUDA graph and
@@ -65,19 +70,16 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="nuscenes")
+    ap.add_argument("--workload", default=None,
+                    help="default: batched_bf16 (vt), deform, lss or ms (the other operators)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--op", choices=["vt", "deform", "lss", "ms"], default="vt")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the hot-L2 and back-to-back forward timings (for launch-list profiling)")
     args = ap.parse_args()
-    if args.op == "deform" and args.workload == "nuscenes":
-        args.workload = "deform"
-    if args.op == "lss" and args.workload == "nuscenes":
-        args.workload = "lss"
-    if args.op == "ms" and args.workload == "nuscenes":
-        args.workload = "ms"
+    if args.workload is None:
+        args.workload = {"vt": "batched_bf16", "deform": "deform", "lss": "lss", "ms": "ms"}[args.op]
     return args
 
 
@@ -233,18 +235,20 @@ def oracle_step_sample(w, rows, threads):
 
 
 def cpu_baseline(w, seconds):
-    """The oracle as it stands, on the host cores, whole workload steps until
-    `seconds` of CPU work (at least one step)."""
+    """The oracle as it stands, on the host cores, on slices of BEV rows at
+    the grid centre (forward + backward over all batch items, cameras and
+    channels of those rows) until `seconds` of CPU work (at least one)."""
     threads = cpu_cores()
+    rows = max(8, w.X // 25)
     spent, elems, steps = 0.0, 0, 0
     while steps == 0 or spent < seconds:
-        t, e = oracle_step_sample(w, w.X, threads)
+        t, e = oracle_step_sample(w, rows, threads)
         spent += t
         elems += e
         steps += 1
     return {"value": elems / spent, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{steps} whole forward+backward step(s) of the {w.name} workload "
-                      f"({spent:.1f} s, OpenMP over BEV rows / (batch, camera))"}
+            "sample": f"{steps} slice(s) of {rows} of the {w.X} BEV rows of the {w.name} workload, forward + "
+                      f"backward ({spent:.1f} s, OpenMP over BEV rows / (batch, camera))"}
 
 
 def run_reference(args):
@@ -518,6 +522,9 @@ def run_ours(args):
     }
     for g in list(graphs.values()) + [step_graph]:
         g.reset()
+    if not args.no_extras:
+        line["by_workload"] = {name: other_workload(I, ops, I.WORKLOADS[name], dev, stream, flush, peak)
+                               for name in ("large", "nuscenes") if name != w.name}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -525,6 +532,53 @@ def run_ours(args):
         if world == 1:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)
+
+
+def other_workload(I, ops, w, dev, stream, flush, peak, reps=100):
+    """Forward (channels-last features) and backward call of another dense
+    workload, each captured as a CUDA graph and replayed between CUDA events
+    on the launching stream with the L2 flushed before every replay; outside
+    the timed region of the main workload."""
+    import torch
+    F = I.make_features(w, layout="nhwc").to(dev)
+    K, E = (t.to(dev) for t in I.make_rigs(w))
+    dout = I.make_dout(w).to(dev)
+    grid = ops.bev_grid_spec(w.ranges, w.res)
+    out = torch.empty((w.B, w.C, w.X, w.Y), dtype=torch.float32, device=dev)
+    dF = torch.empty((w.B, w.N, w.C, w.Hf, w.Wf), dtype=torch.float32, device=dev)
+    ws_b = torch.empty(ops.bev_workspace_size(ops.F32, ops.NCHW, w.B, w.N, w.C, w.Hf, w.Wf, 1), dtype=torch.uint8,
+                       device=dev)
+    calls = {"forward": lambda: ops.bev_sample_forward(F, K, E, w.img_h, w.img_w, grid, layout=ops.NHWC, out=out),
+             "backward": lambda: ops.bev_sample_backward(dout, K, E, w.img_h, w.img_w, grid, w.N, w.Hf, w.Wf,
+                                                         out=dF, workspace=ws_b)}
+    res = {"workload": workload_desc(w)}
+    with torch.cuda.stream(stream):
+        for name, f in calls.items():
+            f()
+            stream.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                f()
+            times = []
+            for k in range(reps + 5):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                gr.replay()
+                e1.record(stream)
+                e1.synchronize()
+                if k >= 5:
+                    times.append(e0.elapsed_time(e1))
+            gr.reset()
+            ms = statistics.median(times)
+            nbytes = (w.B * w.N * w.Hf * w.Wf * w.C * F.element_size() + w.out_elems * 4 if name == "forward"
+                      else w.out_elems * 4 + w.B * w.N * w.C * w.Hf * w.Wf * 4)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            res[name] = {"us": 1e3 * ms, "algorithmic_bytes": nbytes, "GB_per_s": gbs, "frac_of_hbm_peak": gbs / peak,
+                         "elements_per_s": w.out_elems / (ms * 1e-3)}
+    res["note"] = ("median of 100 graph replays, L2 flushed before each; forward on channels-last features "
+                   "(the repack is a separate call), backward = the whole call (zero-init, scatter, layout)")
+    return res
 
 
 DEFORM_METRIC = "deformable aggregation output elements/s (B·Q·C) and achieved HBM GB/s vs roofline, 1×B200"

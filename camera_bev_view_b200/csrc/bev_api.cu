@@ -104,6 +104,22 @@ int cuda_status(cudaError_t e) {
     return BEV_ERR_CUDA;
 }
 
+// Status of a dense launch.  In the bounds-checked build the stream is
+// drained and the kernels' device error word read back: a check that failed
+// on the device gives BEV_ERR_INTERNAL.
+int dense_status(cudaError_t launch, cudaStream_t s, bool backward) {
+    const int st = cuda_status(launch);
+#ifdef BEV_BOUNDS_CHECK
+    if (st != BEV_OK) return st;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_status(cudaErrorUnknown);
+    return (backward ? bev_backward_check_take() : bev_forward_check_take()) ? BEV_ERR_INTERNAL : BEV_OK;
+#else
+    (void)s;
+    (void)backward;
+    return st;
+#endif
+}
+
 // Channel slices of the dense kernels: each lane of a warp owns cpl
 // consecutive channels, so a CTA covers 32 * cpl channels of the Cp padded
 // channels per texel (4-, 8- or 16-byte loads per lane).  Fills a.cpl and
@@ -130,6 +146,14 @@ void single_level(bev::SampleArgs& a, int Hf, int Wf, int img_h, int img_w) {
 }
 
 }  // namespace
+
+BEV_API int bev_bounds_checked(void) {
+#ifdef BEV_BOUNDS_CHECK
+    return 1;
+#else
+    return 0;
+#endif
+}
 
 BEV_API const char* bev_status_string(int status) {
     switch (status) {
@@ -235,7 +259,7 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
     a.out_vec = ((uintptr_t)out % 16) == 0 && (grid->Y % 4) == 0;
     const int slices = channel_slices(a, dtype == BEV_BF16, Cp);
     tile_grid(a, grid);
-    return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, slices, s));
+    return dense_status(bev_launch_forward(a, dtype == BEV_BF16, slices, s), s, false);
 }
 
 BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, int Wf,
@@ -274,7 +298,7 @@ BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, 
     a.out_vec = ((uintptr_t)dout % 16) == 0 && (grid->Y % 4) == 0;
     const int slices = channel_slices(a, false, Cp);
     tile_grid(a, grid);
-    if ((st = cuda_status(bev_launch_backward(a, slices, s))) != BEV_OK) return st;
+    if ((st = dense_status(bev_launch_backward(a, slices, s), s, true)) != BEV_OK) return st;
     return cuda_status(bev_launch_to_nchw(static_cast<const float*>(workspace), B * N, C, Hf * Wf, Cp,
                                           dfeatures, s));
 }
@@ -407,7 +431,7 @@ BEV_API int bev_sample_forward_multiscale(const void* const* features, int nleve
     a.out_vec = ((uintptr_t)out % 16) == 0 && (grid->Y % 4) == 0;
     const int slices = channel_slices(a, dtype == BEV_BF16, Cp);
     tile_grid(a, grid);
-    return cuda_status(bev_launch_forward(a, dtype == BEV_BF16, slices, s));
+    return dense_status(bev_launch_forward(a, dtype == BEV_BF16, slices, s), s, false);
 }
 
 BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const int* Hf, const int* Wf, int B,
@@ -453,7 +477,7 @@ BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const
     a.C = C;
     const int slices = channel_slices(a, false, Cp);
     tile_grid(a, grid);
-    if ((st = cuda_status(bev_launch_backward(a, slices, s))) != BEV_OK) return st;
+    if ((st = dense_status(bev_launch_backward(a, slices, s), s, true)) != BEV_OK) return st;
     for (int l = 0; l < nlevels; ++l) {
         st = cuda_status(bev_launch_to_nchw(base[l], B * N, C, Hf[l] * Wf[l], Cp,
                                             dfeatures[l], s));

@@ -154,6 +154,7 @@ __device__ __forceinline__ void sweep_backward(const SampleArgs& a, const TileSm
         k = __shfl_sync(0xffffffffu, k, 0);
         if (k >= ng) break;
         const Group& gp = s.grp[s.ctl[kCtlOrder + k]];
+        if (!checked(gp.n >= 1 && gp.n <= kGmax, kCheckGroups)) continue;
         const GroupItems it = project_members(a, s, gp.cell, gp.n, cam, ti0, tj0, z0, zc);
         for (int l = 0; l < a.lv.n; ++l) {
             const int Hl = a.lv.Hf[l], Wl = a.lv.Wf[l];
@@ -161,6 +162,7 @@ __device__ __forceinline__ void sweep_backward(const SampleArgs& a, const TileSm
             const size_t rowf = (size_t)Wl * tf;
             float* gl = a.lv.grad[l] + ((size_t)b * a.N + cam) * Hl * rowf + c_base + lane * CPL;
             const Members m = members_box(it, gp.cell, gp.n, Hl, Wl, sW, sH);
+            if (!box_inside(m, Hl, Wl)) continue;
             if (m.entries <= kWarpEntries) {
                 backward_members<CPL>(s, m, it, zc, Hl, Wl, sW, sH, gl, rowf, tf, on, lane, wh, wl);
                 continue;
@@ -168,6 +170,7 @@ __device__ __forceinline__ void sweep_backward(const SampleArgs& a, const TileSm
             for (int q = 0; q < gp.n; ++q) {  // too large together: cell by cell
                 const GroupItems one = project_members(a, s, gp.cell + q, 1, cam, ti0, tj0, z0, zc);
                 const Members m1 = members_box(one, gp.cell + q, 1, Hl, Wl, sW, sH);
+                if (!box_inside(m1, Hl, Wl)) continue;
                 if (m1.entries <= kWarpEntries)
                     backward_members<CPL>(s, m1, one, zc, Hl, Wl, sW, sH, gl, rowf, tf, on, lane, wh, wl);
                 else
@@ -210,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, kTileCtas) sample_backward_kernel(co
         const int c = idx & (SL - 1), i = ti0 + idx / SL;
 #pragma unroll
         for (int cj = 0; cj < kTileJ; ++cj) dv[it][cj] = 0.0f;
-        if (idx < SL * kTileI && c < nch && i < g.X) {
+        if (idx < SL * kTileI && c < nch && i < g.X && checked(b < a.B && c_base + c < a.C, kCheckStore)) {
             const float* dp = a.dout + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0;
             if (a.out_vec && tj0 + kTileJ <= g.Y) {
 #pragma unroll
@@ -262,6 +265,10 @@ static cudaError_t launch(const SampleArgs& a, dim3 grid, cudaStream_t st) {
 }
 
 }  // namespace bev
+
+#ifdef BEV_BOUNDS_CHECK
+unsigned bev_backward_check_take() { return bev::check_take(); }
+#endif
 
 cudaError_t bev_launch_backward(const bev::SampleArgs& a, int slices, cudaStream_t stream) {
     const dim3 grid(a.tiles_i * a.tiles_j, a.B, slices);

@@ -198,6 +198,7 @@ __device__ __forceinline__ void sweep_forward(const SampleArgs& a, const TileSm&
         k = __shfl_sync(0xffffffffu, k, 0);
         if (k >= ng) break;
         const Group& gp = s.grp[s.ctl[kCtlOrder + k]];
+        if (!checked(gp.n >= 1 && gp.n <= kGmax, kCheckGroups)) continue;
         const GroupItems it = project_members(a, s, gp.cell, gp.n, cam, ti0, tj0, z0, zc);
         for (int l = 0; l < a.lv.n; ++l) {
             const int Hl = a.lv.Hf[l], Wl = a.lv.Wf[l];
@@ -206,6 +207,7 @@ __device__ __forceinline__ void sweep_forward(const SampleArgs& a, const TileSm&
             const unsigned char* fl = static_cast<const unsigned char*>(a.lv.feat[l]) +
                                       ((size_t)b * a.N + cam) * Hl * rowb + (size_t)lane_c * esize;
             const Members m = members_box(it, gp.cell, gp.n, Hl, Wl, sW, sH);
+            if (!box_inside(m, Hl, Wl)) continue;
             if (m.entries <= kWarpEntries) {
                 forward_members<BF16, CPL>(s, m, it, zc, Hl, Wl, sW, sH, fl, rowb, tb, on, lane, wh, wl);
                 continue;
@@ -213,6 +215,7 @@ __device__ __forceinline__ void sweep_forward(const SampleArgs& a, const TileSm&
             for (int q = 0; q < gp.n; ++q) {  // too large together: cell by cell
                 const GroupItems one = project_members(a, s, gp.cell + q, 1, cam, ti0, tj0, z0, zc);
                 const Members m1 = members_box(one, gp.cell + q, 1, Hl, Wl, sW, sH);
+                if (!box_inside(m1, Hl, Wl)) continue;
                 if (m1.entries <= kWarpEntries)
                     forward_members<BF16, CPL>(s, m1, one, zc, Hl, Wl, sW, sH, fl, rowb, tb, on, lane, wh, wl);
                 else
@@ -273,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, kTileCtas) sample_forward_kernel(con
 #pragma unroll
         for (int cj = 0; cj < kTileJ; ++cj) v[cj] = tp[cj * s.tile_stride];
         float* op = a.out + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0;
+        if (!checked(b < a.B && c_base + c < a.C, kCheckStore)) continue;
         if (a.out_vec && tj0 + kTileJ <= g.Y) {
 #pragma unroll
             for (int q = 0; q < kTileJ / 4; ++q)
@@ -297,6 +301,10 @@ static cudaError_t launch(const SampleArgs& a, dim3 grid, cudaStream_t st) {
 }
 
 }  // namespace bev
+
+#ifdef BEV_BOUNDS_CHECK
+unsigned bev_forward_check_take() { return bev::check_take(); }
+#endif
 
 cudaError_t bev_launch_forward(const bev::SampleArgs& a, bool bf16, int slices, cudaStream_t stream) {
     const dim3 grid(a.tiles_i * a.tiles_j, a.B, slices);

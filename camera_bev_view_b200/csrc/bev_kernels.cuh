@@ -86,6 +86,12 @@ inline cudaError_t set_smem_attributes(Kernel* k, size_t smem, int carveout,
 // 32 * a.cpl channels each.
 cudaError_t bev_launch_forward(const bev::SampleArgs& a, bool bf16, int slices, cudaStream_t stream);
 cudaError_t bev_launch_backward(const bev::SampleArgs& a, int slices, cudaStream_t stream);
+#ifdef BEV_BOUNDS_CHECK
+// Checked build: read and clear the device error word of the dense forward /
+// backward kernels (call after the launch's stream has drained).
+unsigned bev_forward_check_take();
+unsigned bev_backward_check_take();
+#endif
 cudaError_t bev_launch_to_channels_last(const void* src, int layout, int esize, int BN, int C,
                                         int HW, int Cp, void* dst, cudaStream_t stream);
 cudaError_t bev_launch_to_nchw(const float* src, int BN, int C, int HW, int Cp, float* dst,

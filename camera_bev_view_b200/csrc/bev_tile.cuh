@@ -42,6 +42,39 @@
 
 namespace bev {
 
+// Bounds-checked build (-DBEV_BOUNDS_CHECK).  Before each access whose
+// address comes from geometry -- a group's texel box (every gather load and
+// every gradient reduction lies inside it), a merge word, a group-table slot,
+// an output or count index -- the kernels test it against its buffer or
+// shared-memory region; a violation sets a bit of this translation unit's
+// device error word and the access is skipped (no assert, no trap).  The host
+// side reads and clears the word after the launch (bev_check_take) and turns
+// a non-zero word into BEV_ERR_INTERNAL.  Without the flag every check is
+// `true` and compiles away.
+enum : unsigned {
+    kCheckBox = 1u,       // a group's texel box outside its feature map
+    kCheckMerge = 2u,     // a merge word outside the group's weight array
+    kCheckGroups = 4u,    // a group-table slot or member cell out of range
+    kCheckStore = 8u,     // an output / count / dout index outside its tensor
+};
+#ifdef BEV_BOUNDS_CHECK
+static __device__ unsigned g_check_word;
+__device__ __forceinline__ bool checked(bool ok, unsigned code) {
+    if (!ok) atomicOr(&g_check_word, code);
+    return ok;
+}
+// Read and clear the word of this translation unit (after the stream has
+// drained); host side.
+static inline unsigned check_take() {
+    unsigned w = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&w, g_check_word, sizeof(w)) != cudaSuccess) w = ~0u;
+    cudaMemcpyToSymbol(g_check_word, &z, sizeof(z));
+    return w;
+}
+#else
+__device__ __forceinline__ bool checked(bool, unsigned) { return true; }
+#endif
+
 constexpr int kCells = kTileI * kTileJ;  // cell = ci * kTileJ + cj
 constexpr int kZc = 16;                  // height bins per chunk of the count
 constexpr int kGmax = 8;                 // cells per group
@@ -373,7 +406,8 @@ __device__ inline void count_pass(const SampleArgs& a, const TileSm& s, int b, i
         const int cell = p * im.cpp + (int)threadIdx.x / im.LZ;
         if (in[p] && write_count) {
             const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
-            a.count[(((size_t)b * g.X + i) * g.Y + j) * g.Z + z0 + zz] = (uint8_t)cnt[p];
+            const size_t at = (((size_t)b * g.X + i) * g.Y + j) * g.Z + z0 + zz;
+            if (checked(at < (size_t)a.B * g.X * g.Y * g.Z, kCheckStore)) a.count[at] = (uint8_t)cnt[p];
         }
         if (cell < kCells && zz < zc) s.rc[cell * kZc + zz] = cnt[p] > 0 ? __frcp_rn((float)cnt[p]) : 0.0f;
     }
@@ -451,6 +485,7 @@ __device__ inline void form_groups(const TileSm& s, const unsigned short* xl) {
                 slot = 0;
                 n = 1;
             }
+            if (!checked(gi >= 0 && gi < kCells && slot < kGmax, kCheckGroups)) continue;
             s.grp[gi].cell[slot] = (unsigned char)c;
             if (slot == 0) {
                 s.grp[gi].n = n;
@@ -474,7 +509,12 @@ __device__ inline void form_groups(const TileSm& s, const unsigned short* xl) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         const int gi = lane + 32 * k;
-        if (gi < ng) ctl[kCtlOrder + atomicAdd(&hist[s.grp[gi].n], 1)] = gi;
+        if (gi < ng) {
+            const int n = s.grp[gi].n;
+            if (!checked(n >= 1 && n <= kGmax, kCheckGroups)) continue;
+            const int pos = atomicAdd(&hist[n], 1);
+            if (checked(pos >= 0 && pos < kCells, kCheckGroups)) ctl[kCtlOrder + pos] = gi;
+        }
     }
 }
 
@@ -591,6 +631,14 @@ __device__ __forceinline__ Members members_box(const GroupItems& it, const unsig
     return m;
 }
 
+// Whether a group's box lies inside its feature map (every gather load and
+// every gradient reduction of the group is inside the box); always true
+// outside the checked build.
+__device__ __forceinline__ bool box_inside(const Members& m, int Hf, int Wf) {
+    return checked(m.h <= 0 || m.w <= 0 || (m.y0 >= 0 && m.x0 >= 0 && m.y0 + m.h <= Hf && m.x0 + m.w <= Wf),
+                   kCheckBox);
+}
+
 // Sum w / cnt of every valid voxel of the members into the warp's region
 // ([texel of the union box][member] words), then round each entry to fp32
 // in place (the weights replace the 2^-20 words; the 2^-40 words are
@@ -621,8 +669,10 @@ __device__ inline void merge_members(const TileSm& s, const Members& m, const Gr
             if (!ok[q] || v == 0.0f) continue;
             int hi, lo;
             split_weight(v, hi, lo);
-            if (hi != 0) atomicAdd(&wh[e + off[q]], (unsigned)hi);
-            if (lo != 0) atomicAdd(reinterpret_cast<int*>(wl) + e + off[q], lo);
+            const int eq = e + off[q];
+            if (!checked(eq >= 0 && eq < m.entries && eq < kWarpEntries && k < m.slots, kCheckMerge)) continue;
+            if (hi != 0) atomicAdd(&wh[eq], (unsigned)hi);
+            if (lo != 0) atomicAdd(reinterpret_cast<int*>(wl) + eq, lo);
         }
     }
     __syncwarp();

@@ -33,6 +33,7 @@ from . import build as _build
 
 F32, BF16 = 0, 1
 NCHW, NHWC = 0, 1
+BEV_NOALLOC_SCRATCH_BYTES = 16 << 20  # include/bevsample.h: size of the built-in array of the no-alloc backward
 STATUS = {0: "BEV_OK", -1: "BEV_ERR_INVALID_ARG", -2: "BEV_ERR_UNSUPPORTED",
           -3: "BEV_ERR_WORKSPACE", -4: "BEV_ERR_CUDA", -5: "BEV_ERR_INTERNAL"}
 
@@ -73,6 +74,8 @@ def lib():
                                "(nvcc, sm_100a); this package has no CPU fallback")
         L = ctypes.CDLL(path)
         P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.bev_bounds_checked.argtypes = []
+        L.bev_bounds_checked.restype = I
         L.bev_grid_spec.argtypes = [P, P, ctypes.POINTER(BevGrid)]
         L.bev_grid_spec.restype = I
         L.bev_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
@@ -114,6 +117,11 @@ def lib():
         L.bev_status_string.restype = ctypes.c_char_p
         _lib = L
     return _lib
+
+
+def bev_bounds_checked() -> bool:
+    """True when the loaded library is the bounds-checked build."""
+    return bool(lib().bev_bounds_checked())
 
 
 def bev_status_string(status: int) -> str:
@@ -294,7 +302,12 @@ def bev_sample_backward_noalloc(dout: torch.Tensor, K: torch.Tensor, E: torch.Te
     """Feature gradient without a workspace, for callers that cannot allocate:
     the library accumulates in its own fixed 16 MiB device array.  ``out``
     ([B,N,C,Hf,Wf] fp32) must be supplied; this wrapper allocates nothing."""
+    if dout.dim() != 4 or dout.dtype != torch.float32 or not dout.is_contiguous():
+        raise ValueError("dout must be a contiguous fp32 [B,C,X,Y] tensor")
     B, C = dout.shape[:2]
+    if (tuple(out.shape) != (B, N, C, Hf, Wf) or out.dtype != torch.float32 or not out.is_contiguous()
+            or out.device != dout.device):
+        raise ValueError(f"out must be a contiguous fp32 tensor of shape {(B, N, C, Hf, Wf)} on {dout.device}")
     st = lib().bev_sample_backward_noalloc(
         dout.data_ptr(), B, N, C, Hf, Wf, K.data_ptr(), E.data_ptr(), int(img_h), int(img_w),
         ctypes.byref(grid), out.data_ptr(), _stream_ptr(stream))

@@ -136,6 +136,15 @@ int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, int Wf,
                         float* dfeatures, void* workspace, size_t workspace_bytes,
                         bev_stream_t stream);
 
+/* 1 when this library was built with device-side bounds checks
+ * (-DBEV_BOUNDS_CHECK, libbevsample_checked.so), else 0.  In that build the
+ * dense forward and backward kernels test every geometry-derived address --
+ * each group's texel box, merge word, group-table slot, output, count and dout
+ * index -- before using it; a failed test skips the access and sets a device
+ * error word, which the call reads back after draining `stream` (the call is
+ * then synchronous) and reports as BEV_ERR_INTERNAL.  Host only. */
+int bev_bounds_checked(void);
+
 /* Size of the built-in scratch array used by bev_sample_backward_noalloc. */
 #define BEV_NOALLOC_SCRATCH_BYTES (16u << 20)
 
@@ -154,9 +163,10 @@ int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, int Wf,
  * B * N * Hf * Wf * round_up(C, 4) * 4 bytes, exceeds it are rejected with
  * BEV_ERR_UNSUPPORTED before anything is enqueued.
  *
- * The first call on each device looks up that device's address of the array
- * (cudaGetSymbolAddress, with that device current) and caches it, so make the
- * first call on a device before capturing any stream.  All calls share the one
+ * The first call in each CUDA context looks up that context's address of the
+ * array (cudaGetSymbolAddress, with the context current) and caches it by
+ * device and context id, so make the first call on a device (and again after
+ * a cudaDeviceReset) before capturing any stream.  All calls share the one
  * array and leave their contents in it; each call clears what it uses before
  * accumulating.  Calls whose work may overlap on the GPU (other streams, other
  * host threads) race on the array: serialise them.  Nothing is allocated and

@@ -43,6 +43,27 @@ def test_status_strings(L):
     for s in (-1, -2, -3, -4, -5):
         assert ops.bev_status_string(s) not in ("ok", "unknown status")
     assert ops.bev_status_string(42) == "unknown status"
+    # a device-side check failure of the bounds-checked build is reported as
+    # BEV_ERR_INTERNAL, with its own text and name in the binding's error
+    assert ops.bev_status_string(-5) == "internal consistency check failed"
+    e = ops.BevError(-5, "bev_sample_forward")
+    assert e.status == -5 and "BEV_ERR_INTERNAL" in str(e) and "internal consistency" in str(e)
+
+
+def test_bounds_checked_library_exports_the_same_boundary(L):
+    """The normal library says it is not bounds-checked; its checked twin
+    exports every declared function and says it is."""
+    assert L.bev_bounds_checked() == 0
+    C = ctypes.CDLL(B.LIB_CHECKED)
+    for name in declared_functions():
+        assert hasattr(C, name), name
+    C.bev_bounds_checked.restype = ctypes.c_int
+    assert C.bev_bounds_checked() == 1
+
+
+def test_noalloc_size_constant_matches_the_header():
+    m = re.search(r"#define BEV_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", open(HEADER).read())
+    assert m and int(m.group(1)) << int(m.group(2)) == ops.BEV_NOALLOC_SCRATCH_BYTES
 
 
 def test_grid_spec(L):

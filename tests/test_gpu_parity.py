@@ -25,6 +25,32 @@ TOL = {"f32": 1e-5, "bf16": 2e-2}
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
+def naive_errors(got, ref):
+    """The naive figures reported beside the gate: the largest per-element
+    relative error among elements with |o| >= 1e-3 max|o|, and max|delta| /
+    max|o| (o = the oracle's output)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    top = float(np.abs(ref).max()) if ref.size else 0.0
+    if top == 0.0:
+        return {"rel_on_large": 0.0, "max_abs_over_max": 0.0}
+    big = np.abs(ref) >= 1e-3 * top
+    return {"rel_on_large": float((np.abs(got - ref)[big] / np.abs(ref[big])).max()),
+            "max_abs_over_max": float(np.abs(got - ref).max() / top)}
+
+
+def report(kind, got, ref, err):
+    """Print the gate and the naive figures; append them as a JSON line to
+    $BEV_PARITY_REPORT when that names a file."""
+    row = {"test": os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], "kind": kind,
+           "err_over_bound": err, **naive_errors(got, ref)}
+    print(json.dumps(row))
+    path = os.environ.get("BEV_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(row) + "\n")
+
+
 def rel_err(got, ref, bound):
     got = np.asarray(got, dtype=np.float64)
     zero = bound == 0
@@ -57,6 +83,7 @@ def check_forward(F, K, E, img_h, img_w, ranges, res, tol, layout=ops.NCHW):
     ref, bound, ref_cnt = oracle.forward(F, K, E, img_h, img_w, oracle.Grid(ranges, res))
     np.testing.assert_array_equal(cnt.numpy().astype(np.int32), ref_cnt)
     err = rel_err(out.numpy(), ref, bound)
+    report("forward", out.numpy(), ref, err)
     assert err <= tol, err
     return out, ref, ref_cnt, err
 
@@ -65,6 +92,7 @@ def check_backward(dout, K, E, img_h, img_w, ranges, res, N, Hf, Wf, tol=1e-5):
     dF = gpu_backward(dout, K, E, img_h, img_w, ranges, res, N, Hf, Wf)
     ref, bound = oracle.backward(dout, N, Hf, Wf, K, E, img_h, img_w, oracle.Grid(ranges, res))
     err = rel_err(dF.numpy(), ref, bound)
+    report("backward", dF.numpy(), ref, err)
     assert err <= tol, err
     return dF, ref, err
 

@@ -141,7 +141,10 @@ def test_oracle_matches_tensorized_forward(case):
     cell_ok = ~amb.any(axis=-1)                       # [B,X,Y]
     err = np.abs(out - ref.numpy()) / np.maximum(bound, 1e-30)
     err = np.where(bound > 0, err, np.abs(out - ref.numpy()))
-    assert err.transpose(0, 2, 3, 1)[cell_ok].max() < 2e-3
+    # away from the edge-ambiguous samples the fp64 tensorized form and the
+    # pinned-fp32 oracle differ by the geometry's rounding only (measured
+    # <= 5.3e-6 of the bound on these cases)
+    assert err.transpose(0, 2, 3, 1)[cell_ok].max() < 1e-5
 
 
 @pytest.mark.parametrize("case", CASES[:3] + CASES[5:], ids=[f"{c[0]}{c[1]}" for c in CASES[:3] + CASES[5:]])
@@ -158,7 +161,10 @@ def test_oracle_backward_matches_autograd_of_tensorized(case):
     assert np.abs(dF).max() > 0
     err = np.abs(dF - ref.numpy()) / np.maximum(dB, 1e-30)
     err = np.where(dB > 0, err, np.abs(dF - ref.numpy()))
-    assert err.max() < 2e-3
+    # a texel's bound can be dominated by small bilinear weights, which the
+    # fp64-vs-pinned-fp32 sample position (~1e-6 px) moves by ~1e-4 of
+    # themselves (measured <= 8.1e-5 of the bound on these cases)
+    assert err.max() < 2e-4
 
 
 # --------------------------------------------------------------------------
