@@ -263,28 +263,27 @@ __global__ void __launch_bounds__(kThreads, kTileCtas) sample_forward_kernel(con
     }
     __syncthreads();
 
-    // Store: each thread takes (channel, tile row) pairs and writes the row's
-    // 8 cells along y (two 16-byte stores where out allows).
-    constexpr int SL = 32 * CPL;  // channels of a slice (a power of two)
+    // Store: the row of 8 cells of one (channel, tile row) is 32 bytes along
+    // y; two neighbouring lanes take its two 16-byte halves, so that each
+    // warp store instruction writes whole 32-byte sectors.
+    constexpr int SL = 32 * CPL;        // channels of a slice (a power of two)
+    constexpr int HALVES = kTileJ / 4;  // 16-byte pieces of a tile row
     const int nch = min(SL, a.C - c_base);
-    for (int idx = threadIdx.x; idx < SL * kTileI; idx += kThreads) {
-        const int c = idx & (SL - 1), ci = idx / SL;
-        const int i = ti0 + ci;
+    for (int idx = threadIdx.x; idx < SL * kTileI * HALVES; idx += kThreads) {
+        const int hv = idx % HALVES, c = (idx / HALVES) & (SL - 1), ci = idx / (HALVES * SL);
+        const int i = ti0 + ci, j = tj0 + 4 * hv;
         if (c >= nch || i >= g.X) continue;
-        const float* tp = s.tile + ci * kTileJ * s.tile_stride + c;
-        float v[kTileJ];
-#pragma unroll
-        for (int cj = 0; cj < kTileJ; ++cj) v[cj] = tp[cj * s.tile_stride];
-        float* op = a.out + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + tj0;
+        const float* tp = s.tile + (ci * kTileJ + 4 * hv) * s.tile_stride + c;
+        const float v0 = tp[0], v1 = tp[s.tile_stride], v2 = tp[2 * s.tile_stride], v3 = tp[3 * s.tile_stride];
+        float* op = a.out + (((size_t)b * a.C + c_base + c) * g.X + i) * g.Y + j;
         if (!checked(b < a.B && c_base + c < a.C, kCheckStore)) continue;
-        if (a.out_vec && tj0 + kTileJ <= g.Y) {
-#pragma unroll
-            for (int q = 0; q < kTileJ / 4; ++q)
-                *reinterpret_cast<float4*>(op + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        if (a.out_vec && j + 4 <= g.Y) {
+            *reinterpret_cast<float4*>(op) = make_float4(v0, v1, v2, v3);
         } else {
+            const float v[4] = {v0, v1, v2, v3};
 #pragma unroll
-            for (int cj = 0; cj < kTileJ; ++cj)
-                if (tj0 + cj < g.Y) op[cj] = v[cj];
+            for (int q = 0; q < 4; ++q)
+                if (j + q < g.Y) op[q] = v[q];
         }
     }
 }
