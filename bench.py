@@ -104,7 +104,8 @@ def hbm_peak():
 
 
 KERNEL_SOURCES = {
-    "sample_forward_kernel": ["bev_forward.cu", "bev_tile.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
+    "sample_forward_kernel": ["bev_forward_rows.cu", "bev_forward_rows_ms.cu", "bev_forward_rows.cuh", "bev_rows.cuh",
+                              "bev_kernels.cuh", "bev_geometry.cuh"],
     "sample_backward_kernel": ["bev_backward.cu", "bev_tile.cuh", "bev_kernels.cuh", "bev_geometry.cuh"],
     "deform_forward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],
     "deform_backward_kernel": ["bev_deform.cu", "bev_deform.cuh", "bev_geometry.cuh"],

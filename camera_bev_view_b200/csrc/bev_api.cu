@@ -10,6 +10,7 @@
 #include "bev_deform.cuh"
 #include "bev_lss.cuh"
 #include "bev_kernels.cuh"
+#include "bev_rows.cuh"
 #include "bevsample.h"
 
 #define BEV_API extern "C" __attribute__((visibility("default")))
@@ -105,19 +106,76 @@ int cuda_status(cudaError_t e) {
 }
 
 // Status of a dense launch.  In the bounds-checked build the stream is
-// drained and the kernels' device error word read back: a check that failed
-// on the device gives BEV_ERR_INTERNAL.
-int dense_status(cudaError_t launch, cudaStream_t s, bool backward) {
+// drained and the kernel's device error word read back (by `take`): a check
+// that failed on the device gives BEV_ERR_INTERNAL.
+#ifdef BEV_BOUNDS_CHECK
+using CheckTake = unsigned (*)();
+#define BEV_TAKE(f) (f)
+#else
+using CheckTake = void*;
+#define BEV_TAKE(f) nullptr
+#endif
+
+int dense_status(cudaError_t launch, cudaStream_t s, CheckTake take) {
     const int st = cuda_status(launch);
 #ifdef BEV_BOUNDS_CHECK
     if (st != BEV_OK) return st;
     if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_status(cudaErrorUnknown);
-    return (backward ? bev_backward_check_take() : bev_forward_check_take()) ? BEV_ERR_INTERNAL : BEV_OK;
+    return take() ? BEV_ERR_INTERNAL : BEV_OK;
 #else
     (void)s;
-    (void)backward;
+    (void)take;
     return st;
 #endif
+}
+
+// Lanes per cell L and 16-byte chunks per lane V (<= 8) for a slice of qs
+// chunks (qs <= 32).  Eight lanes per cell is preferred: each load
+// instruction then covers whole 128-byte lines of four cells, and each lane
+// keeps 2V packed accumulators busy per texel.  Wider or narrower groups are
+// used only when eight lanes would leave more than a fifth of the lanes idle.
+void pick_lanes(int qs, int* L, int* V) {
+    const int order[4] = {8, 16, 32, 4};
+    for (int k = 0; k < 4; ++k) {
+        const int l = order[k], v = (qs + l - 1) / l;
+        if (v <= 8 && 5 * (l * v - qs) <= l * v) {
+            *L = l;
+            *V = v;
+            return;
+        }
+    }
+    int best_l = 4, best_v = (qs + 3) / 4, best_waste = 1 << 30;
+    for (int k = 0; k < 4; ++k) {
+        const int l = order[k], v = (qs + l - 1) / l;
+        if (v > 8) continue;
+        if (l * v - qs < best_waste) {
+            best_waste = l * v - qs;
+            best_l = l;
+            best_v = v;
+        }
+    }
+    *L = best_l;
+    *V = best_v;
+}
+
+
+// Launch shape of the row forward for Cp channels in chunks of cpc: channel
+// slices of up to kSliceMax channels, lanes per cell and chunks per lane;
+// returns the chunks per lane V (0 when the slices exceed the grid limit).
+int row_layout(bev::row::SampleArgs& a, int Cp, int cpc, const bev_grid_t* grid, int* slices) {
+    a.Qtot = Cp / cpc;
+    a.chan_per_chunk = cpc;
+    const int max_chunks = bev::row::kSliceMax / cpc;
+    *slices = (a.Qtot + max_chunks - 1) / max_chunks;
+    if (*slices > 65535) return 0;
+    a.slice_chunks = (a.Qtot + *slices - 1) / *slices;
+    int V;
+    pick_lanes(a.slice_chunks, &a.L, &V);
+    a.tile_j = bev::row::kTileJ;
+    a.tiles_i = (grid->X + bev::row::kTileI - 1) / bev::row::kTileI;
+    a.tiles_j = (grid->Y + bev::row::kTileJ - 1) / bev::row::kTileJ;
+    a.out_vec = (grid->Y % 4) == 0;
+    return V;
 }
 
 // Channel slices of the dense kernels: each lane of a warp owns cpl
@@ -243,8 +301,9 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
         if (st != BEV_OK) return st;
         feat = workspace;
     }
-    bev::SampleArgs a;
+    bev::row::SampleArgs a;
     memset(&a, 0, sizeof(a));
+    a.feat = feat;
     a.K = intrinsics;
     a.E = ego2cam;
     a.out = out;
@@ -253,13 +312,12 @@ BEV_API int bev_sample_forward(const void* features, int dtype, int layout, int 
     a.B = B;
     a.N = N;
     a.C = C;
-    single_level(a, Hf, Wf, img_h, img_w);
-    a.lv.feat[0] = feat;
-    a.texel_bytes = Cp * elem_size(dtype);
-    a.out_vec = ((uintptr_t)out % 16) == 0 && (grid->Y % 4) == 0;
-    const int slices = channel_slices(a, dtype == BEV_BF16, Cp);
-    tile_grid(a, grid);
-    return dense_status(bev_launch_forward(a, dtype == BEV_BF16, slices, s), s, false);
+    int slices;
+    const int V = row_layout(a, Cp, cpc, grid, &slices);
+    if (V == 0) return BEV_ERR_UNSUPPORTED;
+    a.out_vec = a.out_vec && ((uintptr_t)out % 16) == 0;
+    return dense_status(bev_launch_forward_rows(a, dtype == BEV_BF16, V, slices, s), s,
+                        BEV_TAKE(bev_launch_forward_rows_check_take));
 }
 
 BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, int Wf,
@@ -298,7 +356,8 @@ BEV_API int bev_sample_backward(const float* dout, int B, int N, int C, int Hf, 
     a.out_vec = ((uintptr_t)dout % 16) == 0 && (grid->Y % 4) == 0;
     const int slices = channel_slices(a, false, Cp);
     tile_grid(a, grid);
-    if ((st = dense_status(bev_launch_backward(a, slices, s), s, true)) != BEV_OK) return st;
+    if ((st = dense_status(bev_launch_backward(a, slices, s), s, BEV_TAKE(bev_backward_check_take))) != BEV_OK)
+        return st;
     return cuda_status(bev_launch_to_nchw(static_cast<const float*>(workspace), B * N, C, Hf * Wf, Cp,
                                           dfeatures, s));
 }
@@ -345,8 +404,9 @@ size_t ms_ws(int dtype, int layout, int B, int N, int C, int nlevels, const int*
     return total;
 }
 
-bev::LevelTable level_table(int nlevels, const int* Hf, const int* Wf, int img_h, int img_w) {
-    bev::LevelTable t;
+template <class Table>
+Table level_table(int nlevels, const int* Hf, const int* Wf, int img_h, int img_w) {
+    Table t;
     memset(&t, 0, sizeof(t));
     t.n = nlevels;
     for (int l = 0; l < nlevels; ++l) {
@@ -415,23 +475,25 @@ BEV_API int bev_sample_forward_multiscale(const void* const* features, int nleve
             base[l] = dst;
         }
     }
-    bev::SampleArgs a;
+    bev::row::SampleArgs a;
     memset(&a, 0, sizeof(a));
+    a.feat = base[0];
     a.K = intrinsics;
     a.E = ego2cam;
     a.out = out;
     a.count = valid_count;
     a.g = geo(grid, Hf[0], Wf[0], img_h, img_w);
-    a.lv = level_table(nlevels, Hf, Wf, img_h, img_w);
+    a.lv = level_table<bev::row::LevelTable>(nlevels, Hf, Wf, img_h, img_w);
     for (int l = 0; l < nlevels; ++l) a.lv.feat[l] = base[l];
     a.B = B;
     a.N = N;
     a.C = C;
-    a.texel_bytes = Cp * elem_size(dtype);
-    a.out_vec = ((uintptr_t)out % 16) == 0 && (grid->Y % 4) == 0;
-    const int slices = channel_slices(a, dtype == BEV_BF16, Cp);
-    tile_grid(a, grid);
-    return dense_status(bev_launch_forward(a, dtype == BEV_BF16, slices, s), s, false);
+    int slices;
+    const int V = row_layout(a, Cp, cpc, grid, &slices);
+    if (V == 0) return BEV_ERR_UNSUPPORTED;
+    a.out_vec = a.out_vec && ((uintptr_t)out % 16) == 0;
+    return dense_status(bev_launch_forward_rows_ms(a, dtype == BEV_BF16, V, slices, s), s,
+                        BEV_TAKE(bev_launch_forward_rows_ms_check_take));
 }
 
 BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const int* Hf, const int* Wf, int B,
@@ -469,7 +531,7 @@ BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const
     a.E = ego2cam;
     a.dout = dout;
     a.g = geo(grid, Hf[0], Wf[0], img_h, img_w);
-    a.lv = level_table(nlevels, Hf, Wf, img_h, img_w);
+    a.lv = level_table<bev::LevelTable>(nlevels, Hf, Wf, img_h, img_w);
     for (int l = 0; l < nlevels; ++l) a.lv.grad[l] = base[l];
     a.out_vec = ((uintptr_t)dout % 16) == 0 && (grid->Y % 4) == 0;
     a.B = B;
@@ -477,7 +539,8 @@ BEV_API int bev_sample_backward_multiscale(const float* dout, int nlevels, const
     a.C = C;
     const int slices = channel_slices(a, false, Cp);
     tile_grid(a, grid);
-    if ((st = dense_status(bev_launch_backward(a, slices, s), s, true)) != BEV_OK) return st;
+    if ((st = dense_status(bev_launch_backward(a, slices, s), s, BEV_TAKE(bev_backward_check_take))) != BEV_OK)
+        return st;
     for (int l = 0; l < nlevels; ++l) {
         st = cuda_status(bev_launch_to_nchw(base[l], B * N, C, Hf[l] * Wf[l], Cp,
                                             dfeatures[l], s));

@@ -82,14 +82,24 @@ inline cudaError_t set_smem_attributes(Kernel* k, size_t smem, int carveout,
 
 }  // namespace bev
 
-// Launchers (defined next to their kernels).  `slices` channel slices of
-// 32 * a.cpl channels each.
-cudaError_t bev_launch_forward(const bev::SampleArgs& a, bool bf16, int slices, cudaStream_t stream);
+// Launchers (defined next to their kernels).  The feature gradient: `slices`
+// channel slices of 32 * a.cpl channels each.
 cudaError_t bev_launch_backward(const bev::SampleArgs& a, int slices, cudaStream_t stream);
+// The forward (bev_rows.cuh): `slices` channel slices, L lanes per cell (in
+// the arguments) and V 16-byte chunks per lane.
+namespace bev {
+namespace row {
+struct SampleArgs;
+}
+}  // namespace bev
+cudaError_t bev_launch_forward_rows(const bev::row::SampleArgs& a, bool bf16, int V, int slices, cudaStream_t stream);
+cudaError_t bev_launch_forward_rows_ms(const bev::row::SampleArgs& a, bool bf16, int V, int slices,
+                                       cudaStream_t stream);
 #ifdef BEV_BOUNDS_CHECK
-// Checked build: read and clear the device error word of the dense forward /
-// backward kernels (call after the launch's stream has drained).
-unsigned bev_forward_check_take();
+// Checked build: read and clear the device error word of a dense kernel's
+// translation unit (call after the launch's stream has drained).
+unsigned bev_launch_forward_rows_check_take();
+unsigned bev_launch_forward_rows_ms_check_take();
 unsigned bev_backward_check_take();
 #endif
 cudaError_t bev_launch_to_channels_last(const void* src, int layout, int esize, int BN, int C,
