@@ -130,11 +130,23 @@ int dense_status(cudaError_t launch, cudaStream_t s, CheckTake take) {
 }
 
 // Lanes per cell L and 16-byte chunks per lane V (<= 8) for a slice of qs
-// chunks (qs <= 32).  Eight lanes per cell is preferred: each load
-// instruction then covers whole 128-byte lines of four cells, and each lane
-// keeps 2V packed accumulators busy per texel.  Wider or narrower groups are
-// used only when eight lanes would leave more than a fifth of the lanes idle.
+// chunks (qs <= 32).  An exact fit with at most five chunks a lane comes
+// first, eight lanes per cell before four, 16 and 32: each load instruction
+// of eight lanes covers whole 128-byte lines of four cells, and no lane
+// idles (80 fp32 channels take four lanes of five chunks, which measured 10%
+// faster than eight lanes of three with a sixth of the slots idle).  Without
+// an exact fit, eight lanes are kept unless they would leave more than a
+// fifth of the slots idle.
 void pick_lanes(int qs, int* L, int* V) {
+    const int exact[4] = {8, 4, 16, 32};
+    for (int k = 0; k < 4; ++k) {
+        const int l = exact[k], v = qs / l;
+        if (v >= 1 && v <= 5 && l * v == qs) {
+            *L = l;
+            *V = v;
+            return;
+        }
+    }
     const int order[4] = {8, 16, 32, 4};
     for (int k = 0; k < 4; ++k) {
         const int l = order[k], v = (qs + l - 1) / l;

@@ -291,14 +291,15 @@ __device__ __forceinline__ void forward_body(const SampleArgs& a) {
 }
 
 template <bool BF16, int L, int V>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_kernel(const SampleArgs a) {
+__global__ void __launch_bounds__(kThreads, (fwd_ctas_per_sm<BF16, L, V, false>())) sample_forward_kernel(const SampleArgs a) {
     forward_body<BF16, L, V, false>(a);
 }
 
 // The level table is indexed at run time: __grid_constant__ lets the body
 // read it in place from the parameter space.
 template <bool BF16, int L, int V>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) sample_forward_ms_kernel(const __grid_constant__ SampleArgs a) {
+__global__ void __launch_bounds__(kThreads, (fwd_ctas_per_sm<BF16, L, V, true>()))
+    sample_forward_ms_kernel(const __grid_constant__ SampleArgs a) {
     forward_body<BF16, L, V, true>(a);
 }
 
@@ -310,7 +311,7 @@ static cudaError_t launch_one(const SampleArgs& a, dim3 grid, size_t smem, cudaS
     else
         k = sample_forward_kernel<BF16, L, V>;
     static std::atomic<long long> attrs[kAttrDevices];
-    const cudaError_t e = set_smem_attributes(k, smem, carveout_percent(smem, kCtasPerSm), attrs);
+    const cudaError_t e = set_smem_attributes(k, smem, carveout_percent(smem, fwd_ctas_per_sm<BF16, L, V, MS>()), attrs);
     if (e != cudaSuccess) return e;
     k<<<grid, kThreads, smem, st>>>(a);
     return cudaGetLastError();

@@ -70,9 +70,23 @@ constexpr int kStageStride = kCellsPerWarp + 1;
 constexpr int kWarpBytes = 2 * sizeof(int) * kWarpPatchCap;
 static_assert((int)sizeof(float) * kSliceMax * kStageStride <= kWarpBytes + 512,
               "staging tile must fit the warp region");
-// CTAs kept resident per SM; shared memory stays small (~34 KB) so that most
-// of the SM's on-chip array serves as L1 for the tiles' texel windows.
-constexpr int kCtasPerSm = 3;
+// CTAs kept resident per SM, per instantiation: three (at most 85 registers
+// a thread) when the per-lane state fits -- the accumulators (cell rounds x
+// chunks x fp32 pairs), the four corners' loads of each chunk (16 registers a
+// chunk) and the two cached projections -- and two (up to 128 registers)
+// when it would spill: the larger slices measured 5 to 14% faster without the
+// spills than with the third CTA.  The multi-scale kernel, which also carries
+// the level loop, measured faster with two.  Shared memory stays small
+// (~38 KB a CTA) so that most of the SM's on-chip array serves as L1 for the
+// tiles' texel windows.
+template <bool BF16, int L, int V, bool MS>
+constexpr int fwd_ctas_per_sm() {
+    constexpr int pairs = BF16 ? 4 : 2;                 // fp32 pairs per 16-byte chunk
+    constexpr int rounds = kCellsPerWarp / (32 / L);    // cell rounds per warp
+    constexpr int zn = z_per_lane_fwd<BF16, L>();
+    constexpr int regs = rounds * V * pairs * 2 + 16 * V + 8 * zn;
+    return (!MS && regs <= 56) ? 3 : 2;
+}
 
 // Feature-pyramid levels of the multi-scale operator.  Every level shares
 // the voxel's projection, validity and count; level l samples its own map at
@@ -306,16 +320,26 @@ __device__ __forceinline__ int group_prefix(int size, int sub, int* total) {
     return before;
 }
 
-// Exact fixed point of the merged weights.  A contribution v = w / cnt (<= 1,
-// fp32) is split into hi = floor(v * 2^20) and lo = round((v - hi 2^-20) 2^40)
-// (the subtraction is exact, lo < 2^20); the halves are summed with 32-bit
-// integer atomics (at most kZPerLaneMax * 32 contributions reach one entry, so
-// neither overflows), and the total hi 2^-20 + lo 2^-40 is independent of the
-// order of the additions.  It is rounded to fp32 once.
+// Exact fixed point of the merged weights.  A contribution v = w / cnt (in
+// [0, 1], fp32) is split into hi = RN(v 2^20) and lo = RN((v 2^20 - hi) 2^20),
+// |lo| <= 2^19.  Both roundings to an integer are done by adding 1.5 * 2^23 in
+// fp32 (the sum lies in [2^23, 2^24), where fp32 spacing is 1) and reading
+// the integer off the bit pattern; the residual v 2^20 - hi is exact (one
+// fma).  The halves are summed with 32-bit integer atomics (at most
+// kZPerLaneMax * 32 contributions reach one entry, so neither overflows), and
+// the total hi 2^-20 + lo 2^-40 is independent of the order of the additions.
+// It is rounded to fp32 once.
 constexpr float kTwo20 = 1048576.0f;
 constexpr float kTwoM20 = 9.5367431640625e-07f;
-constexpr float kTwo40 = 1099511627776.0f;
 constexpr float kTwoM40 = 9.094947017729282379150390625e-13f;
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ void split_weight(float v, int& hi, int& lo) {
+    const float t = __fmaf_rn(v, kTwo20, kRound);
+    hi = __float_as_int(t) - __float_as_int(kRound);
+    const float r = __fmaf_rn(v, kTwo20, -__fsub_rn(t, kRound));  // exact residual, |r| <= 0.5
+    lo = __float_as_int(__fmaf_rn(r, kTwo20, kRound)) - __float_as_int(kRound);
+}
 
 // One cell group's projections for one camera in one height chunk: ZN bins
 // per lane.
@@ -445,9 +469,8 @@ __device__ __forceinline__ void merge_patches(Patch& p, const Items<ZN>& it, con
                 for (int k = 0; k < 4; ++k) {
                     const int yy = c.y0 + (k >> 1), xx = c.x0 + (k & 1);
                     if ((unsigned)yy >= (unsigned)Hf || (unsigned)xx >= (unsigned)Wf) continue;
-                    const float v = ws[k] * rc[t];
-                    const int qh = __float2int_rd(v * kTwo20);
-                    const int ql_ = __float2int_rn(__fmul_rn(__fsub_rn(v, (float)qh * kTwoM20), kTwo40));
+                    int qh, ql_;
+                    split_weight(__fmul_rn(ws[k], rc[t]), qh, ql_);
                     const int e = p.off + (yy - p.y0) * p.w + (xx - p.x0);
                     if (!checked(e >= p.off && e < p.off + n && e < kWarpPatchCap, kCheckMerge)) continue;
                     if (ql_ != 0) atomicAdd(&lo[e], ql_);
