@@ -12,9 +12,10 @@
 // batch item, so no pillar sum can overflow) and added with integer
 // reductions in L2: integer addition is exact and associative, so the sums
 // do not depend on the order in which the points arrive, and one pass over
-// the points suffices.  Bins of one pixel that land in the same pillar are
-// merged in registers first.  A final transpose converts the channels-last
-// integer sums to the fp32 [B,C,X,Y] output.
+// the points suffices.  Consecutive rows of one image column whose bins of
+// one depth land in the same pillar are merged in registers first.  A final
+// transpose converts the channels-last integer sums to the fp32 [B,C,X,Y]
+// output.
 //
 // Backward (a gather, deterministic): dout is made channels-last; each
 // pixel's bins read the dout vector of their pillar:
@@ -154,65 +155,100 @@ __global__ void __launch_bounds__(256) lss_maxabs_kernel(const float* __restrict
     }
 }
 
-// One warp per pixel (b, n, h, w); lanes take channels c = lane + 32 v.
-template <int V>
-__global__ void __launch_bounds__(256) lss_forward_kernel(const LssArgs a) {
-    const int lane = threadIdx.x & 31;
-    const long long pix = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const long long npix = (long long)a.B * a.N * a.Hf * a.Wf;
-    if (pix >= npix) return;
-    const int w = (int)(pix % a.Wf);
-    const int h = (int)((pix / a.Wf) % a.Hf);
-    const long long bn = pix / ((long long)a.Hf * a.Wf);
+// Forward over a block of the feature map: rows h0 .. h0 + kLssRows and
+// columns w0 .. w0 + kLssCols of one camera (b, n), depth bins k0 .. k0 +
+// a.bins_per_cta (at most kLssBins; fewer when the launch would otherwise
+// give under two CTAs per SM).  The CTA stages the block's rays, depths and pillars, then the
+// features channels-last in chunks of kLssChunk channels (global loads run
+// along w, the contiguous axis).  A warp then takes one (column, bin) at a
+// time and walks its rows.  For a camera without pitch or roll the image row
+// moves a point only in ego height, so the bins of one depth along one image
+// column share their pillar (LSS tutorial, "Splat": pillars bin the ground
+// plane only); consecutive rows with one pillar are summed in registers and
+// sent as one 64-bit reduction per channel, and rows of other pillars (a
+// tilted camera) start new runs.  Each term is converted to fixed point on its own, so the integer
+// sums, and the output, do not depend on how the terms are grouped.
+constexpr int kLssCols = 8, kLssRows = 16, kLssBins = 8, kLssChunk = 64;
+constexpr int kLssPix = kLssCols * kLssRows;
+constexpr int kLssThreads = 256;
+
+__global__ void __launch_bounds__(kLssThreads) lss_forward_kernel(const LssArgs a) {
+    __shared__ float fs[kLssPix * (kLssChunk + 1)];  // [pixel][channel of the chunk]; pixel = r * kLssCols + x
+    __shared__ float ds[kLssBins * kLssPix];         // [bin][pixel]: depth probability
+    __shared__ int ps[kLssBins * kLssPix];           // [bin][pixel]: pillar, or -1
+    __shared__ float rx[kLssPix], ry[kLssPix];       // the pixels' rays
+    const int nwb = (a.Wf + kLssCols - 1) / kLssCols;
+    const int w0 = (int)(blockIdx.x % nwb) * kLssCols, h0 = (int)(blockIdx.x / nwb) * kLssRows;
+    const int k0 = blockIdx.y * a.bins_per_cta, kn = min(a.bins_per_cta, a.D - k0);
+    const long long bn = blockIdx.z;
     const int b = (int)(bn / a.N);
     const float* K = a.K + bn * 9;
     const float* E = a.E + bn * 16;
     const size_t hw = (size_t)a.Hf * a.Wf;
-    const size_t poff = (size_t)h * a.Wf + w;
-    const float scale = pow2f(lss_frac_bits(a));
-    const Ray ray = lss_ray(a, K, h, w);
-    float f[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-        const int c = lane + 32 * v;
-        f[v] = c < a.C ? a.feat[((size_t)bn * a.C + c) * hw + poff] : 0.0f;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < kLssPix) {
+        const int h = h0 + tid / kLssCols, w = w0 + tid % kLssCols;
+        Ray ray = {0.0f, 0.0f};
+        if (h < a.Hf && w < a.Wf) ray = lss_ray(a, K, h, w);
+        rx[tid] = ray.xn;
+        ry[tid] = ray.yn;
     }
-    unsigned long long* acc = a.acc + (size_t)b * a.X * a.Y * a.C;
-    long long run[V];
-    int run_cell = -1;
-    for (int k0 = 0; k0 < a.D; k0 += 32) {
-        const int k = k0 + lane;
+    __syncthreads();
+    for (int t = tid; t < kLssBins * kLssPix; t += kLssThreads) {
+        const int kk = t / kLssPix, pix = t % kLssPix;
+        const int h = h0 + pix / kLssCols, w = w0 + pix % kLssCols;
         int cell = -1;
         float al = 0.0f;
-        if (k < a.D) {
-            cell = lss_cell(a, ray, E, k);
-            al = a.depth[((size_t)bn * a.D + k) * hw + poff];
+        if (kk < kn && h < a.Hf && w < a.Wf) {
+            const Ray ray = {rx[pix], ry[pix]};
+            cell = lss_cell(a, ray, E, k0 + kk);
+            al = a.depth[((size_t)bn * a.D + k0 + kk) * hw + (size_t)h * a.Wf + w];
         }
-        const int kn = min(32, a.D - k0);
-        for (int kk = 0; kk < kn; ++kk) {
-            const int ck = __shfl_sync(0xffffffffu, cell, kk);
-            const float ak = __shfl_sync(0xffffffffu, al, kk);
-            if (ck < 0) continue;
-            if (ck != run_cell) {
-                if (run_cell >= 0) {
-#pragma unroll
-                    for (int v = 0; v < V; ++v)
-                        if (lane + 32 * v < a.C)
-                            atomicAdd(acc + (size_t)run_cell * a.C + lane + 32 * v, (unsigned long long)run[v]);
-                }
-                run_cell = ck;
-#pragma unroll
-                for (int v = 0; v < V; ++v) run[v] = 0;
-            }
-#pragma unroll
-            for (int v = 0; v < V; ++v) run[v] += __float2ll_rn(__fmul_rn(__fmul_rn(ak, f[v]), scale));
-        }
+        ps[t] = cell;
+        ds[t] = al;
     }
-    if (run_cell >= 0) {
+    const float scale = pow2f(lss_frac_bits(a));
+    unsigned long long* acc = a.acc + (size_t)b * a.X * a.Y * a.C;
+    for (int c0 = 0; c0 < a.C; c0 += kLssChunk) {
+        __syncthreads();  // pillars staged; the previous chunk's reads done
+        for (int t = tid; t < kLssChunk * kLssPix; t += kLssThreads) {
+            const int cl = t / kLssPix, pix = t % kLssPix;
+            const int h = h0 + pix / kLssCols, w = w0 + pix % kLssCols, c = c0 + cl;
+            fs[pix * (kLssChunk + 1) + cl] =
+                (c < a.C && h < a.Hf && w < a.Wf) ? a.feat[((size_t)bn * a.C + c) * hw + (size_t)h * a.Wf + w] : 0.0f;
+        }
+        __syncthreads();
+        bool on[2];
 #pragma unroll
-        for (int v = 0; v < V; ++v)
-            if (lane + 32 * v < a.C)
-                atomicAdd(acc + (size_t)run_cell * a.C + lane + 32 * v, (unsigned long long)run[v]);
+        for (int v = 0; v < 2; ++v) on[v] = c0 + lane + 32 * v < a.C;
+        for (int it = warp; it < kLssCols * kn; it += kLssThreads / 32) {
+            const int x = it % kLssCols, kk = it / kLssCols;
+            long long run[2] = {0, 0};
+            int run_cell = -1;
+            for (int r = 0; r < kLssRows; ++r) {
+                const int pix = r * kLssCols + x;
+                const int ck = ps[kk * kLssPix + pix];
+                if (ck < 0) continue;
+                if (ck != run_cell) {
+                    if (run_cell >= 0) {
+#pragma unroll
+                        for (int v = 0; v < 2; ++v)
+                            if (on[v]) atomicAdd(acc + (size_t)run_cell * a.C + c0 + lane + 32 * v, (unsigned long long)run[v]);
+                    }
+                    run_cell = ck;
+                    run[0] = run[1] = 0;
+                }
+                const float ak = ds[kk * kLssPix + pix];
+#pragma unroll
+                for (int v = 0; v < 2; ++v)
+                    run[v] += __float2ll_rn(__fmul_rn(__fmul_rn(ak, fs[pix * (kLssChunk + 1) + lane + 32 * v]), scale));
+            }
+            if (run_cell >= 0) {
+#pragma unroll
+                for (int v = 0; v < 2; ++v)
+                    if (on[v]) atomicAdd(acc + (size_t)run_cell * a.C + c0 + lane + 32 * v, (unsigned long long)run[v]);
+            }
+        }
     }
 }
 
@@ -323,20 +359,15 @@ cudaError_t bev_launch_lss_forward(const bev::LssArgs& a, cudaStream_t st) {
     const size_t mx = (nd > nf ? nd : nf);
     const int mblocks = (int)((mx / 4 + 255) / 256 < 148 * 4 ? (mx / 4 + 255) / 256 + 1 : 148 * 4);
     lss_maxabs_kernel<<<mblocks, 256, 0, st>>>(a.depth, nd, a.feat, nf, a.maxabs);
-    const long long npix = (long long)a.B * a.N * a.Hf * a.Wf;
-    const unsigned blocks = (unsigned)((npix + 7) / 8);
-    const int V = (a.C + 31) / 32;
-    switch (V) {
-        case 1: lss_forward_kernel<1><<<blocks, 256, 0, st>>>(a); break;
-        case 2: lss_forward_kernel<2><<<blocks, 256, 0, st>>>(a); break;
-        case 3: lss_forward_kernel<3><<<blocks, 256, 0, st>>>(a); break;
-        case 4: lss_forward_kernel<4><<<blocks, 256, 0, st>>>(a); break;
-        case 5: lss_forward_kernel<5><<<blocks, 256, 0, st>>>(a); break;
-        case 6: lss_forward_kernel<6><<<blocks, 256, 0, st>>>(a); break;
-        case 7: lss_forward_kernel<7><<<blocks, 256, 0, st>>>(a); break;
-        case 8: lss_forward_kernel<8><<<blocks, 256, 0, st>>>(a); break;
-        default: return cudaErrorInvalidValue;
-    }
+    const long long nblk = (long long)((a.Hf + kLssRows - 1) / kLssRows) * ((a.Wf + kLssCols - 1) / kLssCols);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    LssArgs f = a;
+    f.bins_per_cta = kLssBins;
+    while (f.bins_per_cta > 1 && nblk * a.B * a.N * ((a.D + f.bins_per_cta - 1) / f.bins_per_cta) < 2LL * sms)
+        f.bins_per_cta >>= 1;
+    const dim3 fgrid((unsigned)nblk, (unsigned)((a.D + f.bins_per_cta - 1) / f.bins_per_cta), (unsigned)(a.B * a.N));
+    lss_forward_kernel<<<fgrid, kLssThreads, 0, st>>>(f);
     const int XY = a.X * a.Y;
     const dim3 grid((XY + 31) / 32, (a.C + 31) / 32, a.B);
     lss_convert_kernel<<<grid, dim3(32, 8), 0, st>>>(a);

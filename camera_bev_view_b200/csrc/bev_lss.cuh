@@ -27,6 +27,7 @@ struct LssArgs {
     float dmin, dstep;
     float xmin, ymin, zmin, zmax, dx, dy;
     long long points_per_batch;   // N * D * Hf * Wf
+    int bins_per_cta;             // forward: depth bins per CTA (1, 2, 4 or 8), set by the launcher
 };
 
 }  // namespace bev
