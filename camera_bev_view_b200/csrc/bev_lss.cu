@@ -351,6 +351,141 @@ __global__ void __launch_bounds__(kLssWarps * 32) lss_backward_kernel(const LssA
     }
 }
 
+// Backward over a block of the feature map: rows h0 .. h0 + kLssRows and
+// columns w0 .. w0 + kLssBwdCols of one camera.  Warp w takes column
+// w % kLssBwdCols and the bins k of parity w / kLssBwdCols; it holds its
+// column's features (one 64-channel chunk at a time, staged channels-last
+// with loads along w) and the feature-gradient partials of its rows in
+// registers.  Walking the rows of one bin, it reads a pillar's dout vector
+// once per run of rows that share the pillar (a camera without pitch or roll
+// puts the whole column in one pillar, as in the forward), where the
+// per-pixel kernel reads it once per pixel.  The two parities' partials are
+// added in a fixed order, and a later channel chunk adds its dot products to
+// the depth gradient after the earlier ones, so the result is deterministic.
+constexpr int kLssBwdCols = 4, kLssBwdPar = 2;
+constexpr int kLssBwdPix = kLssBwdCols * kLssRows;
+constexpr int kLssBwdThreads = 32 * kLssBwdCols * kLssBwdPar;
+
+__global__ void __launch_bounds__(kLssBwdThreads) lss_backward_cols_kernel(const LssArgs a) {
+    __shared__ float fs[kLssBwdPix * (kLssChunk + 1)];   // [pixel][channel of the chunk]; pixel = r * kLssBwdCols + x
+    __shared__ float dfs[kLssBwdPix * (kLssChunk + 1)];  // the odd-bin warps' feature-gradient partials
+    __shared__ float rx[kLssBwdPix], ry[kLssBwdPix];
+    const int nwb = (a.Wf + kLssBwdCols - 1) / kLssBwdCols;
+    const int w0 = (int)(blockIdx.x % nwb) * kLssBwdCols, h0 = (int)(blockIdx.x / nwb) * kLssRows;
+    const long long bn = blockIdx.y;
+    const int b = (int)(bn / a.N);
+    const float* K = a.K + bn * 9;
+    const float* E = a.E + bn * 16;
+    const size_t hw = (size_t)a.Hf * a.Wf;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int x = warp % kLssBwdCols, kp = warp / kLssBwdCols, w = w0 + x;
+    const float* G = a.dout_cl + (size_t)b * a.X * a.Y * a.C;
+    if (tid < kLssBwdPix) {
+        const int h = h0 + tid / kLssBwdCols, ww = w0 + tid % kLssBwdCols;
+        Ray ray = {0.0f, 0.0f};
+        if (h < a.Hf && ww < a.Wf) ray = lss_ray(a, K, h, ww);
+        rx[tid] = ray.xn;
+        ry[tid] = ray.yn;
+    }
+    for (int c0 = 0; c0 < a.C; c0 += kLssChunk) {
+        __syncthreads();  // rays staged; the previous chunk's shared reads done
+        for (int t = tid; t < kLssChunk * kLssBwdPix; t += kLssBwdThreads) {
+            const int cl = t / kLssBwdPix, pix = t % kLssBwdPix;
+            const int h = h0 + pix / kLssBwdCols, ww = w0 + pix % kLssBwdCols, c = c0 + cl;
+            fs[pix * (kLssChunk + 1) + cl] =
+                (c < a.C && h < a.Hf && ww < a.Wf) ? a.feat[((size_t)bn * a.C + c) * hw + (size_t)h * a.Wf + ww] : 0.0f;
+        }
+        __syncthreads();
+        const bool on0 = c0 + lane < a.C, on1 = c0 + lane + 32 < a.C;
+        float f[kLssRows][2], df[kLssRows][2];
+#pragma unroll
+        for (int r = 0; r < kLssRows; ++r) {
+            const float* fp = fs + (r * kLssBwdCols + x) * (kLssChunk + 1) + lane;
+            f[r][0] = fp[0];
+            f[r][1] = fp[32];
+            df[r][0] = df[r][1] = 0.0f;
+        }
+        const int h = h0 + lane;
+        const bool row_ok = lane < kLssRows && h < a.Hf && w < a.Wf;
+        const Ray ray = {row_ok ? rx[lane * kLssBwdCols + x] : 0.0f, row_ok ? ry[lane * kLssBwdCols + x] : 0.0f};
+        // this lane's row: pillar and depth of the warp's next bin, fetched one
+        // bin ahead so that their latency overlaps the current bin's rows
+        int cell_n = -1;
+        float al_n = 0.0f;
+        if (row_ok && kp < a.D) {
+            cell_n = lss_cell(a, ray, E, kp);
+            al_n = a.depth[((size_t)bn * a.D + kp) * hw + (size_t)h * a.Wf + w];
+        }
+        for (int k = kp; k < a.D; k += kLssBwdPar) {
+            const int cell = cell_n;
+            const float al = al_n;
+            cell_n = -1;
+            al_n = 0.0f;
+            if (row_ok && k + kLssBwdPar < a.D) {
+                cell_n = lss_cell(a, ray, E, k + kLssBwdPar);
+                al_n = a.depth[((size_t)bn * a.D + k + kLssBwdPar) * hw + (size_t)h * a.Wf + w];
+            }
+            // per lane: its two channels' share of each row's dot product
+            float q[kLssRows];
+            float g0 = 0.0f, g1 = 0.0f;
+            int cur = -1;
+#pragma unroll
+            for (int r = 0; r < kLssRows; ++r) {
+                const int ck = __shfl_sync(0xffffffffu, cell, r);
+                const float ak = __shfl_sync(0xffffffffu, al, r);
+                q[r] = 0.0f;
+                if (ck < 0) continue;
+                if (ck != cur) {
+                    cur = ck;
+                    g0 = on0 ? G[(size_t)ck * a.C + c0 + lane] : 0.0f;
+                    g1 = on1 ? G[(size_t)ck * a.C + c0 + lane + 32] : 0.0f;
+                }
+                q[r] = __fmaf_rn(g1, f[r][1], __fmul_rn(g0, f[r][0]));
+                df[r][0] = __fmaf_rn(ak, g0, df[r][0]);
+                df[r][1] = __fmaf_rn(ak, g1, df[r][1]);
+            }
+            // reduce the 16 rows over the 32 lanes at once (recursive halving:
+            // at each step a lane keeps half of its rows and adds its partner's
+            // share of them); lanes 2r and 2r + 1 end with row r's total
+#pragma unroll
+            for (int half = kLssRows / 2, o = 16; half >= 1; half >>= 1, o >>= 1) {
+                const bool up = (lane & o) != 0;
+#pragma unroll
+                for (int i = 0; i < half; ++i) {
+                    const float send = up ? q[i] : q[i + half];
+                    const float keep = up ? q[i + half] : q[i];
+                    q[i] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                }
+            }
+            const float dd = __fadd_rn(q[0], __shfl_xor_sync(0xffffffffu, q[0], 1));
+            const int hr = h0 + (lane >> 1);
+            if ((lane & 1) == 0 && hr < a.Hf && w < a.Wf) {
+                float* p = a.ddepth + ((size_t)bn * a.D + k) * hw + (size_t)hr * a.Wf + w;
+                *p = c0 == 0 ? dd : __fadd_rn(*p, dd);
+            }
+        }
+        if (kp == 1) {
+#pragma unroll
+            for (int r = 0; r < kLssRows; ++r) {
+                float* dp = dfs + (r * kLssBwdCols + x) * (kLssChunk + 1) + lane;
+                dp[0] = df[r][0];
+                dp[32] = df[r][1];
+            }
+        }
+        __syncthreads();
+        if (kp == 0 && w < a.Wf) {
+#pragma unroll
+            for (int r = 0; r < kLssRows; ++r) {
+                if (h0 + r >= a.Hf) break;
+                const float* dp = dfs + (r * kLssBwdCols + x) * (kLssChunk + 1) + lane;
+                float* out = a.dfeat + ((size_t)bn * a.C + c0 + lane) * hw + (size_t)(h0 + r) * a.Wf + w;
+                if (on0) out[0] = __fadd_rn(df[r][0], dp[0]);
+                if (on1) out[32 * hw] = __fadd_rn(df[r][1], dp[32]);
+            }
+        }
+    }
+}
+
 }  // namespace bev
 
 cudaError_t bev_launch_lss_forward(const bev::LssArgs& a, cudaStream_t st) {
@@ -376,6 +511,15 @@ cudaError_t bev_launch_lss_forward(const bev::LssArgs& a, cudaStream_t st) {
 
 cudaError_t bev_launch_lss_backward(const bev::LssArgs& a, cudaStream_t st) {
     using namespace bev;
+    // Column blocks when they give at least one CTA per SM; one CTA per pixel
+    // otherwise (small maps, where the blocks would leave SMs idle).
+    const long long nblk = (long long)((a.Hf + kLssRows - 1) / kLssRows) * ((a.Wf + kLssBwdCols - 1) / kLssBwdCols);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (nblk * a.B * a.N >= sms) {
+        lss_backward_cols_kernel<<<dim3((unsigned)nblk, (unsigned)(a.B * a.N)), kLssBwdThreads, 0, st>>>(a);
+        return cudaGetLastError();
+    }
     const long long npix = (long long)a.B * a.N * a.Hf * a.Wf;
     const int V = (a.C + 31) / 32;
     const dim3 grid((unsigned)npix);
