@@ -253,20 +253,24 @@ __global__ void __launch_bounds__(kLssThreads) lss_forward_kernel(const LssArgs 
 }
 
 // Fixed-point channels-last sums [B][X*Y][C] -> fp32 out [B][C][X*Y], 32x32
-// tiles through shared memory.
+// tiles through shared memory.  Each sum is widened to double and scaled by
+// 2^-s (an exact multiply by a power of two), then rounded to fp32.  A thread
+// issues its four loads before converting any of them.
 __global__ void __launch_bounds__(256) lss_convert_kernel(const LssArgs a) {
     __shared__ float tile[32][33];
     const int b = blockIdx.z;
     const int p0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
     const int XY = a.X * a.Y;
-    const int s = lss_frac_bits(a);
+    const double inv = __longlong_as_double((long long)(1023 - lss_frac_bits(a)) << 52);  // 2^-s
     const unsigned long long* acc = a.acc + (size_t)b * XY * a.C;
-    for (int r = threadIdx.y; r < 32; r += 8) {
-        const int p = p0 + r, c = c0 + threadIdx.x;
-        float v = 0.0f;
-        if (p < XY && c < a.C) v = (float)ldexp((double)(long long)acc[(size_t)p * a.C + c], -s);
-        tile[r][threadIdx.x] = v;
+    long long v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int p = p0 + threadIdx.y + 8 * q, c = c0 + threadIdx.x;
+        v[q] = (p < XY && c < a.C) ? (long long)__ldg(acc + (size_t)p * a.C + c) : 0;
     }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tile[threadIdx.y + 8 * q][threadIdx.x] = __double2float_rn(__ll2double_rn(v[q]) * inv);
     __syncthreads();
     for (int r = threadIdx.y; r < 32; r += 8) {
         const int c = c0 + r, p = p0 + threadIdx.x;
