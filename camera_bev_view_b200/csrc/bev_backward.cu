@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, kTileCtas) sample_backward_kernel(co
 
     for (int z0 = 0; z0 < g.Z; z0 += kZc) {
         const int zc = min(kZc, g.Z - z0);
-        count_pass(a, s, b, ti0, tj0, z0, zc, false);
+        count_pass(a, s, ti0, tj0, z0, zc);
         if (z0 == 0) {
 #pragma unroll
             for (int it = 0; it < kIt; ++it) {

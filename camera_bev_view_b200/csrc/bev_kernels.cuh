@@ -27,22 +27,18 @@ struct LevelTable {
     int n;                            // levels, 1 .. kMaxLevels
     int Hf[kMaxLevels], Wf[kMaxLevels];
     float sW[kMaxLevels], sH[kMaxLevels];  // (float)W_l / img_w, (float)H_l / img_h, host IEEE divide
-    const void* feat[kMaxLevels];     // forward: channels-last features of level l
-    float* grad[kMaxLevels];          // backward: fp32 channels-last gradient buffer of level l
+    float* grad[kMaxLevels];          // fp32 channels-last gradient buffer of level l
 };
 
 struct SampleArgs {
     const float* K;         // [B,N,3,3]
     const float* E;         // [B,N,4,4]
-    float* out;             // forward: [B,C,X,Y]
-    uint8_t* count;         // forward: [B,X,Y,Z] or null
-    const float* dout;      // backward: [B,C,X,Y]
+    const float* dout;      // [B,C,X,Y]
     GeoParams g;            // grid and image (level sizes come from lv)
     int B, N, C;
     int cpl;                // channels per lane: a channel slice is 32 * cpl channels
     int cpad;               // channels per texel in the channels-last buffers (padded)
-    int texel_bytes;        // forward: bytes per texel of the channels-last features
-    int out_vec;            // out (forward) / dout (backward) is 16-byte aligned and Y % 4 == 0
+    int out_vec;            // dout is 16-byte aligned and Y % 4 == 0
     int tiles_i, tiles_j;   // tiles along X and Y
     LevelTable lv;          // feature levels
 };

@@ -1,5 +1,5 @@
-// bev_tile.cuh -- CTA machinery shared by the dense Sampling-VT forward and
-// backward kernels (sm_100a): block-level geometry and texel reuse.
+// bev_tile.cuh -- CTA machinery of the dense Sampling-VT feature gradient
+// (sm_100a): block-level geometry and shared scatters.
 //
 // FlashBEV's reading notes recompute the channel-independent geometry for
 // every channel ("Method" item 3), name that recompute as the cost that grows
@@ -16,23 +16,23 @@
 //            are grouped, up to kGmax at a time.  A vertical column of voxels
 //            projects to a near-vertical segment, so cells of one group share
 //            nearly all of their texels (the union box is ~94% filled on the
-//            seeded rigs): a texel's channel vector is then loaded once for
-//            the whole group and applied to every member cell from registers.
+//            seeded rigs): one reduction per texel then carries the whole
+//            group's sum sum_g w_g dout_g, where a per-cell scatter would send
+//            one per member.
 //   sweep    warps take groups in turn, largest first.  For its group a warp
 //            projects the members' voxels exactly (image-plane positions held
 //            in registers), bounds their texels, sums the bilinear weights
-//            w / cnt of the members' bins per
-//            (cell, texel) into a dense [texel][member] array of its own
-//            shared-memory region -- 32-bit integer atomics on an exact fixed
-//            point split in two words (2^-20 and 2^-40), so the order of the
-//            additions does not matter -- rounds them once to fp32, and walks
-//            the union box once (the forward gathers, the backward scatters).
+//            w / cnt of the members' bins per (cell, texel) into a dense
+//            [texel][member] array of its own shared-memory region -- 32-bit
+//            integer atomics on an exact fixed point split in two words
+//            (2^-20 and 2^-40), so the order of the additions does not
+//            matter -- rounds them once to fp32, and walks the union box once.
 //
 // A group whose merged weights would not fit the warp's region is taken
 // cell by cell; a cell whose box alone does not fit is swept bin by bin
-// ("direct").  With several feature levels, a group is swept level by
-// level on the same projections.  Every step is deterministic except the order of the
-// backward's global reductions.
+// ("direct").  With several feature levels, a group is swept level by level
+// on the same projections.  Every step is deterministic except the order of
+// the global reductions.
 #pragma once
 
 #include <limits.h>
@@ -353,15 +353,14 @@ __device__ __forceinline__ void level_position(float2 uv, float sW, float sH, fl
     fy = __fadd_rn(__fmul_rn(uv.y, sH), -0.5f);
 }
 
-// Count pass over the bins [z0, z0 + zc): 1 / cnt per item, the optional
-// uint8 count output, and per (active camera, cell) the leftmost level-0
+// Count pass over the bins [z0, z0 + zc): 1 / cnt per item, and per (active
+// camera, cell) the leftmost level-0
 // feature column the cell's valid voxels reach (from the position the
 // validity test used; it only steers the grouping).  Cameras are the outer
 // loop, so each camera's constants are read once per thread.
 constexpr int kMaxPasses = kCells * 16 / kThreads;  // item passes at 16 lanes per cell
 
-__device__ inline void count_pass(const SampleArgs& a, const TileSm& s, int b, int ti0, int tj0, int z0, int zc,
-                                  bool write_count) {
+__device__ inline void count_pass(const SampleArgs& a, const TileSm& s, int ti0, int tj0, int z0, int zc) {
     const GeoParams& g = a.g;
     const ItemMap im = item_map(zc);
     const int nA = s.ctl[kCtlNA];
@@ -404,11 +403,6 @@ __device__ inline void count_pass(const SampleArgs& a, const TileSm& s, int b, i
     for (int p = 0; p < kMaxPasses; ++p) {
         if (p >= im.passes) break;
         const int cell = p * im.cpp + (int)threadIdx.x / im.LZ;
-        if (in[p] && write_count) {
-            const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
-            const size_t at = (((size_t)b * g.X + i) * g.Y + j) * g.Z + z0 + zz;
-            if (checked(at < (size_t)a.B * g.X * g.Y * g.Z, kCheckStore)) a.count[at] = (uint8_t)cnt[p];
-        }
         if (cell < kCells && zz < zc) s.rc[cell * kZc + zz] = cnt[p] > 0 ? __frcp_rn((float)cnt[p]) : 0.0f;
     }
 }
@@ -696,58 +690,6 @@ __device__ __forceinline__ void clear_members(const Members& m, unsigned* wh) {
     const int lane = threadIdx.x & 31;
     for (int e = 4 * lane; e < m.entries; e += 128) *reinterpret_cast<uint4*>(wh + e) = make_uint4(0u, 0u, 0u, 0u);
     __syncwarp();
-}
-
-// ---------------------------------------------------------------------------
-// Per-lane channel vectors
-// ---------------------------------------------------------------------------
-
-// CPL channels of one texel for this lane, widened to fp32.  Raw words:
-// fp32 CPL channels, or bf16 pairs (the bf16 bits are the high half of the
-// fp32 word, so widening is exact).
-template <bool BF16, int CPL>
-struct LaneVec {
-    static constexpr int kWords = BF16 ? CPL / 2 : CPL;
-    unsigned w[kWords];
-
-    __device__ __forceinline__ void load(const unsigned char* p) {
-        if constexpr (kWords == 4) {
-            const uint4 d = __ldg(reinterpret_cast<const uint4*>(p));
-            w[0] = d.x; w[1] = d.y; w[2] = d.z; w[3] = d.w;
-        } else if constexpr (kWords == 2) {
-            const uint2 d = __ldg(reinterpret_cast<const uint2*>(p));
-            w[0] = d.x; w[1] = d.y;
-        } else {
-            w[0] = __ldg(reinterpret_cast<const unsigned*>(p));
-        }
-    }
-    __device__ __forceinline__ void zero() {
-#pragma unroll
-        for (int k = 0; k < kWords; ++k) w[k] = 0u;
-    }
-    __device__ __forceinline__ float get(int c) const {
-        if constexpr (BF16)
-            return (c & 1) ? __uint_as_float(w[c >> 1] & 0xffff0000u) : __uint_as_float(w[c >> 1] << 16);
-        else
-            return __uint_as_float(w[c]);
-    }
-};
-
-// acc += wt * v over the lane's CPL channels (packed fp32x2 FMA of sm_100,
-// each half an IEEE fma.rn).
-template <int CPL>
-__device__ __forceinline__ void fma_lane(float (&acc)[CPL], float wt, const float (&v)[CPL]) {
-    if constexpr (CPL == 1) {
-        acc[0] = __fmaf_rn(wt, v[0], acc[0]);
-    } else {
-#pragma unroll
-        for (int p = 0; p < CPL / 2; ++p) {
-            const float2 r = __ffma2_rn(make_float2(wt, wt), make_float2(v[2 * p], v[2 * p + 1]),
-                                        make_float2(acc[2 * p], acc[2 * p + 1]));
-            acc[2 * p] = r.x;
-            acc[2 * p + 1] = r.y;
-        }
-    }
 }
 
 // S weights of one texel of a group's array.
