@@ -122,6 +122,30 @@ def test_forward_channels_last_input(name):
     assert torch.equal(out_nhwc, out_nchw)   # same kernel, same order: bitwise equal
 
 
+def _tilted_rigs(w, seed):
+    Ks, Es = zip(*(I.random_rig(seed + b, w.N, w.img_h, w.img_w) for b in range(w.B)))
+    return torch.from_numpy(np.stack(Ks)), torch.from_numpy(np.stack(Es))
+
+
+@pytest.mark.parametrize("name", ["batched_bf16", "large"])
+def test_forward_full_size_tilted_rigs(name):
+    """The full-size workloads on rigs with random yaw, +-8 degree pitch and
+    roll and off-centre principal points: a cell's voxels then project to a
+    slanted segment, so merged patches are wider than two columns and the
+    unmerged path is taken more often."""
+    w = I.WORKLOADS[name]
+    K, E = _tilted_rigs(w, 300)
+    check_forward(I.make_features(w), K, E, w.img_h, w.img_w, w.ranges, w.res, TOL[w.dtype])
+
+
+def test_backward_full_size_tilted_rigs():
+    """The feature gradient at the batched_bf16 sizes (B4, C128, 200x200x16)
+    on the tilted rigs: groups of cells then share slanted boxes."""
+    w = I.WORKLOADS["batched_bf16"]
+    K, E = _tilted_rigs(w, 300)
+    check_backward(I.make_dout(w), K, E, w.img_h, w.img_w, w.ranges, w.res, w.N, w.Hf, w.Wf)
+
+
 def test_backward_workload_full_size():
     w = I.WORKLOADS["backward"]
     K, E = I.make_rigs(w)
