@@ -192,7 +192,7 @@ __device__ __forceinline__ void forward_body(const SampleArgs& a) {
     const int i = ti0 + warp;
     const float x = voxel_centre(g.xmin, i, g.dx);
     const bool write_count = a.count != nullptr && blockIdx.z == 0;
-    constexpr int ZN = z_per_lane_fwd<BF16, L>();
+    constexpr int ZN = z_per_lane_fwd<BF16, L, V>();
     const int zn = min(ZN, (g.Z + L - 1) / L);  // bins per lane per chunk
 
     float2 acc[CG][V][P];

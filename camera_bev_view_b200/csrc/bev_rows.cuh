@@ -48,10 +48,11 @@ static_assert(kCellsPerWarp == kTileJ && kWarps == kTileI, "one warp per tile ro
 // group), and taller grids take more chunks.  The forward's accumulators
 // already fill the register file: fp32 slices with eight or more lanes per
 // cell take one bin per lane (two spill), bf16 slices and four-lane cells
-// take two (one is slower there).  The backward, which holds dout instead,
-// takes four.
-template <bool BF16, int L>
-constexpr int z_per_lane_fwd() { return (!BF16 && L >= 8) ? 1 : 2; }
+// take two (one is slower there), except fp32 slices of four lanes with five
+// chunks each (80 channels), which run two CTAs per SM and measured 2%
+// faster with four.  The backward, which holds dout instead, takes four.
+template <bool BF16, int L, int V>
+constexpr int z_per_lane_fwd() { return (!BF16 && L >= 8) ? 1 : (!BF16 && L == 4 && V == 5) ? 4 : 2; }
 constexpr int kZPerLaneBwd = 4;
 constexpr int kZPerLaneMax = kZPerLaneBwd;
 // Merged-weight entries of one warp for one (camera, height chunk): the
@@ -83,7 +84,7 @@ template <bool BF16, int L, int V, bool MS>
 constexpr int fwd_ctas_per_sm() {
     constexpr int pairs = BF16 ? 4 : 2;                 // fp32 pairs per 16-byte chunk
     constexpr int rounds = kCellsPerWarp / (32 / L);    // cell rounds per warp
-    constexpr int zn = z_per_lane_fwd<BF16, L>();
+    constexpr int zn = z_per_lane_fwd<BF16, L, V>();
     constexpr int regs = rounds * V * pairs * 2 + 16 * V + 8 * zn;
     return (!MS && regs <= 56) ? 3 : 2;
 }
