@@ -162,6 +162,7 @@ __device__ __forceinline__ void sweep_backward(const SampleArgs& a, const TileSm
             const size_t rowf = (size_t)Wl * tf;
             float* gl = a.lv.grad[l] + ((size_t)b * a.N + cam) * Hl * rowf + c_base + lane * CPL;
             const Members m = members_box(it, gp.cell, gp.n, Hl, Wl, sW, sH);
+            if (m.h <= 0 || m.w <= 0) continue;  // no member has a valid voxel on this level
             if (!box_inside(m, Hl, Wl)) continue;
             if (m.entries <= kWarpEntries) {
                 backward_members<CPL>(s, m, it, zc, Hl, Wl, sW, sH, gl, rowf, tf, on, lane, wh, wl);
@@ -232,7 +233,10 @@ __global__ void __launch_bounds__(kThreads, kTileCtas) sample_backward_kernel(co
 
     for (int z0 = 0; z0 < g.Z; z0 += kZc) {
         const int zc = min(kZc, g.Z - z0);
-        count_pass(a, s, ti0, tj0, z0, zc);
+        if (nA == 1)
+            single_camera_pass(a, s, ti0, tj0, z0, zc);
+        else
+            count_pass(a, s, ti0, tj0, z0, zc);
         if (z0 == 0) {
 #pragma unroll
             for (int it = 0; it < kIt; ++it) {

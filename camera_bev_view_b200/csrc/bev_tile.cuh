@@ -407,6 +407,50 @@ __device__ inline void count_pass(const SampleArgs& a, const TileSm& s, int ti0,
     }
 }
 
+// Tiles that one camera alone can see (one active camera after the cull):
+// every valid voxel then has cnt = 1, so 1 / cnt is 1 and the geometry is
+// needed only to form the groups.  A cell joins the camera's groups unless
+// the five validity margins of corner_margins, taken at the two end voxels
+// of its column in the chunk (each margin is linear along the column, so its
+// maximum is at an end), rule out every voxel; its key is the leftmost
+// level-0 feature column the two end voxels reach (an approximation, which
+// only steers the grouping; the sweep projects every voxel exactly).  A
+// cell that joins with no valid voxel adds nothing.
+__device__ inline void single_camera_pass(const SampleArgs& a, const TileSm& s, int ti0, int tj0, int z0, int zc) {
+    const GeoParams& g = a.g;
+    for (int t = threadIdx.x; t < kCells * kZc; t += kThreads) s.rc[t] = 1.0f;
+    if (threadIdx.x < kCells) {
+        const int cell = threadIdx.x;
+        const int i = ti0 + cell / kTileJ, j = tj0 + cell % kTileJ;
+        unsigned short key = 0xffffu;
+        if (i < g.X && j < g.Y) {
+            const float* cam = s.cams + s.ctl[kCtlActive] * kCamFloats;
+            const float px = voxel_centre(g.xmin, i, g.dx), py = voxel_centre(g.ymin, j, g.dy);
+            const float sW0 = a.lv.sW[0];
+            const int W0 = a.lv.Wf[0];
+            float m[5] = {-1e30f, -1e30f, -1e30f, -1e30f, -1e30f};
+            int x0 = INT_MAX;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float pz = voxel_centre(g.zmin, e ? z0 + zc - 1 : z0, g.dz);
+                float me[5];
+                corner_margins(cam, px, py, pz, g.img_w, g.img_h, me);
+#pragma unroll
+                for (int q = 0; q < 5; ++q) m[q] = fmaxf(m[q], me[q]);
+                const float depth = cam_row(cam + 8, px, py, pz);
+                if (depth > 0.1f) {
+                    const float* k = cam + 12;
+                    const float uh = k[0] * cam_row(cam, px, py, pz) + k[1] * cam_row(cam + 4, px, py, pz) + k[2] * depth;
+                    x0 = min(x0, min(max((int)floorf(__fdividef(uh, depth) * sW0 - 0.5f), 0), W0 - 1));
+                }
+            }
+            if (m[0] >= 0.0f && m[1] >= 0.0f && m[2] >= 0.0f && m[3] >= 0.0f && m[4] >= 0.0f)
+                key = (unsigned short)(x0 == INT_MAX ? 0 : x0);
+        }
+        s.xlo[cell] = key;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Grouping (warp 0)
 // ---------------------------------------------------------------------------
