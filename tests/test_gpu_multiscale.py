@@ -71,6 +71,16 @@ def test_multiscale_workload_full_size(name):
     check(I.MS_WORKLOADS[name])
 
 
+@pytest.mark.parametrize("name", ["ms", "ms_bf16"])
+def test_multiscale_full_size_tilted_rigs(name):
+    """The full-size pyramids on rigs with random yaw, +-8 degree pitch and
+    roll and off-centre principal points: slanted projections on every
+    level, forward and every level's gradient."""
+    w = I.MS_WORKLOADS[name]
+    Ks, Es = zip(*(I.random_rig(400 + b, w.N, w.img_h, w.img_w) for b in range(w.B)))
+    check(w, K=torch.from_numpy(np.stack(Ks)), E=torch.from_numpy(np.stack(Es)))
+
+
 def test_one_level_is_bitwise_the_single_level_forward():
     w = I.WORKLOADS["nuscenes"]
     F = I.make_features(w)
